@@ -1,0 +1,333 @@
+// C ABI of the dropless top-k MoE layer: argument validation, workspace
+// carving and the fixed launch sequence of the forward and backward passes.
+// No entry point allocates, frees or synchronises (moe_get_device_status
+// excepted, since it must return a host value).
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+inline bool aligned16(const void* p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
+inline size_t elem_bytes(moe_dtype dt) { return dt == MOE_F32 ? 4 : 2; }
+inline size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Sizes shared by every entry point.
+moe_status check_shape(int N, int H, int E, int K, moe_dtype dt) {
+  if (dt != MOE_F32 && dt != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (N < 0 || H <= 0 || E <= 0 || K <= 0 || K > E) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)N * K > (int64_t)0x7fffffff - (int64_t)E * kTile) return MOE_ERR_UNSUPPORTED;
+  if (E > 256 || K > 32) return MOE_ERR_UNSUPPORTED;
+  if (dt == MOE_F32 && H % 4 != 0) return MOE_ERR_UNSUPPORTED;
+  if (dt == MOE_BF16 && H % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_ffn(int H, int F, moe_dtype dt) {
+  if (F <= 0) return MOE_ERR_INVALID_ARG;
+  if (dt == MOE_BF16 && !umma_shape_supported(H, F)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int64_t p_max(int N, int E, int K) { return round_up((int64_t)N * K + (int64_t)E * (kTile - 1), kTile); }
+
+// Layer workspace, in order; every region 256-byte aligned.
+struct LayerWs {
+  int* status;
+  void* route_scratch;
+  void* meta_scratch;
+  int32_t* pos;
+  void* x_perm;
+  void* act;
+  void* out;
+  void* gate_up;     // training only
+  void* d_out;       // training only (backward scratch from here on)
+  void* d_gate_up;
+  void* dx_perm;
+  float* dlogit;
+  void* ur_scratch;
+  size_t total;
+};
+
+size_t route_scratch_bytes(int H, int E, moe_dtype dt) {
+  return dt == MOE_BF16 ? route_umma_scratch(H, E) : 0;
+}
+
+LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int training) {
+  LayerWs w;
+  memset(&w, 0, sizeof(w));
+  char* p = (char*)base;
+  size_t off = 0;
+  const int64_t P = p_max(N, E, K), NK = (int64_t)N * K;
+  const size_t eb = elem_bytes(dt);
+  auto take = [&](size_t bytes) -> void* {
+    void* r = p ? (void*)(p + off) : nullptr;
+    off += al256(bytes);
+    return r;
+  };
+  w.status = (int*)take(kStatusBytes);
+  w.route_scratch = take(route_scratch_bytes(H, E, dt));
+  w.meta_scratch = take(meta_workspace_bytes(NK, E));
+  w.pos = (int32_t*)take(NK * 4);
+  w.x_perm = take(P * H * eb);
+  w.act = take(P * F * eb);
+  w.out = take(P * H * eb);
+  if (training) {
+    w.gate_up = take(2 * P * F * eb);
+    w.d_out = take(P * H * eb);
+    w.d_gate_up = take(2 * P * F * eb);
+    w.dx_perm = take(P * H * eb);
+    w.dlogit = (float*)take(NK * 4);
+    w.ur_scratch = take(unpermute_router_bwd_scratch(H, E, P));
+  }
+  w.total = off;
+  return w;
+}
+
+moe_status route_any(const void* x, const void* W_r, int N, int H, int E, int K, moe_dtype dt,
+                     float* logits, float* probs, int32_t* top, float* w, void* scratch, int* status,
+                     cudaStream_t s) {
+  if (N == 0) return MOE_OK;
+  if (dt == MOE_BF16 && route_umma_supported(N, H, E, K))
+    return route_umma(x, W_r, N, H, E, K, logits, probs, top, w, scratch, status, s);
+  if (route_simt_supported(H, E, K, (int)elem_bytes(dt)))
+    return route_simt(x, W_r, N, H, E, K, dt, logits, probs, top, w, s);
+  return MOE_ERR_UNSUPPORTED;
+}
+
+moe_status swiglu_any(const void* x_perm, const void* W1, const void* W3, const void* W2,
+                      const int32_t* pb, int E, int H, int F, int64_t P, moe_dtype dt, void* act,
+                      void* out, void* gate_up, int* status, cudaStream_t s) {
+  if (dt == MOE_F32)
+    return grouped_swiglu_simt(x_perm, W1, W3, W2, pb, E, H, F, P, dt, act, out, gate_up, s);
+  return grouped_swiglu_umma(x_perm, W1, W3, W2, pb, E, H, F, P, act, out, gate_up, status, s);
+}
+
+moe_status swiglu_bwd_any(const void* d_out, const void* x_perm, const void* act, const void* gate_up,
+                          const void* W1, const void* W3, const void* W2, const int32_t* pb, int E,
+                          int H, int F, int64_t P, moe_dtype dt, void* d_gate_up, void* dW1,
+                          void* dW3, void* dW2, void* dx_perm, int* status, cudaStream_t s) {
+  if (dt == MOE_F32)
+    return grouped_swiglu_bwd_simt(d_out, x_perm, act, gate_up, W1, W3, W2, pb, E, H, F, P, dt,
+                                   d_gate_up, dW1, dW3, dW2, dx_perm, s);
+  return grouped_swiglu_bwd_umma(d_out, x_perm, act, gate_up, W1, W3, W2, pb, E, H, F, P, d_gate_up,
+                                 dW1, dW3, dW2, dx_perm, status, s);
+}
+
+}  // namespace
+
+#define MOE_TRY(expr)                      \
+  do {                                     \
+    moe_status _st = (expr);               \
+    if (_st != MOE_OK) return _st;         \
+  } while (0)
+
+extern "C" {
+
+int32_t moe_tile_rows(void) { return kTile; }
+
+int64_t moe_padded_rows_max(int32_t N, int32_t E, int32_t K) {
+  if (N < 0 || E <= 0 || K <= 0) return 0;
+  return p_max(N, E, K);
+}
+
+size_t moe_route_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, moe_dtype dt) {
+  (void)N; (void)K;
+  return al256(kStatusBytes) + al256(route_scratch_bytes(H, E, dt));
+}
+
+size_t moe_dispatch_meta_workspace_size(int32_t N, int32_t K, int32_t E) {
+  return al256(kStatusBytes) + al256(meta_workspace_bytes((int64_t)N * K, E));
+}
+
+size_t moe_grouped_workspace_size(void) { return al256(kStatusBytes); }
+
+size_t moe_unpermute_router_bwd_workspace_size(int32_t H, int32_t E, int64_t P) {
+  return al256(kStatusBytes) + al256(unpermute_router_bwd_scratch(H, E, P));
+}
+
+size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
+                          int32_t training) {
+  if (check_shape(N, H, E, K, dt) != MOE_OK || F <= 0) return 0;
+  return carve(nullptr, N, H, E, K, F, dt, training).total;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ws || ws_bytes < (size_t)kStatusBytes) return MOE_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, (cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_get_device_status(const void* ws, int32_t* status_out, moe_stream_t stream) {
+  if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  *status_out = v;
+  return MOE_OK;
+}
+
+moe_status moe_route(const void* x, const void* W_r, int32_t N, int32_t H, int32_t E, int32_t K,
+                     moe_dtype dt, float* logits, float* probs, int32_t* top_experts, float* weights,
+                     void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(N, H, E, K, dt));
+  if (N > 0 && (!x || !W_r || !top_experts || !weights)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_route_workspace_size(N, H, E, K, dt)) return MOE_ERR_WORKSPACE;
+  char* base = (char*)ws;
+  return route_any(x, W_r, N, H, E, K, dt, logits, probs, top_experts, weights,
+                   base + al256(kStatusBytes), (int*)ws, (cudaStream_t)stream);
+}
+
+moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, int32_t E,
+                             int32_t* indices, int32_t* bin_ids, int32_t* bins, int32_t* padded_bins,
+                             int32_t* pos, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (N < 0 || K <= 0 || E <= 0 || K > E) return MOE_ERR_INVALID_ARG;
+  if (E > 256) return MOE_ERR_UNSUPPORTED;
+  if (!padded_bins || (N > 0 && (!top_experts || !pos))) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_dispatch_meta_workspace_size(N, K, E)) return MOE_ERR_WORKSPACE;
+  char* base = (char*)ws;
+  return dispatch_meta(top_experts, (int64_t)N * K, E, indices, bin_ids, bins, padded_bins, pos,
+                       base + al256(kStatusBytes), (int*)ws, (cudaStream_t)stream);
+}
+
+moe_status moe_permute(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* padded_bins,
+                       int32_t N, int32_t H, int32_t E, int32_t K, moe_dtype dt, void* x_perm,
+                       moe_stream_t stream) {
+  MOE_TRY(check_shape(N, H, E, K, dt));
+  if (!bins || !padded_bins || !x_perm || (N > 0 && (!x || !pos))) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  return permute_rows(x, pos, bins, padded_bins, N, H, E, K, dt, x_perm, (cudaStream_t)stream);
+}
+
+moe_status moe_grouped_swiglu(const void* x_perm, const void* W1, const void* W3, const void* W2,
+                              const int32_t* padded_bins, int32_t E, int32_t H, int32_t F, int64_t P,
+                              moe_dtype dt, void* act, void* out, void* gate_up, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(0, H, E, 1, dt));
+  MOE_TRY(check_ffn(H, F, dt));
+  if (P < 0 || P % kTile != 0) return MOE_ERR_INVALID_ARG;
+  if (!x_perm || !W1 || !W3 || !W2 || !padded_bins || !act || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(act) ||
+      !aligned16(out) || !aligned16(gate_up))
+    return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_grouped_workspace_size()) return MOE_ERR_WORKSPACE;
+  if (P == 0) return MOE_OK;
+  return swiglu_any(x_perm, W1, W3, W2, padded_bins, E, H, F, P, dt, act, out, gate_up, (int*)ws,
+                    (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const void* out, const float* weights, const int32_t* pos, int32_t N, int32_t K,
+                       int32_t H, moe_dtype dt, void* y, moe_stream_t stream) {
+  MOE_TRY(check_shape(N, H, K, K, dt));
+  if (N == 0) return MOE_OK;
+  if (!out || !weights || !pos || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  return combine_rows(out, weights, pos, N, K, H, dt, y, (cudaStream_t)stream);
+}
+
+moe_status moe_combine_bwd(const void* dy, const void* out, const float* weights, const int32_t* pos,
+                           const int32_t* bins, const int32_t* padded_bins, int32_t N, int32_t K,
+                           int32_t H, int32_t E, moe_dtype dt, float* dw, float* dlogit, void* d_out,
+                           moe_stream_t stream) {
+  MOE_TRY(check_shape(N, H, E, K, dt));
+  if (!bins || !padded_bins || !d_out || (N > 0 && (!dy || !out || !weights || !pos || !dlogit)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(out) || !aligned16(d_out)) return MOE_ERR_INVALID_ARG;
+  return combine_bwd_rows(dy, out, weights, pos, bins, padded_bins, N, K, H, E, dt, dw, dlogit, d_out,
+                          (cudaStream_t)stream);
+}
+
+moe_status moe_grouped_swiglu_bwd(const void* d_out, const void* x_perm, const void* act,
+                                  const void* gate_up, const void* W1, const void* W3, const void* W2,
+                                  const int32_t* padded_bins, int32_t E, int32_t H, int32_t F, int64_t P,
+                                  moe_dtype dt, void* d_gate_up, void* dW1, void* dW3, void* dW2,
+                                  void* dx_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(0, H, E, 1, dt));
+  MOE_TRY(check_ffn(H, F, dt));
+  if (P < 0 || P % kTile != 0) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {d_out, x_perm, act, gate_up, W1, W3, W2, d_gate_up, dW1, dW3, dW2, dx_perm};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (!padded_bins) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_grouped_workspace_size()) return MOE_ERR_WORKSPACE;
+  return swiglu_bwd_any(d_out, x_perm, act, gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
+                        d_gate_up, dW1, dW3, dW2, dx_perm, (int*)ws, (cudaStream_t)stream);
+}
+
+moe_status moe_unpermute_router_bwd(const void* dx_perm, const float* dlogit, const void* x,
+                                    const void* W_r, const int32_t* top_experts, const int32_t* pos,
+                                    const int32_t* indices, const int32_t* bins,
+                                    const int32_t* padded_bins, int32_t N, int32_t H, int32_t E,
+                                    int32_t K, int64_t P, moe_dtype dt, void* dx, void* dW_r, void* ws,
+                                    size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(N, H, E, K, dt));
+  if (P < 0 || P % kTile != 0) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins, dx, dW_r};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_unpermute_router_bwd_workspace_size(H, E, P))
+    return MOE_ERR_WORKSPACE;
+  return unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins, N,
+                              H, E, K, P, dt, dx, dW_r, (char*)ws + al256(kStatusBytes),
+                              (cudaStream_t)stream);
+}
+
+moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const void* W3, const void* W2,
+                         int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
+                         int32_t training, void* y, int32_t* top_experts, float* weights,
+                         int32_t* indices, int32_t* bins, int32_t* padded_bins, void* ws,
+                         size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_shape(N, H, E, K, dt));
+  MOE_TRY(check_ffn(H, F, dt));
+  const void* ptrs[] = {x, W_r, W1, W3, W2, y, top_experts, weights, indices, bins, padded_bins};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_workspace_size(N, H, E, K, F, dt, training);
+  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  LayerWs w = carve(ws, N, H, E, K, F, dt, training);
+  const int64_t P = p_max(N, E, K);
+  MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, nullptr, top_experts, weights, w.route_scratch,
+                    w.status, s));
+  MOE_TRY(dispatch_meta(top_experts, (int64_t)N * K, E, indices, nullptr, bins, padded_bins, w.pos,
+                        w.meta_scratch, w.status, s));
+  if (N == 0) return MOE_OK;
+  MOE_TRY(permute_rows(x, w.pos, bins, padded_bins, N, H, E, K, dt, w.x_perm, s));
+  MOE_TRY(swiglu_any(w.x_perm, W1, W3, W2, padded_bins, E, H, F, P, dt, w.act, w.out,
+                     training ? w.gate_up : nullptr, w.status, s));
+  MOE_TRY(combine_rows(w.out, weights, w.pos, N, K, H, dt, y, s));
+  return MOE_OK;
+}
+
+moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const void* W1, const void* W3,
+                         const void* W2, const int32_t* top_experts, const float* weights,
+                         const int32_t* indices, const int32_t* bins, const int32_t* padded_bins,
+                         int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt, void* dx,
+                         void* dW_r, void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+  MOE_TRY(check_shape(N, H, E, K, dt));
+  MOE_TRY(check_ffn(H, F, dt));
+  const void* ptrs[] = {dy, x, W_r, W1, W3, W2, top_experts, weights, indices, bins, padded_bins,
+                        dx, dW_r, dW1, dW3, dW2};
+  for (const void* q : ptrs)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_workspace_size(N, H, E, K, F, dt, 1);
+  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  LayerWs w = carve(ws, N, H, E, K, F, dt, 1);
+  const int64_t P = p_max(N, E, K);
+  MOE_TRY(combine_bwd_rows(dy, w.out, weights, w.pos, bins, padded_bins, N, K, H, E, dt, nullptr,
+                           w.dlogit, w.d_out, s));
+  MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, w.gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
+                         w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s));
+  MOE_TRY(unpermute_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, indices, bins,
+                               padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, s));
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,730 @@
+// Persistent tcgen05 / TMEM grouped GEMM for bf16 expert FFNs (sm_100a).
+//
+// The expert FFN of the dropless layer is a set of per-expert GEMMs over
+// variable-size row groups ("MegaBlocks - architecture", sec. 2.1, grouped
+// path gmm -> act -> gmm; sec. 4: backward through the same grouping).  Every
+// expert's rows are padded to multiples of 128, so each 128-row M tile lies in
+// one expert; the tile -> expert map is a search in the device-side
+// padded_bins, so the schedule never needs the counts on the host (the
+// MegaBlocks grouped path copies them to the host; MoonEP sec. 02 argues for
+// static shapes without host sync).
+//
+// One CTA per SM, 6 warps:
+//   warp 0      TMA producer: A and B tiles into a STAGES-deep smem ring
+//   warp 1      TMEM allocator and MMA issuer (one thread): 128 x BN x 16
+//               tcgen05.mma per k-step, fp32 accumulators in TMEM, two
+//               accumulator buffers so the epilogue of tile i overlaps the
+//               main loop of tile i+1
+//   warps 2..5  epilogue: tcgen05.ld rows -> registers -> fused math -> global
+// Schedules
+//   ROWS   C[rows of group e, :] = A[rows, :] * B_e   (forward, dgrad)
+//   WGRAD  C_e = A[group e rows, :]^T * B[group e rows, :]   (weight grads;
+//          K = the group's padded rows, zero rows contribute nothing)
+//   DENSE  C = A * B over plain row tiles (router logits)
+// Every accumulation runs in a fixed order (k-steps in sequence, no split-K),
+// so results are bitwise reproducible.  Every wait is bounded (status bit
+// MOE_DEVERR_TIMEOUT); no TMA multicast is used.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "umma.cuh"
+
+namespace moe {
+namespace umma {
+
+constexpr int BM = 128;
+constexpr int BK = 64;              // one 128-byte swizzle row of bf16
+constexpr int kThreads = 192;
+constexpr int kA_BYTES = BM * BK * 2;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+constexpr int kGroupM = 8;          // M tiles per raster group (L2 reuse of B panels)
+
+enum Sched { SCHED_ROWS = 0, SCHED_WGRAD = 1, SCHED_DENSE = 2 };
+enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3, EPI_WGRAD_PAIR = 4,
+           EPI_ROUTER = 5 };
+enum Split { SPLIT_NONE = 0, SPLIT_K = 1, SPLIT_N = 2 };
+
+struct Params {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  const int32_t* padded_bins;
+  int E;
+  int64_t P;          // rows of row-indexed buffers (ROWS/WGRAD) or tokens (DENSE)
+  int kdim;           // ROWS/DENSE: K extent (both halves for SPLIT_K)
+  int ksplit;         // SPLIT_K: first k of the second operand pair
+  int n_mma;          // MMA N (== BN except DENSE, where it is E)
+  int n_tiles;        // tiles along N
+  int m_tiles_w;      // WGRAD: tiles along M
+  __nv_bfloat16* out0;
+  __nv_bfloat16* out1;
+  __nv_bfloat16* out2;
+  const __nv_bfloat16* aux0;
+  const __nv_bfloat16* aux1;
+  int64_t ldo;        // row stride (elements) of out* / aux*
+  int64_t out_estride;// WGRAD: elements between consecutive experts' outputs
+  float* logits;      // DENSE router outputs
+  float* probs;
+  int32_t* top;
+  float* weights;
+  int K;
+  int* status;
+};
+
+struct Tile {
+  int e;
+  int64_t row0;    // ROWS/DENSE: first A row; WGRAD: first contraction row
+  int m0;          // WGRAD: first output row (of the weight gradient)
+  int n0;          // first output column (per output matrix)
+  int nkb;         // k-blocks of BK
+};
+
+template <int SCHED, int BN, int EPI>
+__device__ __forceinline__ int64_t total_tiles(const Params& p) {
+  if constexpr (SCHED == SCHED_ROWS) {
+    int64_t rows = p.padded_bins[p.E - 1];
+    if (rows > p.P) rows = p.P;
+    return (rows / BM) * p.n_tiles;
+  } else if constexpr (SCHED == SCHED_WGRAD) {
+    return (int64_t)p.E * p.m_tiles_w * p.n_tiles;
+  } else {
+    return cdiv(p.P, BM);
+  }
+}
+
+template <int SCHED, int BN, int EPI>
+__device__ __forceinline__ Tile get_tile(const Params& p, int64_t t) {
+  constexpr int NOUT = (EPI == EPI_SWIGLU || EPI == EPI_WGRAD_PAIR) ? BN / 2 : BN;
+  Tile tl;
+  if constexpr (SCHED == SCHED_ROWS) {
+    int64_t rows = p.padded_bins[p.E - 1];
+    if (rows > p.P) rows = p.P;
+    const int64_t num_m = rows / BM;
+    const int64_t per_group = (int64_t)kGroupM * p.n_tiles;
+    const int64_t g = t / per_group;
+    const int64_t first_m = g * kGroupM;
+    const int64_t gm = (num_m - first_m) < kGroupM ? (num_m - first_m) : kGroupM;
+    const int64_t local = t - g * per_group;
+    const int64_t mt = first_m + local % gm;
+    const int64_t nt = local / gm;
+    tl.row0 = mt * BM;
+    tl.e = expert_of_row(p.padded_bins, p.E, tl.row0);
+    tl.m0 = 0;
+    tl.n0 = (int)(nt * NOUT);
+    tl.nkb = p.kdim / BK;
+  } else if constexpr (SCHED == SCHED_WGRAD) {
+    const int64_t per_e = (int64_t)p.m_tiles_w * p.n_tiles;
+    tl.e = (int)(t / per_e);
+    const int64_t r = t - (int64_t)tl.e * per_e;
+    tl.m0 = (int)((r / p.n_tiles) * BM);
+    tl.n0 = (int)((r % p.n_tiles) * NOUT);
+    const int64_t lo = tl.e ? p.padded_bins[tl.e - 1] : 0;
+    int64_t hi = p.padded_bins[tl.e];
+    if (hi > p.P) hi = p.P;
+    tl.row0 = lo;
+    tl.nkb = hi > lo ? (int)((hi - lo) / BK) : 0;
+  } else {
+    tl.e = 0;
+    tl.row0 = t * BM;
+    tl.m0 = 0;
+    tl.n0 = 0;
+    tl.nkb = p.kdim / BK;
+  }
+  return tl;
+}
+
+__device__ __forceinline__ void store_row_bf16x32(__nv_bfloat16* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+__device__ __forceinline__ void load_row_bf16x32(const __nv_bfloat16* src, float* v) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 w = s[q];
+    v[8 * q + 0] = bf16_lo(w.x); v[8 * q + 1] = bf16_hi(w.x);
+    v[8 * q + 2] = bf16_lo(w.y); v[8 * q + 3] = bf16_hi(w.y);
+    v[8 * q + 4] = bf16_lo(w.z); v[8 * q + 5] = bf16_hi(w.z);
+    v[8 * q + 6] = bf16_lo(w.w); v[8 * q + 7] = bf16_hi(w.w);
+  }
+}
+
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals)[KMAX], int (&ids)[KMAX]) {
+  // Descending list; strict '>' keeps an earlier (lower-id) equal value above.
+#pragma unroll
+  for (int j = KMAX - 1; j >= 0; --j) {
+    if (j < K && v > vals[j]) {
+      if (j > 0 && v > vals[j - 1]) {
+        vals[j] = vals[j - 1];
+        ids[j] = ids[j - 1];
+      } else {
+        vals[j] = v;
+        ids[j] = id;
+      }
+    }
+  }
+}
+
+template <int BN, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
+__global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
+  constexpr int B_BYTES = BN * BK * 2;
+  constexpr int STAGE_BYTES = kA_BYTES + B_BYTES;
+  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  constexpr uint32_t TMEM_COLS = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
+  static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte swizzle atoms aligned");
+  static_assert(STAGES >= 2, "pipeline needs at least two stages");
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw_base);
+  const uint32_t bar_base = base + STAGES * STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.ta0);
+    tma_prefetch_desc(&p.tb0);
+    if (SPLIT != SPLIT_NONE) tma_prefetch_desc(&p.tb1);
+    if (SPLIT == SPLIT_K) tma_prefetch_desc(&p.ta1);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int64_t ntiles = total_tiles<SCHED, BN, EPI>(p);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t tx = kA_BYTES + (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)B_BYTES);
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile tl = get_tile<SCHED, BN, EPI>(p, t);
+        for (int kb = 0; kb < tl.nkb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
+          const uint32_t sa = base + stage * STAGE_BYTES;
+          const uint32_t sb = sa + kA_BYTES;
+          const uint32_t fb = full_bar(stage);
+          mbar_expect_tx(fb, tx);
+          if constexpr (SCHED == SCHED_WGRAD) {
+            const int krow = (int)(tl.row0 + (int64_t)kb * BK);
+            // A = X^T tile: two 64-wide MN boxes of the [rows, M] matrix
+            tma_load_2d(sa, &p.ta0, fb, tl.m0, krow);
+            tma_load_2d(sa + 8192, &p.ta0, fb, tl.m0 + 64, krow);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) {
+              if (SPLIT == SPLIT_N && j >= BN / 128)
+                tma_load_2d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), krow);
+              else
+                tma_load_2d(sb + j * 8192, &p.tb0, fb, tl.n0 + 64 * j, krow);
+            }
+          } else {
+            int k = kb * BK;
+            const CUtensorMap* ta = &p.ta0;
+            const CUtensorMap* tb = &p.tb0;
+            if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
+            tma_load_2d(sa, ta, fb, k, (int)tl.row0);
+            if constexpr (SCHED == SCHED_DENSE) {
+              tma_load_2d(sb, tb, fb, k, 0);
+            } else if constexpr (B_MN) {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j) {
+                if (SPLIT == SPLIT_N && j >= BN / 128)
+                  tma_load_3d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), k, tl.e);
+                else
+                  tma_load_3d(sb + j * 8192, tb, fb, tl.n0 + 64 * j, k, tl.e);
+              }
+            } else {
+              tma_load_3d(sb, tb, fb, k, tl.n0, tl.e);
+            }
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // give the loads already issued a bounded chance to land
+        for (int s = 0; s < STAGES; ++s) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(full_bar(s), 0) && !mbar_try_wait(full_bar(s), 1) &&
+                 globaltimer() - t0 < 50000000ull) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const int n_mma = (SCHED == SCHED_DENSE) ? p.n_mma : BN;
+      const uint32_t idesc = idesc_bf16(BM, n_mma, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile tl = get_tile<SCHED, BN, EPI>(p, t);
+        if (tl.nkb == 0) continue;
+        if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < tl.nkb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + stage * STAGE_BYTES;
+          const uint32_t sb = sa + kA_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? desc_mn_sw128(sa + kk * 2048, 8192) : desc_k_sw128(sa + kk * 32);
+            const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
+            mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(empty_bar(stage));      // smem slot free once these MMAs are done
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar(acc));          // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) {
+        mma_commit(drain_bar);
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(drain_bar, 0) && globaltimer() - t0 < 50000000ull) {}
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                       // TMEM lane quarter of this warp
+    const int row = q * 32 + lane;                // row inside the 128-row tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const Tile tl = get_tile<SCHED, BN, EPI>(p, t);
+      if constexpr (SCHED == SCHED_WGRAD) {
+        if (tl.nkb == 0) {                        // expert with no rows: zero gradient
+          const float z[32] = {0.f};
+          if constexpr (EPI == EPI_WGRAD_PAIR) {
+            __nv_bfloat16* d0 = p.out0 + (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
+            __nv_bfloat16* d1 = p.out1 + (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
+#pragma unroll
+            for (int c = 0; c < BN / 2; c += 32) { store_row_bf16x32(d0 + c, z); store_row_bf16x32(d1 + c, z); }
+          } else {
+            __nv_bfloat16* d0 = p.out0 + (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
+#pragma unroll
+            for (int c = 0; c < BN; c += 32) store_row_bf16x32(d0 + c, z);
+          }
+          continue;
+        }
+      }
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag, p.status, kTimeoutNs) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int64_t grow = tl.row0 + row;         // ROWS/DENSE global row
+
+      if constexpr (EPI == EPI_SWIGLU) {
+        __nv_bfloat16* act = p.out0 + grow * p.ldo + tl.n0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32(tacc + c, g);
+          tmem_ld_32(tacc + BN / 2 + c, u);
+          tmem_ld_wait();
+          float a[32], gf[32], uf[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            gf[j] = __uint_as_float(g[j]);
+            uf[j] = __uint_as_float(u[j]);
+            a[j] = silu_f(gf[j]) * uf[j];
+          }
+          store_row_bf16x32(act + c, a);
+          if (p.out1) {
+            store_row_bf16x32(p.out1 + grow * p.ldo + tl.n0 + c, gf);
+            store_row_bf16x32(p.out2 + grow * p.ldo + tl.n0 + c, uf);
+          }
+        }
+      } else if constexpr (EPI == EPI_STORE) {
+        __nv_bfloat16* dst = p.out0 + grow * p.ldo + tl.n0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32(tacc + c, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          store_row_bf16x32(dst + c, v);
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        const int64_t off = grow * p.ldo + tl.n0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32(tacc + c, r);
+          float gf[32], uf[32], dg[32], du[32];
+          load_row_bf16x32(p.aux0 + off + c, gf);
+          load_row_bf16x32(p.aux1 + off + c, uf);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float da = __uint_as_float(r[j]);
+            const float sig = 1.f / (1.f + expf(-gf[j]));
+            dg[j] = da * uf[j] * sig * (1.f + gf[j] * (1.f - sig));
+            du[j] = da * gf[j] * sig;
+          }
+          store_row_bf16x32(p.out0 + off + c, dg);
+          store_row_bf16x32(p.out1 + off + c, du);
+        }
+      } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) {
+        const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32(tacc + c, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (EPI == EPI_WGRAD_PAIR && c >= BN / 2)
+            store_row_bf16x32(p.out1 + off + (c - BN / 2), v);
+          else
+            store_row_bf16x32(p.out0 + off + c, v);
+        }
+      } else {  // EPI_ROUTER: softmax, top-K, renormalise on this row's E logits
+        constexpr int KMAX = 16;
+        const int E = p.n_mma, K = p.K;
+        const bool live = grow < p.P;
+        float vals[KMAX];
+        int ids[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
+        float m = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < E; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32(tacc + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (c + j < E) {
+              const float v = __uint_as_float(r[j]);
+              m = fmaxf(m, v);
+              topk_insert<KMAX>(v, c + j, K, vals, ids);
+              if (live && p.logits) p.logits[grow * E + c + j] = v;
+            }
+          }
+        }
+        if (p.probs) {
+          float Z = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < E; c += 32) {
+            uint32_t r[32];
+            tmem_ld_32(tacc + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < E) Z += expf(__uint_as_float(r[j]) - m);
+          }
+#pragma unroll 1
+          for (int c = 0; c < E; c += 32) {
+            uint32_t r[32];
+            tmem_ld_32(tacc + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (live && c + j < E) p.probs[grow * E + c + j] = expf(__uint_as_float(r[j]) - m) / Z;
+          }
+        }
+        if (live) {
+          float S = 0.f, ev[KMAX];
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) {
+            ev[j] = (j < K) ? expf(vals[j] - vals[0]) : 0.f;
+            S += ev[j];
+          }
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) {
+            if (j < K) {
+              p.top[grow * K + j] = ids[j];
+              p.weights[grow * K + j] = ev[j] / S;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [outer, inner] matrix, 128-byte swizzle.
+static bool map2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_elems,
+                  uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 map over [d2, d1, d0] (d0 contiguous), 128-byte swizzle, box depth 1.
+static bool map3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint32_t box0, uint32_t box1) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+template <int BN, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
+static moe_status launch(const Params& p, int64_t tiles_upper, cudaStream_t s) {
+  constexpr int STAGE_BYTES = kA_BYTES + BN * BK * 2;
+  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  const size_t smem = (size_t)STAGES * STAGE_BYTES + 1024 + 8 * (2 * STAGES + 5) + 16;
+  auto kern = umma_gemm_kernel<BN, SCHED, EPI, A_MN, B_MN, SPLIT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  int64_t grid = tiles_upper < sm_count() ? tiles_upper : sm_count();
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, kThreads, smem, s>>>(p);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+static Params blank_params(const int32_t* pb, int E, int64_t P, int* status) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.padded_bins = pb;
+  p.E = E;
+  p.P = P;
+  p.status = status;
+  return p;
+}
+
+}  // namespace umma
+
+using namespace umma;
+
+bool umma_shape_supported(int H, int F) { return H % 128 == 0 && F % 128 == 0 && H >= 128 && F >= 128; }
+
+moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W3, const void* W2,
+                               const int32_t* pb, int E, int H, int F, int64_t P, void* act, void* out,
+                               void* gate_up, int* status, cudaStream_t s) {
+  typedef __nv_bfloat16 bf;
+  // GEMM1 + SwiGLU: [G | U] = x_perm * [W1_e | W3_e], act = silu(G) * U
+  {
+    Params p = blank_params(pb, E, P, status);
+    if (!map2d(&p.ta0, x_perm, H, P, H, 64, 128) || !map3d(&p.tb0, W1, F, H, E, 64, 64) ||
+        !map3d(&p.tb1, W3, F, H, E, 64, 64))
+      return MOE_ERR_CUDA;
+    p.kdim = H;
+    p.n_mma = 256;
+    p.n_tiles = F / 128;
+    p.out0 = (bf*)act;
+    p.out1 = gate_up ? (bf*)gate_up : nullptr;
+    p.out2 = gate_up ? (bf*)gate_up + (size_t)P * F : nullptr;
+    p.ldo = F;
+    moe_status st = launch<256, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>(p, (P / BM) * p.n_tiles, s);
+    if (st != MOE_OK) return st;
+  }
+  // GEMM2: out = act * W2_e
+  {
+    Params p = blank_params(pb, E, P, status);
+    const int bn = (H % 256 == 0) ? 256 : 128;
+    if (!map2d(&p.ta0, act, F, P, F, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, 64)) return MOE_ERR_CUDA;
+    p.kdim = F;
+    p.n_mma = bn;
+    p.n_tiles = H / bn;
+    p.out0 = (bf*)out;
+    p.ldo = H;
+    if (bn == 256) return launch<256, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s);
+    return launch<128, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s);
+  }
+}
+
+moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const void* act,
+                                   const void* gate_up, const void* W1, const void* W3, const void* W2,
+                                   const int32_t* pb, int E, int H, int F, int64_t P, void* d_gate_up,
+                                   void* dW1, void* dW3, void* dW2, void* dx_perm, int* status,
+                                   cudaStream_t s) {
+  typedef __nv_bfloat16 bf;
+  const bf* G = (const bf*)gate_up;
+  const bf* U = G + (size_t)P * F;
+  bf* dG = (bf*)d_gate_up;
+  bf* dU = dG + (size_t)P * F;
+  moe_status st;
+  // dA = d_out * W2_e^T with the SwiGLU backward in the epilogue
+  {
+    Params p = blank_params(pb, E, P, status);
+    const int bn = (F % 256 == 0) ? 256 : 128;
+    if (!map2d(&p.ta0, d_out, H, P, H, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, bn)) return MOE_ERR_CUDA;
+    p.kdim = H;
+    p.n_mma = bn;
+    p.n_tiles = F / bn;
+    p.aux0 = G;
+    p.aux1 = U;
+    p.out0 = dG;
+    p.out1 = dU;
+    p.ldo = F;
+    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s)
+                   : launch<128, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s);
+    if (st != MOE_OK) return st;
+  }
+  // dW2_e = act_e^T * d_out_e   [F, H]
+  {
+    Params p = blank_params(pb, E, P, status);
+    const int bn = (H % 256 == 0) ? 256 : 128;
+    if (!map2d(&p.ta0, act, F, P, F, 64, 64) || !map2d(&p.tb0, d_out, H, P, H, 64, 64)) return MOE_ERR_CUDA;
+    p.n_mma = bn;
+    p.m_tiles_w = F / BM;
+    p.n_tiles = H / bn;
+    p.out0 = (bf*)dW2;
+    p.ldo = H;
+    p.out_estride = (int64_t)F * H;
+    const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
+    st = bn == 256 ? launch<256, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>(p, tiles, s)
+                   : launch<128, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>(p, tiles, s);
+    if (st != MOE_OK) return st;
+  }
+  // dW1_e | dW3_e = x_perm_e^T * [dG_e | dU_e]   [H, F] each
+  {
+    Params p = blank_params(pb, E, P, status);
+    if (!map2d(&p.ta0, x_perm, H, P, H, 64, 64) || !map2d(&p.tb0, dG, F, P, F, 64, 64) ||
+        !map2d(&p.tb1, dU, F, P, F, 64, 64))
+      return MOE_ERR_CUDA;
+    p.n_mma = 256;
+    p.m_tiles_w = H / BM;
+    p.n_tiles = F / 128;
+    p.out0 = (bf*)dW1;
+    p.out1 = (bf*)dW3;
+    p.ldo = F;
+    p.out_estride = (int64_t)H * F;
+    const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
+    st = launch<256, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>(p, tiles, s);
+    if (st != MOE_OK) return st;
+  }
+  // dx_perm = dG * W1_e^T + dU * W3_e^T  (one K = 2F contraction)
+  {
+    Params p = blank_params(pb, E, P, status);
+    const int bn = (H % 256 == 0) ? 256 : 128;
+    if (!map2d(&p.ta0, dG, F, P, F, 64, 128) || !map2d(&p.ta1, dU, F, P, F, 64, 128) ||
+        !map3d(&p.tb0, W1, F, H, E, 64, bn) || !map3d(&p.tb1, W3, F, H, E, 64, bn))
+      return MOE_ERR_CUDA;
+    p.kdim = 2 * F;
+    p.ksplit = F;
+    p.n_mma = bn;
+    p.n_tiles = H / bn;
+    p.out0 = (bf*)dx_perm;
+    p.ldo = H;
+    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>(p, (P / BM) * p.n_tiles, s)
+                   : launch<128, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>(p, (P / BM) * p.n_tiles, s);
+    if (st != MOE_OK) return st;
+  }
+  return MOE_OK;
+}
+
+// ---- router on tensor cores -----------------------------------------------
+
+bool route_umma_supported(int N, int H, int E, int K) {
+  (void)N;
+  return E >= 16 && E <= 256 && E % 16 == 0 && K <= 16 && H % 64 == 0;
+}
+
+size_t route_umma_scratch(int H, int E) { return (size_t)E * H * 2; }
+
+moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K, float* logits,
+                      float* probs, int32_t* top, float* w, void* scratch, int* status, cudaStream_t s) {
+  // B operand K-major: W_r^T [E, H] kept in the workspace
+  moe_status st = transpose_matrix(W_r, H, E, MOE_BF16, scratch, s);
+  if (st != MOE_OK) return st;
+  Params p = blank_params(nullptr, 1, N, status);
+  if (!map2d(&p.ta0, x, H, N, H, 64, 128) || !map2d(&p.tb0, scratch, H, E, H, 64, E)) return MOE_ERR_CUDA;
+  p.kdim = H;
+  p.n_mma = E;
+  p.K = K;
+  p.logits = logits;
+  p.probs = probs;
+  p.top = top;
+  p.weights = w;
+  return launch<256, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>(p, cdiv(N, BM), s);
+}
+
+}  // namespace moe

@@ -1,0 +1,237 @@
+"""Torch-facing wrappers over the C ABI, one per entry point, same names.
+
+Each wrapper checks devices and dtypes, allocates the output tensors with
+torch (device memory is torch's job here) and passes raw pointers plus the
+current CUDA stream to libmoe_b200.so.  No arithmetic of the layer happens
+in Python.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import MOE_BF16, MOE_F32, call, load
+
+_DT = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    return _DT[t.dtype]
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def tile_rows() -> int:
+    return load().moe_tile_rows()
+
+
+def padded_rows_max(N: int, E: int, K: int) -> int:
+    return load().moe_padded_rows_max(N, E, K)
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """Caller-owned device workspace with its status word zeroed."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    call("moe_workspace_init", ws.data_ptr(), ws.numel(), _stream())
+    return ws
+
+
+def device_status(ws: torch.Tensor) -> int:
+    import ctypes
+    v = ctypes.c_int32(0)
+    call("moe_get_device_status", ws.data_ptr(), ctypes.addressof(v), _stream())
+    return v.value
+
+
+def moe_route(x, W_r, K: int, want_logits: bool = False, want_probs: bool = False, ws=None) -> dict:
+    N, H = x.shape
+    E = W_r.shape[1]
+    dev = x.device
+    dt = _dt(x)
+    if ws is None:
+        ws = workspace(load().moe_route_workspace_size(N, H, E, K, dt), dev)
+    out = {
+        "top_experts": torch.empty(N, K, dtype=torch.int32, device=dev),
+        "weights": torch.empty(N, K, dtype=torch.float32, device=dev),
+        "logits": torch.empty(N, E, dtype=torch.float32, device=dev) if want_logits else None,
+        "probs": torch.empty(N, E, dtype=torch.float32, device=dev) if want_probs else None,
+        "ws": ws,
+    }
+    call("moe_route", _p(x), _p(W_r), N, H, E, K, dt, _p(out["logits"]), _p(out["probs"]),
+         _p(out["top_experts"]), _p(out["weights"]), ws.data_ptr(), ws.numel(), _stream())
+    return out
+
+
+def moe_dispatch_meta(top_experts, E: int, ws=None) -> dict:
+    N, K = top_experts.shape
+    dev = top_experts.device
+    if ws is None:
+        ws = workspace(load().moe_dispatch_meta_workspace_size(N, K, E), dev)
+    NK = N * K
+    out = {k: torch.empty(NK, dtype=torch.int32, device=dev) for k in ("indices", "bin_ids", "pos")}
+    out["bins"] = torch.empty(E, dtype=torch.int32, device=dev)
+    out["padded_bins"] = torch.empty(E, dtype=torch.int32, device=dev)
+    out["ws"] = ws
+    call("moe_dispatch_meta", _p(top_experts), N, K, E, _p(out["indices"]), _p(out["bin_ids"]),
+         _p(out["bins"]), _p(out["padded_bins"]), _p(out["pos"]), ws.data_ptr(), ws.numel(),
+         _stream())
+    return out
+
+
+def moe_permute(x, pos, bins, padded_bins, K: int, P: Optional[int] = None, out=None):
+    N, H = x.shape
+    E = bins.shape[0]
+    if P is None:
+        P = padded_rows_max(N, E, K)
+    if out is None:
+        out = torch.empty(P, H, dtype=x.dtype, device=x.device)
+    call("moe_permute", _p(x), _p(pos), _p(bins), _p(padded_bins), N, H, E, K, _dt(x), _p(out),
+         _stream())
+    return out
+
+
+def moe_grouped_swiglu(x_perm, W1, W3, W2, padded_bins, save_gate_up: bool = False, ws=None):
+    P, H = x_perm.shape
+    E, _, F = W1.shape
+    dev = x_perm.device
+    if ws is None:
+        ws = workspace(load().moe_grouped_workspace_size(), dev)
+    act = torch.empty(P, F, dtype=x_perm.dtype, device=dev)
+    out = torch.empty(P, H, dtype=x_perm.dtype, device=dev)
+    gate_up = torch.empty(2, P, F, dtype=x_perm.dtype, device=dev) if save_gate_up else None
+    call("moe_grouped_swiglu", _p(x_perm), _p(W1), _p(W3), _p(W2), _p(padded_bins), E, H, F, P,
+         _dt(x_perm), _p(act), _p(out), _p(gate_up), ws.data_ptr(), ws.numel(), _stream())
+    return act, out, gate_up
+
+
+def moe_combine(out, weights, pos, N: int, y=None):
+    _, H = out.shape
+    K = weights.shape[1]
+    if y is None:
+        y = torch.empty(N, H, dtype=out.dtype, device=out.device)
+    call("moe_combine", _p(out), _p(weights), _p(pos), N, K, H, _dt(out), _p(y), _stream())
+    return y
+
+
+def moe_combine_bwd(dy, out, weights, pos, bins, padded_bins):
+    N, H = dy.shape
+    K = weights.shape[1]
+    E = bins.shape[0]
+    P = out.shape[0]
+    dev = dy.device
+    dw = torch.empty(N, K, dtype=torch.float32, device=dev)
+    dlogit = torch.empty(N, K, dtype=torch.float32, device=dev)
+    d_out = torch.empty(P, H, dtype=dy.dtype, device=dev)
+    call("moe_combine_bwd", _p(dy), _p(out), _p(weights), _p(pos), _p(bins), _p(padded_bins), N, K, H,
+         E, _dt(dy), _p(dw), _p(dlogit), _p(d_out), _stream())
+    return dw, dlogit, d_out
+
+
+def moe_grouped_swiglu_bwd(d_out, x_perm, act, gate_up, W1, W3, W2, padded_bins, ws=None):
+    P, H = x_perm.shape
+    E, _, F = W1.shape
+    dev = x_perm.device
+    if ws is None:
+        ws = workspace(load().moe_grouped_workspace_size(), dev)
+    dt = x_perm.dtype
+    d_gate_up = torch.empty(2, P, F, dtype=dt, device=dev)
+    dW1 = torch.empty(E, H, F, dtype=dt, device=dev)
+    dW3 = torch.empty(E, H, F, dtype=dt, device=dev)
+    dW2 = torch.empty(E, F, H, dtype=dt, device=dev)
+    dx_perm = torch.empty(P, H, dtype=dt, device=dev)
+    call("moe_grouped_swiglu_bwd", _p(d_out), _p(x_perm), _p(act), _p(gate_up), _p(W1), _p(W3), _p(W2),
+         _p(padded_bins), E, H, F, P, _dt(x_perm), _p(d_gate_up), _p(dW1), _p(dW3), _p(dW2),
+         _p(dx_perm), ws.data_ptr(), ws.numel(), _stream())
+    return {"d_gate_up": d_gate_up, "dW1": dW1, "dW3": dW3, "dW2": dW2, "dx_perm": dx_perm}
+
+
+def moe_unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins,
+                             ws=None):
+    N, H = x.shape
+    E = W_r.shape[1]
+    K = top_experts.shape[1]
+    P = dx_perm.shape[0]
+    dev = x.device
+    if ws is None:
+        ws = workspace(load().moe_unpermute_router_bwd_workspace_size(H, E, P), dev)
+    dx = torch.empty(N, H, dtype=x.dtype, device=dev)
+    dW_r = torch.empty(H, E, dtype=x.dtype, device=dev)
+    call("moe_unpermute_router_bwd", _p(dx_perm), _p(dlogit), _p(x), _p(W_r), _p(top_experts), _p(pos),
+         _p(indices), _p(bins), _p(padded_bins), N, H, E, K, P, _dt(x), _p(dx), _p(dW_r),
+         ws.data_ptr(), ws.numel(), _stream())
+    return dx, dW_r
+
+
+class MoELayer:
+    """Whole-layer forward / backward through moe_layer_fwd / moe_layer_bwd.
+
+    Holds the workspace between the forward and the backward pass.  Weights
+    are passed per call so the caller owns them (and their gradients).
+    """
+
+    def __init__(self, N: int, H: int, E: int, K: int, F: int, dtype=torch.bfloat16,
+                 training: bool = False, device="cuda"):
+        self.N, self.H, self.E, self.K, self.F = N, H, E, K, F
+        self.dtype, self.training = dtype, training
+        self.device = torch.device(device)
+        self.dt = _DT[dtype]
+        nbytes = load().moe_workspace_size(N, H, E, K, F, self.dt, int(training))
+        if nbytes == 0:
+            raise _lib.MoEError("moe_workspace_size", _lib.MOE_ERR_UNSUPPORTED)
+        self.ws = workspace(nbytes, self.device)
+        dev = self.device
+        self.y = torch.empty(N, H, dtype=dtype, device=dev)
+        self.top_experts = torch.empty(N, K, dtype=torch.int32, device=dev)
+        self.weights = torch.empty(N, K, dtype=torch.float32, device=dev)
+        self.indices = torch.empty(N * K, dtype=torch.int32, device=dev)
+        self.bins = torch.empty(E, dtype=torch.int32, device=dev)
+        self.padded_bins = torch.empty(E, dtype=torch.int32, device=dev)
+        self._grads = None
+
+    def forward(self, x, W_r, W1, W3, W2, y=None):
+        y = self.y if y is None else y
+        call("moe_layer_fwd", _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), self.N, self.H, self.E, self.K,
+             self.F, self.dt, int(self.training), _p(y), _p(self.top_experts), _p(self.weights),
+             _p(self.indices), _p(self.bins), _p(self.padded_bins), self.ws.data_ptr(),
+             self.ws.numel(), _stream())
+        return y
+
+    def grad_buffers(self):
+        if self._grads is None:
+            dev, dt = self.device, self.dtype
+            N, H, E, F = self.N, self.H, self.E, self.F
+            self._grads = {"dx": torch.empty(N, H, dtype=dt, device=dev),
+                           "dW_r": torch.empty(H, E, dtype=dt, device=dev),
+                           "dW1": torch.empty(E, H, F, dtype=dt, device=dev),
+                           "dW3": torch.empty(E, H, F, dtype=dt, device=dev),
+                           "dW2": torch.empty(E, F, H, dtype=dt, device=dev)}
+        return self._grads
+
+    def backward(self, dy, x, W_r, W1, W3, W2, grads=None):
+        if not self.training:
+            raise RuntimeError("layer was built with training=False")
+        g = self.grad_buffers() if grads is None else grads
+        call("moe_layer_bwd", _p(dy), _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), _p(self.top_experts),
+             _p(self.weights), _p(self.indices), _p(self.bins), _p(self.padded_bins), self.N, self.H,
+             self.E, self.K, self.F, self.dt, _p(g["dx"]), _p(g["dW_r"]), _p(g["dW1"]), _p(g["dW3"]),
+             _p(g["dW2"]), self.ws.data_ptr(), self.ws.numel(), _stream())
+        return g
+
+    def status(self) -> int:
+        return device_status(self.ws)

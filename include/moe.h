@@ -1,0 +1,225 @@
+/*
+ * moe.h - C ABI of the B200 dropless top-k Mixture-of-Experts layer library
+ * (libmoe_b200.so, sm_100a).
+ *
+ * The layer (one device, forward and backward), after the pages describing it:
+ *   router      logits = x W_r, probs = softmax(logits), keep the K largest,
+ *               renormalise the kept values to sum to one
+ *               ("MoE computation principle and execution", sec. 2.1-2.2)
+ *   metadata    sort assignments by expert, histogram, cumsum, round each
+ *               expert's count up to 128 rows, cumsum
+ *               ("MegaBlocks - architecture", sec. 2.1 and 2.3)
+ *   permute     gather token rows into expert order, zero-padded groups
+ *               (MegaBlocks sec. 2.1, padded_gather)
+ *   experts     SwiGLU per expert: A = silu(X W1_e) * (X W3_e), O = A W2_e
+ *               ("LLaMA MoE tutorial", sec. 2.1; icman sec. 2.3), as grouped
+ *               GEMMs over the padded groups (MegaBlocks sec. 2.1, grouped path)
+ *   combine     y_t = sum_k w_{t,k} O[pos(t,k)]  (icman sec. 2.3; MegaBlocks
+ *               sec. 2.1, padded_scatter)
+ *   backward    the chain rule of the above; the gather/scatter pair swap
+ *               roles (MegaBlocks sec. 4) and the router receives gradient
+ *               through the kept softmax weights only (icman sec. 2.2).
+ *
+ * Conventions for every entry point
+ *   - Every pointer argument is a DEVICE pointer allocated by the caller,
+ *     unless stated otherwise; the library never allocates, frees or
+ *     synchronises (except moe_get_device_status, which must return a value).
+ *   - Matrices are dense row-major.  x[N,H]; W_r[H,E]; W1, W3 [E,H,F];
+ *     W2 [E,F,H]; y, dy, dx [N,H]; top_experts, weights [N,K]; flat assignment
+ *     id i = t*K + k.  Element type: MOE_F32 -> float, MOE_BF16 -> bfloat16
+ *     for x, W_r, W1, W3, W2, y and the activations; routing weights,
+ *     logits and probabilities are always float32, ids and offsets int32.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream).
+ *   - The return value reports host-detectable errors only (shapes, dtype,
+ *     alignment, workspace size).  Errors found on the device (an expert id
+ *     outside [0,E), a padded-row count above the buffer, a bounded wait that
+ *     gave up) are OR-ed into the 32-bit status word at the start of the
+ *     workspace; read it with moe_get_device_status.  Kernels never trap.
+ *   - Outputs are overwritten, never accumulated into.
+ *   - Results are bitwise identical from run to run for identical inputs:
+ *     no floating-point atomics, every reduction has a fixed order.
+ *   - Pointers must be 16-byte aligned.  BF16 layers need H and F multiples
+ *     of 128 and E <= 256; F32 layers need H multiple of 4 (tensor cores are
+ *     not used for F32, so F32 results keep full single precision).
+ *   - Rows of padded buffers at or beyond padded_bins[E-1] are never read
+ *     and are left unwritten.
+ */
+#ifndef DROPLESS_TOP_MOE_B200_MOE_H
+#define DROPLESS_TOP_MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, K > E, misalignment */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid shape outside what the kernels implement */
+  MOE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+  MOE_ERR_CUDA = 4           /* a CUDA runtime call failed (launch error etc.) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Bits of the device status word (first 4 bytes of every workspace). */
+#define MOE_DEVERR_EXPERT_ID 0x1   /* a top_experts entry was outside [0,E) */
+#define MOE_DEVERR_TIMEOUT 0x2     /* a bounded pipeline wait gave up */
+#define MOE_DEVERR_ROWS 0x4        /* padded rows exceeded the buffer's rows */
+
+/* The caller's cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+/* Rows per expert group tile: each expert's rows are padded to a multiple of
+ * this (MegaBlocks sec. 2.1 rounds up to 128).  Returns 128. */
+int32_t moe_tile_rows(void);
+
+/* Static upper bound on padded rows for N tokens, E experts, top-K:
+ * round_up(N*K + E*127, 128).  Buffers of this many rows never overflow,
+ * whatever the routing; no host synchronisation is needed to size them. */
+int64_t moe_padded_rows_max(int32_t N, int32_t E, int32_t K);
+
+/* Workspace bytes for each entry point.  A workspace is caller-owned device
+ * memory; its first 256 bytes hold the device status word and must be
+ * zeroed once (moe_workspace_init) before first use. */
+size_t moe_route_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, moe_dtype dt);
+size_t moe_dispatch_meta_workspace_size(int32_t N, int32_t K, int32_t E);
+size_t moe_grouped_workspace_size(void);
+/* Whole layer.  training != 0 adds the activations the backward pass reads
+ * (the same workspace must then be passed to moe_layer_bwd unchanged). */
+size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F,
+                          moe_dtype dt, int32_t training);
+
+/* Zero the device status word of `ws` (async on `stream`). */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Copy the device status word to *status_out (host pointer).  Synchronises
+ * `stream`.  0 means no device-side error since the last moe_workspace_init. */
+moe_status moe_get_device_status(const void* ws, int32_t* status_out, moe_stream_t stream);
+
+/* Router: logits = x W_r (fp32 accumulation), probs = softmax(logits),
+ * top_experts[t, 0..K-1] = the K largest, in descending order, equal values
+ * resolved to the lower expert id; weights = kept probs / their sum.
+ * (icman sec. 2.1-2.2.)  Selection is made on the fp32 logits, which orders
+ * experts exactly as the probabilities do (softmax is monotone).
+ *   x [N,H], W_r [H,E] (dt); logits, probs [N,E] float32 (each may be NULL);
+ *   top_experts [N,K] int32; weights [N,K] float32.
+ *   Needs 1 <= K <= E <= 256. */
+moe_status moe_route(const void* x, const void* W_r, int32_t N, int32_t H, int32_t E, int32_t K,
+                     moe_dtype dt, float* logits, float* probs, int32_t* top_experts,
+                     float* weights, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Dispatch metadata (MegaBlocks sec. 2.1/2.3): stable sort of the N*K flat
+ * assignment ids by expert, histogram, inclusive cumsums.
+ *   top_experts [N*K] int32 in [0,E).
+ *   indices [N*K]  flat ids in expert order (stable: increasing id within an expert)
+ *   bin_ids [N*K]  expert of indices[j]
+ *   bins [E]       inclusive cumsum of the per-expert counts
+ *   padded_bins [E] inclusive cumsum of counts rounded up to 128
+ *   pos [N*K]      padded row of assignment i: start of its expert's padded
+ *                  group + its rank among that expert's assignments
+ * Any output pointer except padded_bins and pos may be NULL.  Ids outside
+ * [0,E) set MOE_DEVERR_EXPERT_ID; their pos is -1 and they are skipped. */
+moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, int32_t E,
+                             int32_t* indices, int32_t* bin_ids, int32_t* bins,
+                             int32_t* padded_bins, int32_t* pos, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* Padded gather (MegaBlocks sec. 2.1): x_perm[pos[t*K+k], :] = x[t, :]; the
+ * pad rows of every expert group (count..round_up(count,128)) are zeroed.
+ *   x [N,H]; x_perm [P,H] with P >= padded_bins[E-1] (dt); bins, padded_bins [E]. */
+moe_status moe_permute(const void* x, const int32_t* pos, const int32_t* bins,
+                       const int32_t* padded_bins, int32_t N, int32_t H, int32_t E, int32_t K,
+                       moe_dtype dt, void* x_perm, moe_stream_t stream);
+
+/* Grouped SwiGLU experts over padded groups: rows [padded_bins[e-1],
+ * padded_bins[e]) use expert e:
+ *   G = X W1_e, U = X W3_e, act = silu(G) * U, out = act W2_e
+ * (LLaMA MoE tutorial sec. 2.1; icman sec. 2.3).  fp32 accumulation; act and
+ * out are rounded once to dt.  P = rows of x_perm/act/out (multiple of 128).
+ *   x_perm [P,H]; W1, W3 [E,H,F]; W2 [E,F,H]; act [P,F]; out [P,H];
+ *   gate_up: NULL, or [2,P,F] receiving G then U (dt) for the backward pass. */
+moe_status moe_grouped_swiglu(const void* x_perm, const void* W1, const void* W3, const void* W2,
+                              const int32_t* padded_bins, int32_t E, int32_t H, int32_t F, int64_t P,
+                              moe_dtype dt, void* act, void* out, void* gate_up,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Weighted combine (icman sec. 2.3): y[t] = sum_{k=0..K-1} weights[t,k] *
+ * out[pos[t*K+k]], summed in increasing k in fp32, rounded once.
+ *   out [P,H]; weights [N,K]; y [N,H]. */
+moe_status moe_combine(const void* out, const float* weights, const int32_t* pos,
+                       int32_t N, int32_t K, int32_t H, moe_dtype dt, void* y,
+                       moe_stream_t stream);
+
+/* Backward of combine and of the router's renormalised weights
+ * (MegaBlocks sec. 4 duality; icman sec. 2.2):
+ *   dw[t,k]  = <dy_t, out[pos[t*K+k]]>           (fixed-order fp32 dot)
+ *   d_out[pos[t*K+k]] = weights[t,k] * dy_t      (pad rows zeroed)
+ *   dlogit[t,k] = weights[t,k] * (dw[t,k] - sum_j weights[t,j] dw[t,j])
+ * dlogit is the gradient of the router logit of expert top_experts[t,k]
+ * (all other logits get zero).  dw, dlogit [N,K] float32 (dw may be NULL);
+ * d_out [P,H] (dt). */
+moe_status moe_combine_bwd(const void* dy, const void* out, const float* weights,
+                           const int32_t* pos, const int32_t* bins, const int32_t* padded_bins,
+                           int32_t N, int32_t K, int32_t H, int32_t E, moe_dtype dt,
+                           float* dw, float* dlogit, void* d_out, moe_stream_t stream);
+
+/* Backward of the grouped SwiGLU experts, per padded group e:
+ *   dA = d_out W2_e^T;  dG = dA * U * silu'(G);  dU = dA * silu(G)
+ *   dW2_e = act^T d_out;  dW1_e = X^T dG;  dW3_e = X^T dU
+ *   dx_perm = dG W1_e^T + dU W3_e^T
+ * gate_up is the [2,P,F] saved by moe_grouped_swiglu.  Experts with no rows
+ * get zero weight gradients.  d_gate_up [2,P,F] is caller scratch.
+ *   dW1, dW3 [E,H,F]; dW2 [E,F,H]; dx_perm [P,H] (dt). */
+moe_status moe_grouped_swiglu_bwd(const void* d_out, const void* x_perm, const void* act,
+                                  const void* gate_up, const void* W1, const void* W3,
+                                  const void* W2, const int32_t* padded_bins, int32_t E,
+                                  int32_t H, int32_t F, int64_t P, moe_dtype dt,
+                                  void* d_gate_up, void* dW1, void* dW3, void* dW2,
+                                  void* dx_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Backward of the permute and of the router GEMM:
+ *   dx[t] = sum_k dx_perm[pos[t*K+k]] + sum_k dlogit[t,k] * W_r[:, top_experts[t,k]]
+ *   dW_r[:, e] = sum over assignments i of expert e, in sorted order, of
+ *                dlogit_i * x[token(i)]
+ * (sums in fixed order, fp32).  indices/bins/padded_bins from
+ * moe_dispatch_meta; P = rows of dx_perm.  ws: moe_unpermute_router_bwd_workspace_size.
+ *   dx [N,H]; dW_r [H,E] (dt). */
+size_t moe_unpermute_router_bwd_workspace_size(int32_t H, int32_t E, int64_t P);
+moe_status moe_unpermute_router_bwd(const void* dx_perm, const float* dlogit, const void* x,
+                                    const void* W_r, const int32_t* top_experts,
+                                    const int32_t* pos, const int32_t* indices,
+                                    const int32_t* bins, const int32_t* padded_bins, int32_t N,
+                                    int32_t H, int32_t E, int32_t K, int64_t P, moe_dtype dt,
+                                    void* dx, void* dW_r, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/* Whole layer forward: route -> dispatch_meta -> permute -> grouped SwiGLU
+ * -> combine, all on `stream`, no host synchronisation.
+ *   y [N,H] (dt); top_experts [N,K]; weights [N,K]; indices [N*K];
+ *   bins, padded_bins [E] (all outputs required).
+ * ws: moe_workspace_size(..., training) bytes; with training != 0 it keeps
+ * what moe_layer_bwd reads. */
+moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const void* W3,
+                         const void* W2, int32_t N, int32_t H, int32_t E, int32_t K, int32_t F,
+                         moe_dtype dt, int32_t training, void* y, int32_t* top_experts,
+                         float* weights, int32_t* indices, int32_t* bins, int32_t* padded_bins,
+                         void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Whole layer backward for the forward run last with this workspace
+ * (training != 0).  dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F],
+ * dW2 [E,F,H], all dt, overwritten. */
+moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const void* W1,
+                         const void* W3, const void* W2, const int32_t* top_experts,
+                         const float* weights, const int32_t* indices, const int32_t* bins,
+                         const int32_t* padded_bins, int32_t N, int32_t H, int32_t E, int32_t K,
+                         int32_t F, moe_dtype dt, void* dx, void* dW_r, void* dW1, void* dW3,
+                         void* dW2, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DROPLESS_TOP_MOE_B200_MOE_H */

@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/moe.h declares, and rejects bad arguments before any
+device work.  Pointers passed here are never dereferenced (validation
+returns first)."""
+import os
+import re
+
+import pytest
+
+from dropless_top_moe_b200 import _lib
+from dropless_top_moe_b200._lib import (MOE_BF16, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED,
+                                        MOE_ERR_WORKSPACE, MOE_F32, load)
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|int32_t|int64_t)\s+(moe_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dropless_top_moe_b200.build import build
+    build()
+    return load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"{n} missing from the binding"
+    assert set(_lib.SIGNATURES) == set(names)
+
+
+def test_static_sizes(lib):
+    assert lib.moe_tile_rows() == 128
+    assert lib.moe_padded_rows_max(4096, 8, 2) == 9216
+    assert lib.moe_padded_rows_max(8192, 256, 8) == 98048
+    assert lib.moe_padded_rows_max(16384, 64, 6) == 106496
+    assert lib.moe_padded_rows_max(16384, 64, 4) == 73728
+    assert lib.moe_padded_rows_max(0, 4, 2) == 512
+
+
+def test_workspace_sizes(lib):
+    inf = lib.moe_workspace_size(4096, 4096, 8, 2, 14336, MOE_BF16, 0)
+    trn = lib.moe_workspace_size(4096, 4096, 8, 2, 14336, MOE_BF16, 1)
+    P = 9216
+    assert inf >= P * (4096 * 2 + 14336) * 2
+    assert trn > inf + 2 * P * 14336 * 2
+    assert lib.moe_workspace_size(4096, 4000, 8, 2, 14336, MOE_BF16, 0) == 0   # H % 128
+    assert lib.moe_workspace_size(16, 8, 4, 5, 8, MOE_F32, 0) == 0             # K > E
+    assert lib.moe_dispatch_meta_workspace_size(100, 2, 4) >= 256
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_route_rejects_bad_shapes(lib):
+    ws_size = 1 << 20
+    assert lib.moe_route(FAKE, FAKE, 16, 128, 4, 5, MOE_F32, None, None, FAKE, FAKE, FAKE, ws_size,
+                         None) == MOE_ERR_INVALID_ARG
+    assert lib.moe_route(FAKE, FAKE, 16, 100, 4, 2, MOE_BF16, None, None, FAKE, FAKE, FAKE, ws_size,
+                         None) == MOE_ERR_UNSUPPORTED
+    assert lib.moe_route(FAKE, FAKE, 16, 128, 300, 2, MOE_BF16, None, None, FAKE, FAKE, FAKE, ws_size,
+                         None) == MOE_ERR_UNSUPPORTED
+    assert lib.moe_route(FAKE + 4, FAKE, 16, 128, 4, 2, MOE_F32, None, None, FAKE, FAKE, FAKE, ws_size,
+                         None) == MOE_ERR_INVALID_ARG
+    assert lib.moe_route(FAKE, FAKE, 16, 128, 4, 2, MOE_F32, None, None, FAKE, FAKE, FAKE, 8,
+                         None) == MOE_ERR_WORKSPACE
+
+
+def test_layer_rejects_bad_arguments(lib):
+    args = [FAKE] * 5 + [64, 128, 4, 2, 256, MOE_BF16, 0] + [FAKE] * 6
+    assert lib.moe_layer_fwd(*args, FAKE, 1024, None) == MOE_ERR_WORKSPACE
+    bad = list(args)
+    bad[0] = None
+    assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_INVALID_ARG
+    bad = list(args)
+    bad[9] = 100   # F not a multiple of 128 on the tensor-core path
+    assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[8] = 5     # K > E
+    assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_INVALID_ARG
+
+
+def test_meta_and_grouped_reject_bad_arguments(lib):
+    assert lib.moe_dispatch_meta(FAKE, 10, 3, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
+                                 None) == MOE_ERR_INVALID_ARG
+    assert lib.moe_dispatch_meta(FAKE, 10, 2, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+                                 None) == MOE_ERR_WORKSPACE
+    # P must be a multiple of 128
+    assert lib.moe_grouped_swiglu(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, 100, MOE_BF16, FAKE, FAKE,
+                                  None, FAKE, 4096, None) == MOE_ERR_INVALID_ARG

@@ -1,0 +1,137 @@
+"""Whole-layer parity (forward and backward) of the CUDA path against the CPU
+oracle, through moe_layer_fwd / moe_layer_bwd (GPU only)."""
+import numpy as np
+import pytest
+import torch
+
+import dropless_top_moe_b200 as moe
+from gen import WORKLOADS
+from oracle import moe_oracle as om
+from tests._cases import TOL, W_TOL, assert_scaled, make_case, small_shape
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fwd(shape, c, training=False):
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=training)
+    y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"]).clone()
+    return layer, y
+
+
+def check_routing_and_meta(layer, shape, ref):
+    np.testing.assert_array_equal(layer.top_experts.cpu().numpy(), ref["top_experts"])
+    assert np.max(np.abs(layer.weights.cpu().numpy() - ref["weights"])) <= W_TOL
+    m = om.dispatch_meta(ref["top_experts"], shape.E)
+    np.testing.assert_array_equal(layer.indices.cpu().numpy(), m["indices"])
+    np.testing.assert_array_equal(layer.bins.cpu().numpy(), m["bins"])
+    np.testing.assert_array_equal(layer.padded_bins.cpu().numpy(), m["padded_bins"])
+    return m
+
+
+FWD_SMALL = [
+    small_shape("tiny_fp32_like", N=256, H=128, E=4, K=2, F=256, dtype="f32"),
+    small_shape("f32_ragged", N=203, H=64, E=5, K=3, F=96, dtype="f32"),
+    small_shape("bf16_e8", N=700, H=256, E=8, K=2, F=512),
+    small_shape("bf16_e64_k6_zipf", N=900, H=256, E=64, K=6, F=384, skew="zipf", skew_param=1.0),
+    small_shape("bf16_e256_k8", N=600, H=256, E=256, K=8, F=256, skew="normal", skew_param=1.0),
+    small_shape("bf16_k1", N=333, H=128, E=16, K=1, F=128),
+    small_shape("bf16_k_eq_e", N=250, H=128, E=16, K=16, F=128),
+    small_shape("f32_single_expert", N=77, H=32, E=1, K=1, F=48, dtype="f32"),
+    small_shape("megablocks_dmoe_test_dims", N=1024, H=512, E=8, K=2, F=1024),
+]
+
+
+@pytest.mark.parametrize("shape", FWD_SMALL, ids=lambda s: s.name)
+def test_layer_forward_small(shape):
+    c = make_case(shape, seed=3)
+    layer, y = run_fwd(shape, c)
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    check_routing_and_meta(layer, shape, ref)
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(),
+                        shape.K, routing=ref)["y"]
+    assert_scaled(y, yr, shape.dtype, "y")
+
+
+def test_layer_forward_tiny_fp32_workload():
+    shape = WORKLOADS["tiny_fp32"]
+    c = make_case(shape, seed=0)
+    layer, y = run_fwd(shape, c)
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    check_routing_and_meta(layer, shape, ref)
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(),
+                        shape.K, routing=ref)["y"]
+    assert_scaled(y, yr, "f32", "y")
+
+
+def test_one_expert_takes_every_token():
+    shape = small_shape("hot", N=512, H=128, E=8, K=2, F=128, skew="zipf", skew_param=1.0)
+    c = make_case(shape, seed=4, repair=False)
+    c["W_r"][0, :] = 0
+    c["W_r"][0, 5] = 60.0          # expert 5 first for every token
+    c["W_r"][0, 2] = 30.0          # expert 2 second
+    layer, y = run_fwd(shape, c)
+    te = layer.top_experts.cpu().numpy()
+    assert np.all(te[:, 0] == 5) and np.all(te[:, 1] == 2)
+    bins = layer.bins.cpu().numpy()
+    assert bins[-1] == 1024 and np.count_nonzero(np.diff(np.concatenate([[0], bins]))) == 2
+    ref = om.route(c["x"].cpu(), c["W_r"].cpu(), 2)
+    yr = om.moe_forward(c["x"].cpu(), c["W_r"].cpu(), c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), 2,
+                        routing=ref)["y"]
+    assert_scaled(y, yr, "bf16", "y")
+
+
+def test_layer_forward_mixtral_full_size_sampled():
+    shape = WORKLOADS["mixtral"]
+    c = make_case(shape, seed=0)
+    layer, y = run_fwd(shape, c)
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    m = check_routing_and_meta(layer, shape, ref)
+    assert om.maxvio(m["hist"], shape.N, shape.K, shape.E) < 0.3
+    tok = np.sort(np.random.default_rng(0).choice(shape.N, 1024, replace=False))
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"], c["W3"], c["W2"], shape.K, routing=ref,
+                        tokens=tok)["y"]
+    assert_scaled(y[torch.as_tensor(tok, device="cuda")], yr, "bf16", "y sampled")
+
+
+BWD_SMALL = [
+    small_shape("f32_bwd", N=256, H=64, E=4, K=2, F=96, dtype="f32", training=True),
+    small_shape("f32_bwd_k3", N=190, H=32, E=6, K=3, F=64, dtype="f32", training=True),
+    small_shape("bf16_bwd", N=640, H=256, E=8, K=2, F=256, training=True),
+    small_shape("bf16_bwd_e64", N=900, H=256, E=64, K=4, F=384, training=True),
+    small_shape("bf16_bwd_h128", N=400, H=128, E=16, K=4, F=128, training=True),
+]
+
+
+def _bwd_case(shape, seed):
+    c = make_case(shape, seed=seed, with_dy=True)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=True)
+    layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    g = layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    return c, layer, g
+
+
+@pytest.mark.parametrize("shape", BWD_SMALL, ids=lambda s: s.name)
+def test_layer_backward_small(shape):
+    c, layer, g = _bwd_case(shape, seed=5)
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    check_routing_and_meta(layer, shape, ref)
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(),
+                         shape.K, c["dy"].cpu(), routing=ref)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(g[k], gr[k], shape.dtype, k)
+
+
+def test_layer_is_bitwise_deterministic():
+    shape = small_shape("det", N=1500, H=256, E=64, K=4, F=256, training=True)
+    outs = []
+    for _ in range(2):
+        c, layer, g = _bwd_case(shape, seed=6)
+        outs.append([layer.y.clone(), layer.top_experts.clone(), layer.weights.clone()] +
+                    [g[k].clone() for k in ("dx", "dW_r", "dW1", "dW3", "dW2")])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
