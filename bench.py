@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 dropless top-k MoE layer.
+
+One step = one training pass of the whole layer (forward + backward: router,
+dispatch metadata, permute, grouped SwiGLU GEMMs, combine and all backward
+kernels) over one batch of synthetic tokens, through the C ABI.  Default
+workload: the training-step configuration N=16384, H=4096, E=64, top_k=4,
+F=2048, bf16 (the one workload that exercises every step of the layer).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica on its own batch: the layer has no exchange step of its own, so the
+data path has no collective; the only collective is the max-over-ranks of
+the timing.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s on 1 B200; grouped-GEMM % bf16 peak; meta/gather % HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="train_step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0, help="override N (small profiling cases)")
+    ap.add_argument("--experts", type=int, default=0, help="override E (small profiling cases)")
+    return ap.parse_args()
+
+
+def workload(args):
+    from gen import WORKLOADS
+    s = WORKLOADS[args.workload]
+    if args.tokens:
+        s = s.with_(N=args.tokens, name=s.name + f"_N{args.tokens}")
+    if args.experts:
+        s = s.with_(E=args.experts, name=s.name + f"_E{args.experts}")
+    return s
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- work model
+
+def flops_by_kernel(s):
+    """Algorithmic FLOPs per launch (padding rows and recompute not counted)."""
+    NKHF = s.N * s.K * s.H * s.F
+    return {"gemm1_swiglu": 4 * NKHF, "gemm2": 2 * NKHF, "dgrad_w2_swiglu_bwd": 2 * NKHF,
+            "wgrad_w2": 2 * NKHF, "wgrad_w1_w3": 4 * NKHF, "dgrad_x": 4 * NKHF,
+            "route_umma": 2 * s.N * s.H * s.E}
+
+
+def bytes_by_kernel(s, padded_rows):
+    """Algorithmic HBM bytes per launch of the bandwidth-bound kernels."""
+    b = 2 if s.dtype == "bf16" else 4
+    N, K, H, E = s.N, s.K, s.H, s.E
+    return {"route_simt": N * H * b + H * E * b + N * K * 8,
+            "permute": N * H * b + padded_rows * H * b + N * K * 4,
+            "combine": N * K * H * b + N * K * 8 + N * H * b,
+            "combine_bwd": N * H * b + N * K * H * b + padded_rows * H * b + N * K * 12,
+            "unpermute_dx": N * K * H * b + N * H * b + N * K * 12,
+            "router_wgrad_partial": N * K * H * b + N * K * 8,
+            "meta_count": N * K * 4, "meta_place": N * K * 4 * 3}
+
+
+def step_tokens(s):
+    return s.N
+
+
+def layer_flops(s):
+    fwd = 6 * s.N * s.K * s.H * s.F + 2 * s.N * s.H * s.E
+    return fwd * 3 if s.training else fwd
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- traffic
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, only while the
+    kernel's source is unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = os.path.join(ROOT, "dropless_top_moe_b200", "csrc")
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        parts = line.split()
+        if len(parts) < 4 or parts[0] != kernel:
+            continue
+        bytes_, fname, sha = float(parts[1]), parts[2], parts[3]
+        try:
+            cur = hashlib.sha256(open(os.path.join(src, fname), "rb").read()).hexdigest()[:16]
+        except OSError:
+            return None
+        return bytes_ if cur == sha else None
+    return None
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from gen import WORKLOADS, make_inputs, token_rows
+    from gen.moe_inputs import _gen
+
+    import dropless_top_moe_b200 as moe
+    from dropless_top_moe_b200._lib import call, load
+
+    shape = workload(args)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(shape, seed=0, device=dev, with_dy=shape.training)
+    if world > 1:   # each replica its own batch, same weights
+        inp["x"] = token_rows(shape, shape.N, _gen(1000 + rank, dev), dev)
+        if shape.training:
+            inp["dy"] = torch.randn(shape.N, shape.H, generator=_gen(2000 + rank, dev), device=dev).to(shape.torch_dtype)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=shape.training, device=dev)
+    grads = layer.grad_buffers() if shape.training else None
+
+    def step():
+        layer.forward(inp["x"], inp["W_r"], inp["W1"], inp["W3"], inp["W2"])
+        if shape.training:
+            layer.backward(inp["dy"], inp["x"], inp["W_r"], inp["W1"], inp["W3"], inp["W2"], grads)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    # launches per step (counted through the trace hook)
+    def make_events(n):
+        # torch creates the underlying cudaEvent on first record
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in es:
+            e.record()
+        torch.cuda.synchronize()
+        return es
+
+    cap = 4096
+    evs = make_events(2 * cap)
+    ev_arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in evs])
+    labels = (ctypes.c_char_p * cap)()
+    count = ctypes.c_int32(0)
+    call("moe_trace_attach", ev_arr, cap, labels, ctypes.byref(count))
+    step()
+    torch.cuda.synchronize()
+    per_step = count.value
+    call("moe_trace_detach")
+    steps = args.steps
+    cap_needed = per_step * steps
+    if cap_needed > cap:
+        evs += make_events(2 * (cap_needed - cap))
+        cap = cap_needed
+        ev_arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in evs])
+        labels = (ctypes.c_char_p * cap)()
+
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    call("moe_trace_attach", ev_arr, cap, labels, ctypes.byref(count))
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    call("moe_trace_detach")
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end) / steps
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    status = layer.status()
+
+    # per-kernel device time over the timed region
+    per = {}
+    for i in range(count.value):
+        name = labels[i].decode()
+        d = evs[2 * i].elapsed_time(evs[2 * i + 1])
+        tot, n = per.get(name, (0.0, 0))
+        per[name] = (tot + d, n + 1)
+    padded_rows = int(layer.padded_bins[-1].item())
+    fl = flops_by_kernel(shape)
+    by = bytes_by_kernel(shape, padded_rows)
+    peaks, peak_src = load_peaks()
+    kernels = {}
+    for name, (tot, n) in per.items():
+        avg = tot / n
+        k = {"launches": n, "ms_avg": round(avg, 4), "share": round(tot / (ms * steps), 4)}
+        if name in fl:
+            k["tflops"] = round(fl[name] / (avg * 1e-3) / 1e12, 1)
+        elif name in by:
+            k["gbs"] = round(by[name] / (avg * 1e-3) / 1e9, 1)
+        kernels[name] = k
+    dom = max(per, key=lambda n: per[n][0])
+    dom_avg_s = per[dom][0] / per[dom][1] * 1e-3
+    if dom in fl:
+        peak = peaks["bf16_tflops_sustained"]
+        achieved = fl[dom] / dom_avg_s / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} sustained bf16 (kernel timed inside a long step)"}
+    else:
+        peak = peaks["hbm_gbs"]
+        achieved = by.get(dom, 0) / dom_avg_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} copy bandwidth"}
+    tr = recorded_traffic(dom)
+    roof["traffic"] = tr
+
+    result = {
+        "metric": METRIC, "value": None, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded normal inputs and random-init weights of the stated shapes)",
+        "config": {"workload": f"{shape.name}: N={shape.N} H={shape.H} E={shape.E} top_k={shape.K} "
+                               f"F={shape.F} SwiGLU, {'forward+backward' if shape.training else 'forward'}",
+                   "tokens_per_step_per_gpu": shape.N, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
+                         (3 * shape.E * shape.H * shape.F * 2 / 1e9)},
+        "tflops": round(layer_flops(shape) / (ms_max * 1e-3) / 1e12, 1),
+        "roofline": roof, "kernels": kernels, "gpu_launches": count.value,
+        "launches_per_step": per_step, "device_status": status, "clocks": clk,
+    }
+    result["value"] = round(shape.N * world / (ms_max * 1e-3), 1)
+
+    # end to end through the same entry points, host buffers, copies timed
+    if not args.no_e2e:
+        xh = inp["x"].cpu().pin_memory()
+        dyh = inp["dy"].cpu().pin_memory() if shape.training else None
+        yh = torch.empty_like(xh).pin_memory()
+        dxh = torch.empty_like(xh).pin_memory() if shape.training else None
+        xd, dyd = torch.empty_like(inp["x"]), (torch.empty_like(inp["dy"]) if shape.training else None)
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            if shape.training:
+                dyd.copy_(dyh, non_blocking=True)
+            y = layer.forward(xd, inp["W_r"], inp["W1"], inp["W3"], inp["W2"])
+            if shape.training:
+                g = layer.backward(dyd, xd, inp["W_r"], inp["W1"], inp["W3"], inp["W2"], grads)
+                dxh.copy_(g["dx"], non_blocking=True)
+            yh.copy_(y, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n_e2e = max(5, steps // 2)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        ems = s0.elapsed_time(s1) / n_e2e
+        te = torch.tensor([ems], device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        ems = float(te.item())
+        eb = xh.element_size()
+        result["e2e"] = {"value": round(shape.N * world / (ems * 1e-3), 1), "unit": "tokens/s",
+                         "ms_per_step": round(ems, 4),
+                         "h2d_bytes_per_step": xh.numel() * eb * (2 if shape.training else 1),
+                         "d2h_bytes_per_step": xh.numel() * eb * (2 if shape.training else 1)}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(shape, inp, budget_s=20.0)
+    return result
+
+
+# ---------------------------------------------------------------- oracle legs
+
+def _oracle_inputs(shape, inp=None):
+    """float64 host copies of one workload's inputs (made once, outside timing)."""
+    import torch
+    from gen import make_inputs
+    from oracle import moe_oracle as om
+    if inp is None:
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        inp = make_inputs(shape, seed=0, device=dev, with_dy=True)
+        if "dy" not in inp:
+            inp["dy"] = torch.randn(shape.N, shape.H, device=dev).to(shape.torch_dtype)
+    dy = inp.get("dy")
+    if dy is None:
+        dy = torch.zeros(shape.N, shape.H)
+    return {k: om.f64(v) for k, v in (("x", inp["x"]), ("W_r", inp["W_r"]), ("W1", inp["W1"]),
+                                      ("W3", inp["W3"]), ("W2", inp["W2"]), ("dy", dy))}
+
+
+def _oracle_step(shape, o, tokens):
+    from oracle import moe_oracle as om
+    xs = o["x"][tokens]
+    out = om.moe_forward(xs, o["W_r"], o["W1"], o["W3"], o["W2"], shape.K)
+    if shape.training:
+        om.moe_backward(xs, o["W_r"], o["W1"], o["W3"], o["W2"], shape.K, o["dy"][tokens],
+                        routing=out["routing"])
+    return out
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(shape, inp=None, budget_s=20.0, o=None):
+    """The oracle, as it stands, on a bounded token sample of the workload."""
+    import numpy as np
+    o = o if o is not None else _oracle_inputs(shape, inp)
+    rng = np.random.default_rng(0)
+    n = 8
+    t0 = time.perf_counter()
+    _oracle_step(shape, o, np.sort(rng.choice(shape.N, n, replace=False)))
+    t_cal = time.perf_counter() - t0
+    n = int(min(shape.N, max(8, n * (budget_s * 0.7) / max(t_cal, 1e-3))))
+    tok = np.sort(rng.choice(shape.N, n, replace=False))
+    t0 = time.perf_counter()
+    _oracle_step(shape, o, tok)
+    dt = time.perf_counter() - t0
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"{n} of {shape.N} tokens of {shape.name} ({'fwd+bwd' if shape.training else 'fwd'}), "
+                      f"float64 numpy oracle, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle on this workload's config, host cores."""
+    from gen import WORKLOADS
+    import numpy as np
+    if rank != 0:
+        return None
+    shape = workload(args)
+    o = _oracle_inputs(shape)
+    rng = np.random.default_rng(1)
+    # size each step so the whole run stays within a few minutes
+    t0 = time.perf_counter()
+    _oracle_step(shape, o, np.sort(rng.choice(shape.N, 4, replace=False)))
+    per_tok = (time.perf_counter() - t0) / 4
+    n_steps = args.steps + args.warmup
+    n = int(max(1, min(shape.N, (150.0 / max(n_steps, 1)) / max(per_tok, 1e-6))))
+    for _ in range(args.warmup):
+        _oracle_step(shape, o, np.sort(rng.choice(shape.N, n, replace=False)))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(shape, o, np.sort(rng.choice(shape.N, n, replace=False)))
+    dt = time.perf_counter() - t0
+    v = n * args.steps / dt
+    ms = dt / args.steps * 1e3
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{shape.name}: N={shape.N} H={shape.H} E={shape.E} top_k={shape.K} "
+                                   f"F={shape.F} SwiGLU, {'forward+backward' if shape.training else 'forward'}",
+                       "tokens_per_step": n},
+            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+                             "sample": f"{n} of {shape.N} tokens per step"},
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    if rank == 0:
+        from dropless_top_moe_b200.build import build
+        build()
+    if world > 1:
+        dist.barrier()
+    res = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

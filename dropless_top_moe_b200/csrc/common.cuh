@@ -93,7 +93,21 @@ __device__ __forceinline__ int expert_of_row(const int32_t* padded_bins, int E, 
   return lo;
 }
 
+namespace trace {
+// Bracket one kernel launch with caller-owned events (no-op unless attached).
+void begin(const char* name, cudaStream_t s);
+void end(cudaStream_t s);
+}  // namespace trace
+
 }  // namespace moe
+
+// Launch `launch` (a kernel<<<...>>>(...) statement) between trace events.
+#define MOE_TRACED(name, s, launch)     \
+  do {                                  \
+    moe::trace::begin(name, s);         \
+    launch;                             \
+    moe::trace::end(s);                 \
+  } while (0)
 
 // Launch-error check used by the host wrappers.
 #define MOE_LAUNCH_CHECK()                                   \

@@ -163,15 +163,15 @@ static moe_status swiglu_fwd_simt_t(const void* x_perm, const void* W1, const vo
   T* U = gate_up ? (T*)gate_up + (size_t)P * F : nullptr;
   dim3 g1((unsigned)cdiv(F, kSB), (unsigned)(P / kSB));
   // G, U = X W1_e, X W3_e ; W1 [E,H,F]: B(e,k=h,n=f) = W1[e*H*F + h*F + f]
-  gemm_rows_simt_kernel<T, SIMT_SWIGLU><<<g1, 256, 0, s>>>(
+  MOE_TRACED("simt_gemm1_swiglu", s, (gemm_rows_simt_kernel<T, SIMT_SWIGLU><<<g1, 256, 0, s>>>(
       (const T*)x_perm, nullptr, H, (const T*)W1, (const T*)W3, (int64_t)H * F, F, 1, pb, E, H, F,
-      (T*)act, G, U, F, nullptr, nullptr);
+      (T*)act, G, U, F, nullptr, nullptr)));
   MOE_LAUNCH_CHECK();
   dim3 g2((unsigned)cdiv(H, kSB), (unsigned)(P / kSB));
   // O = A W2_e ; W2 [E,F,H]
-  gemm_rows_simt_kernel<T, SIMT_STORE><<<g2, 256, 0, s>>>(
+  MOE_TRACED("simt_gemm2", s, (gemm_rows_simt_kernel<T, SIMT_STORE><<<g2, 256, 0, s>>>(
       (const T*)act, nullptr, F, (const T*)W2, nullptr, (int64_t)F * H, H, 1, pb, E, F, H, (T*)out,
-      nullptr, nullptr, H, nullptr, nullptr);
+      nullptr, nullptr, H, nullptr, nullptr)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -194,27 +194,27 @@ static moe_status swiglu_bwd_simt_t(const void* d_out, const void* x_perm, const
   T* dU = dG + (size_t)P * F;
   // dA = dO W2_e^T : B(e,k=h,n=f) = W2[e*F*H + f*H + h]  -> sBk = 1, sBn = H
   dim3 g1((unsigned)cdiv(F, kSB), (unsigned)(P / kSB));
-  gemm_rows_simt_kernel<T, SIMT_SWIGLU_BWD><<<g1, 256, 0, s>>>(
+  MOE_TRACED("simt_dgrad_w2_swiglu_bwd", s, (gemm_rows_simt_kernel<T, SIMT_SWIGLU_BWD><<<g1, 256, 0, s>>>(
       (const T*)d_out, nullptr, H, (const T*)W2, nullptr, (int64_t)F * H, 1, H, pb, E, H, F, dG, dU,
-      nullptr, F, G, U);
+      nullptr, F, G, U)));
   MOE_LAUNCH_CHECK();
   // dW2_e = act^T dO  [F,H];  dW1_e = X^T dG, dW3_e = X^T dU  [H,F]
   dim3 gw2((unsigned)cdiv(H, kSB), (unsigned)cdiv(F, kSB), (unsigned)E);
-  gemm_wgrad_simt_kernel<T><<<gw2, 256, 0, s>>>((const T*)act, F, (const T*)d_out, H, pb, F, H,
-                                                (T*)dW2, (int64_t)F * H, H);
+  MOE_TRACED("simt_wgrad_w2", s, (gemm_wgrad_simt_kernel<T><<<gw2, 256, 0, s>>>((const T*)act, F, (const T*)d_out, H, pb, F, H,
+                                                (T*)dW2, (int64_t)F * H, H)));
   MOE_LAUNCH_CHECK();
   dim3 gw1((unsigned)cdiv(F, kSB), (unsigned)cdiv(H, kSB), (unsigned)E);
-  gemm_wgrad_simt_kernel<T><<<gw1, 256, 0, s>>>((const T*)x_perm, H, dG, F, pb, H, F, (T*)dW1,
-                                                (int64_t)H * F, F);
+  MOE_TRACED("simt_wgrad_w1", s, (gemm_wgrad_simt_kernel<T><<<gw1, 256, 0, s>>>((const T*)x_perm, H, dG, F, pb, H, F, (T*)dW1,
+                                                (int64_t)H * F, F)));
   MOE_LAUNCH_CHECK();
-  gemm_wgrad_simt_kernel<T><<<gw1, 256, 0, s>>>((const T*)x_perm, H, dU, F, pb, H, F, (T*)dW3,
-                                                (int64_t)H * F, F);
+  MOE_TRACED("simt_wgrad_w3", s, (gemm_wgrad_simt_kernel<T><<<gw1, 256, 0, s>>>((const T*)x_perm, H, dU, F, pb, H, F, (T*)dW3,
+                                                (int64_t)H * F, F)));
   MOE_LAUNCH_CHECK();
   // dx_perm = dG W1_e^T + dU W3_e^T : B(e,k=f,n=h) = W1[e*H*F + h*F + f] -> sBk = 1, sBn = F
   dim3 g3((unsigned)cdiv(H, kSB), (unsigned)(P / kSB));
-  gemm_rows_simt_kernel<T, SIMT_DUAL><<<g3, 256, 0, s>>>(
+  MOE_TRACED("simt_dgrad_x", s, (gemm_rows_simt_kernel<T, SIMT_DUAL><<<g3, 256, 0, s>>>(
       dG, dU, F, (const T*)W1, (const T*)W3, (int64_t)H * F, 1, F, pb, E, F, H, (T*)dx_perm, nullptr,
-      nullptr, H, nullptr, nullptr);
+      nullptr, H, nullptr, nullptr)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

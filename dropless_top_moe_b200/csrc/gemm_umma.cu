@@ -553,7 +553,7 @@ static int sm_count() {
 }
 
 template <int BN, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
-static moe_status launch(const Params& p, int64_t tiles_upper, cudaStream_t s) {
+static moe_status launch(const char* name, const Params& p, int64_t tiles_upper, cudaStream_t s) {
   constexpr int STAGE_BYTES = kA_BYTES + BN * BK * 2;
   constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
   const size_t smem = (size_t)STAGES * STAGE_BYTES + 1024 + 8 * (2 * STAGES + 5) + 16;
@@ -564,7 +564,7 @@ static moe_status launch(const Params& p, int64_t tiles_upper, cudaStream_t s) {
   }
   int64_t grid = tiles_upper < sm_count() ? tiles_upper : sm_count();
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, kThreads, smem, s>>>(p);
+  MOE_TRACED(name, s, (kern<<<(unsigned)grid, kThreads, smem, s>>>(p)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -602,7 +602,7 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.out1 = gate_up ? (bf*)gate_up : nullptr;
     p.out2 = gate_up ? (bf*)gate_up + (size_t)P * F : nullptr;
     p.ldo = F;
-    moe_status st = launch<256, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>(p, (P / BM) * p.n_tiles, s);
+    moe_status st = launch<256, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p, (P / BM) * p.n_tiles, s);
     if (st != MOE_OK) return st;
   }
   // GEMM2: out = act * W2_e
@@ -615,8 +615,8 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.n_tiles = H / bn;
     p.out0 = (bf*)out;
     p.ldo = H;
-    if (bn == 256) return launch<256, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s);
-    return launch<128, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s);
+    if (bn == 256) return launch<256, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
+    return launch<128, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
   }
 }
 
@@ -644,8 +644,8 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.out0 = dG;
     p.out1 = dU;
     p.ldo = F;
-    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s)
-                   : launch<128, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>(p, (P / BM) * p.n_tiles, s);
+    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, (P / BM) * p.n_tiles, s)
+                   : launch<128, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, (P / BM) * p.n_tiles, s);
     if (st != MOE_OK) return st;
   }
   // dW2_e = act_e^T * d_out_e   [F, H]
@@ -660,8 +660,8 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.ldo = H;
     p.out_estride = (int64_t)F * H;
     const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
-    st = bn == 256 ? launch<256, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>(p, tiles, s)
-                   : launch<128, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>(p, tiles, s);
+    st = bn == 256 ? launch<256, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s)
+                   : launch<128, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
     if (st != MOE_OK) return st;
   }
   // dW1_e | dW3_e = x_perm_e^T * [dG_e | dU_e]   [H, F] each
@@ -678,7 +678,7 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.ldo = F;
     p.out_estride = (int64_t)H * F;
     const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
-    st = launch<256, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>(p, tiles, s);
+    st = launch<256, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
     if (st != MOE_OK) return st;
   }
   // dx_perm = dG * W1_e^T + dU * W3_e^T  (one K = 2F contraction)
@@ -694,8 +694,8 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.n_tiles = H / bn;
     p.out0 = (bf*)dx_perm;
     p.ldo = H;
-    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>(p, (P / BM) * p.n_tiles, s)
-                   : launch<128, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>(p, (P / BM) * p.n_tiles, s);
+    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, (P / BM) * p.n_tiles, s)
+                   : launch<128, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, (P / BM) * p.n_tiles, s);
     if (st != MOE_OK) return st;
   }
   return MOE_OK;
@@ -724,7 +724,7 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   p.probs = probs;
   p.top = top;
   p.weights = w;
-  return launch<256, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>(p, cdiv(N, BM), s);
+  return launch<256, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
 }
 
 }  // namespace moe

@@ -139,17 +139,17 @@ moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices
   int32_t* chunk_counts = (int32_t*)scratch;
   int32_t* sorted_start = chunk_counts + (size_t)n_chunks * E;
   int32_t* padded_start = sorted_start + E;
-  meta_count_kernel<<<n_chunks, 256, E * sizeof(int), s>>>(top, NK, E, chunk_counts, status);
+  MOE_TRACED("meta_count", s, (meta_count_kernel<<<n_chunks, 256, E * sizeof(int), s>>>(top, NK, E, chunk_counts, status)));
   MOE_LAUNCH_CHECK();
-  meta_scan_kernel<<<1, 256, 0, s>>>(chunk_counts, n_chunks, E, bins, padded_bins, sorted_start,
-                                     padded_start);
+  MOE_TRACED("meta_scan", s, (meta_scan_kernel<<<1, 256, 0, s>>>(chunk_counts, n_chunks, E, bins, padded_bins, sorted_start,
+                                     padded_start)));
   MOE_LAUNCH_CHECK();
   if (NK > 0) {
     const size_t smem = (size_t)(kMetaPlaceThreads / 32 + 2) * E * sizeof(int);
     cudaFuncSetAttribute(meta_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    meta_place_kernel<<<n_chunks, kMetaPlaceThreads, smem, s>>>(top, NK, E, chunk_counts,
+    MOE_TRACED("meta_place", s, (meta_place_kernel<<<n_chunks, kMetaPlaceThreads, smem, s>>>(top, NK, E, chunk_counts,
                                                                 sorted_start, padded_start, indices,
-                                                                bin_ids, pos);
+                                                                bin_ids, pos)));
     MOE_LAUNCH_CHECK();
   }
   return MOE_OK;

@@ -293,8 +293,8 @@ template <typename T>
 static moe_status permute_t(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* pb,
                             int N, int H, int E, int K, void* x_perm, cudaStream_t s) {
   const int64_t work = (int64_t)N > (int64_t)E * kTile ? N : (int64_t)E * kTile;
-  permute_kernel<T><<<row_grid(work), kRowThreads, 0, s>>>((const T*)x, pos, bins, pb, N, H, E, K,
-                                                           (T*)x_perm);
+  MOE_TRACED("permute", s, (permute_kernel<T><<<row_grid(work), kRowThreads, 0, s>>>((const T*)x, pos, bins, pb, N, H, E, K,
+                                                           (T*)x_perm)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -308,7 +308,7 @@ moe_status permute_rows(const void* x, const int32_t* pos, const int32_t* bins, 
 template <typename T>
 static moe_status combine_t(const void* out, const float* w, const int32_t* pos, int N, int K, int H,
                             void* y, cudaStream_t s) {
-  combine_kernel<T><<<row_grid(N), kRowThreads, 0, s>>>((const T*)out, w, pos, N, K, H, (T*)y);
+  MOE_TRACED("combine", s, (combine_kernel<T><<<row_grid(N), kRowThreads, 0, s>>>((const T*)out, w, pos, N, K, H, (T*)y)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -324,8 +324,8 @@ static moe_status combine_bwd_t(const void* dy, const void* out, const float* w,
                                 const int32_t* bins, const int32_t* pb, int N, int K, int H, int E,
                                 float* dw, float* dlogit, void* d_out, cudaStream_t s) {
   const int64_t work = (int64_t)N > (int64_t)E * kTile ? N : (int64_t)E * kTile;
-  combine_bwd_kernel<T><<<row_grid(work), kRowThreads, 0, s>>>(
-      (const T*)dy, (const T*)out, w, pos, bins, pb, N, K, H, E, dw, dlogit, (T*)d_out);
+  MOE_TRACED("combine_bwd", s, (combine_bwd_kernel<T><<<row_grid(work), kRowThreads, 0, s>>>(
+      (const T*)dy, (const T*)out, w, pos, bins, pb, N, K, H, E, dw, dlogit, (T*)d_out)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -341,10 +341,10 @@ moe_status combine_bwd_rows(const void* dy, const void* out, const float* w, con
 moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s) {
   dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R, 32)), block(32, 8);
   if (dt == MOE_F32)
-    transpose_kernel<float><<<grid, block, 0, s>>>((const float*)in, R, C, (float*)outT);
+    MOE_TRACED("transpose", s, (transpose_kernel<float><<<grid, block, 0, s>>>((const float*)in, R, C, (float*)outT)));
   else
-    transpose_kernel<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)in, R, C,
-                                                           (__nv_bfloat16*)outT);
+    MOE_TRACED("transpose", s, (transpose_kernel<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)in, R, C,
+                                                           (__nv_bfloat16*)outT)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -363,16 +363,16 @@ static moe_status unpermute_router_bwd_t(const void* dx_perm, const float* dlogi
   float* part = (float*)((char*)scratch + (size_t)E * H * 4);
   moe_status st = transpose_matrix(W_r, H, E, sizeof(T) == 4 ? MOE_F32 : MOE_BF16, WrT, s);
   if (st != MOE_OK) return st;
-  unpermute_dx_kernel<T><<<row_grid(N), kRowThreads, 0, s>>>((const T*)dx_perm, dlogit, WrT, top, pos,
-                                                             N, H, K, (T*)dx);
+  MOE_TRACED("unpermute_dx", s, (unpermute_dx_kernel<T><<<row_grid(N), kRowThreads, 0, s>>>((const T*)dx_perm, dlogit, WrT, top, pos,
+                                                             N, H, K, (T*)dx)));
   MOE_LAUNCH_CHECK();
   constexpr int V = Vec<T>::N;
   dim3 g1((unsigned)(P / kTile), (unsigned)cdiv(H, kRowThreads * V));
-  router_wgrad_partial_kernel<T><<<g1, kRowThreads, 0, s>>>(dlogit, (const T*)x, indices, bins,
-                                                            padded_bins, E, H, K, part);
+  MOE_TRACED("router_wgrad_partial", s, (router_wgrad_partial_kernel<T><<<g1, kRowThreads, 0, s>>>(dlogit, (const T*)x, indices, bins,
+                                                            padded_bins, E, H, K, part)));
   MOE_LAUNCH_CHECK();
   dim3 g2((unsigned)cdiv(H, 256), (unsigned)E);
-  router_wgrad_reduce_kernel<T><<<g2, 256, 0, s>>>(part, padded_bins, E, H, (T*)dWr);
+  MOE_TRACED("router_wgrad_reduce", s, (router_wgrad_reduce_kernel<T><<<g2, 256, 0, s>>>(part, padded_bins, E, H, (T*)dWr)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

@@ -115,8 +115,9 @@ static moe_status launch_route_simt(const T* x, const T* W_r, int N, int H, int 
   if (E <= EM) {                                                                               \
     cudaFuncSetAttribute(route_simt_kernel<T, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                          (int)smem);                                                           \
-    route_simt_kernel<T, EM><<<blocks, threads, smem, s>>>(x, W_r, N, H, E, K, logits, probs,  \
-                                                           top, w);                            \
+    MOE_TRACED("route_simt", s,                                                                 \
+               (route_simt_kernel<T, EM><<<blocks, threads, smem, s>>>(x, W_r, N, H, E, K, logits,  \
+                                                                       probs, top, w)));       \
     MOE_LAUNCH_CHECK();                                                                        \
     return MOE_OK;                                                                             \
   }

@@ -218,6 +218,15 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                          int32_t F, moe_dtype dt, void* dx, void* dW_r, void* dW1, void* dW3,
                          void* dW2, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Per-launch timing.  While attached, every kernel launch made by any entry
+ * point records events[2*i] on its stream just before launch i and
+ * events[2*i+1] just after it, stores a static kernel name in labels[i]
+ * (labels may be NULL) and increments *count (host memory), for up to
+ * `capacity` launches.  The caller creates the events (cudaEvent_t, timing
+ * enabled) and owns every buffer.  Process-wide, not thread-safe. */
+moe_status moe_trace_attach(void* const* events, int32_t capacity, const char** labels, int32_t* count);
+moe_status moe_trace_detach(void);
+
 #ifdef __cplusplus
 }
 #endif
