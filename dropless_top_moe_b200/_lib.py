@@ -43,6 +43,7 @@ SIGNATURES = {
                             P, SZ, P]),
     "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
                             P, P, P, P, P, P, SZ, P]),
+    "moe_dispatch_meta_noalloc": (I32, [P, I32, I32, I32, P, P, P, P, P, P, P]),
     "moe_trace_attach": (I32, [P, I32, P, P]),
     "moe_trace_detach": (I32, []),
 }

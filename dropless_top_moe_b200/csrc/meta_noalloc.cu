@@ -1,0 +1,56 @@
+// Dispatch metadata without a caller workspace (moe_dispatch_meta_noalloc).
+//
+// Some callers cannot call cudaMalloc: code embedded in another runtime that
+// owns all device memory and gives its plugins no allocator, or a
+// latency-critical path where an allocation (which may synchronise the
+// device) is not allowed.  This entry point keeps the metadata kernels'
+// scratch (per-chunk expert counts and the per-expert starts) in a fixed
+// file-scope device array instead of a workspace.  The caller still passes
+// every input and output.
+//
+// The array is sized for n_chunks * E <= kNoAllocChunkExperts, where
+// n_chunks = ceil(N*K / 2048); with E = 256 that is N*K <= 1,048,576.  Every
+// device that loads the library holds the array (about 514 KB) until exit.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+constexpr int kNoAllocChunkExperts = 131072;
+constexpr int kNoAllocScratchInts = kNoAllocChunkExperts + 2 * 256;
+
+// Shared by every call on a device; keeps the last call's contents.
+__device__ __align__(256) int32_t g_meta_scratch[kNoAllocScratchInts];
+
+// Device address of g_meta_scratch per device, looked up on first use.
+void* g_scratch_addr[64] = {nullptr};
+
+}  // namespace
+
+extern "C" moe_status moe_dispatch_meta_noalloc(const int32_t* top_experts, int32_t N, int32_t K,
+                                                int32_t E, int32_t* indices, int32_t* bin_ids,
+                                                int32_t* bins, int32_t* padded_bins, int32_t* pos,
+                                                int32_t* status, moe_stream_t stream) {
+  if (N < 0 || K <= 0 || E <= 0 || K > E) return MOE_ERR_INVALID_ARG;
+  if (E > 256) return MOE_ERR_UNSUPPORTED;
+  if (!padded_bins || (N > 0 && (!top_experts || !pos))) return MOE_ERR_INVALID_ARG;
+  const int64_t NK = (int64_t)N * K;
+  if (moe::meta_workspace_bytes(NK, E) > sizeof(g_meta_scratch)) return MOE_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  if (!g_scratch_addr[dev]) {
+    // set-up, once per device, with that device current: the array's name is
+    // a host-side stand-in, so the kernels get its device address instead
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_meta_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  // The count kernel writes every chunk count (zeros included) and the scan
+  // writes every start, so nothing in the array needs clearing first.
+  return moe::dispatch_meta(top_experts, NK, E, indices, bin_ids, bins, padded_bins, pos,
+                            g_scratch_addr[dev], status, (cudaStream_t)stream);
+}

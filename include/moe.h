@@ -127,6 +127,30 @@ moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, i
                              int32_t* padded_bins, int32_t* pos, void* ws, size_t ws_bytes,
                              moe_stream_t stream);
 
+/* Dispatch metadata for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this entry point.  Some callers cannot call
+ * cudaMalloc: code embedded in another runtime that owns all device memory
+ * and gives its plugins no allocator, or a latency-critical path where an
+ * allocation (which may synchronise the device) is not allowed.  Same
+ * outputs as moe_dispatch_meta, but the scratch lives in a fixed device
+ * array inside the library (about 514 KB per device that loads it, held
+ * until exit) instead of a workspace; the caller still passes every input
+ * and output.
+ *   Limit: ceil(N*K / 2048) * E <= 131072 (with E = 256: N*K <= 1048576);
+ *   larger sizes return MOE_ERR_WORKSPACE before any device work.
+ *   status: NULL, or a device int32 the caller zeroed; MOE_DEVERR_* bits are
+ *   OR-ed into it.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  All calls on a device share the one array,
+ *   which keeps the last call's contents: calls that overlap on the GPU (on
+ *   different streams without ordering) race and give wrong results.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+moe_status moe_dispatch_meta_noalloc(const int32_t* top_experts, int32_t N, int32_t K, int32_t E,
+                                     int32_t* indices, int32_t* bin_ids, int32_t* bins,
+                                     int32_t* padded_bins, int32_t* pos, int32_t* status,
+                                     moe_stream_t stream);
+
 /* Padded gather (MegaBlocks sec. 2.1): x_perm[pos[t*K+k], :] = x[t, :]; the
  * pad rows of every expert group (count..round_up(count,128)) are zeroed.
  *   x [N,H]; x_perm [P,H] with P >= padded_bins[E-1] (dt); bins, padded_bins [E]. */
