@@ -36,7 +36,8 @@ namespace umma {
 
 constexpr int BM = 128;
 constexpr int BK = 64;              // one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;              // two warps per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kA_BYTES = BM * BK * 2;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr int kGroupM = 8;          // M tiles per raster group (L2 reuse of B panels)
@@ -77,14 +78,46 @@ struct Tile {
   int m0;          // WGRAD: first output row (of the weight gradient)
   int n0;          // first output column (per output matrix)
   int nkb;         // k-blocks of BK
+  int halves;      // 128-row halves of the M tile in use (1 or 2)
 };
 
-template <int SCHED, int BN, int EPI>
-__device__ __forceinline__ int64_t total_tiles(const Params& p) {
+// Compile-time shape of one kernel instance.  MT = 128-row M halves per tile:
+// with MT = 2 two M=128 MMAs share every B tile, so a 256 x BN tile moves
+// (2*128 + BN) rows of operands per k-step instead of (128 + BN) per half.
+template <int BN, int MT>
+struct Shape {
+  static constexpr int A_BYTES = MT * BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int ACC_COLS = MT * BN;                       // one accumulator set
+  static constexpr int ACC_BUFS = 2 * ACC_COLS <= 512 ? 2 : 1;   // double-buffer when it fits
+  static constexpr int USED_COLS = ACC_BUFS * ACC_COLS;
+  static constexpr uint32_t TMEM_COLS =
+      USED_COLS <= 32 ? 32 : (USED_COLS <= 64 ? 64 : (USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512)));
+  static constexpr int N_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + 8 * N_BARS + 16 + 4 * 260;
+};
+
+// Rows of the grouped buffers actually used, clamped to the buffers' rows.
+__device__ __forceinline__ int64_t used_rows(const Params& p) {
+  int64_t rows = p.padded_bins[p.E - 1];
+  return rows > p.P ? p.P : rows;
+}
+
+// Number of M units for the ROWS schedule: 128-row tiles (MT = 1) or pairs
+// of 128-row tiles of the same expert (MT = 2; an odd last tile of an expert
+// forms a unit of one half).  s_unit_start[e] = first unit of expert e.
+template <int MT>
+__device__ __forceinline__ int64_t rows_units(const Params& p, const int32_t* s_unit_start) {
+  if constexpr (MT == 1) return used_rows(p) / BM;
+  return s_unit_start[p.E];
+}
+
+template <int SCHED, int BN, int MT, int EPI>
+__device__ __forceinline__ int64_t total_tiles(const Params& p, const int32_t* s_unit_start) {
   if constexpr (SCHED == SCHED_ROWS) {
-    int64_t rows = p.padded_bins[p.E - 1];
-    if (rows > p.P) rows = p.P;
-    return (rows / BM) * p.n_tiles;
+    return rows_units<MT>(p, s_unit_start) * p.n_tiles;
   } else if constexpr (SCHED == SCHED_WGRAD) {
     return (int64_t)p.E * p.m_tiles_w * p.n_tiles;
   } else {
@@ -92,23 +125,37 @@ __device__ __forceinline__ int64_t total_tiles(const Params& p) {
   }
 }
 
-template <int SCHED, int BN, int EPI>
-__device__ __forceinline__ Tile get_tile(const Params& p, int64_t t) {
+template <int SCHED, int BN, int MT, int EPI>
+__device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32_t* s_unit_start) {
   constexpr int NOUT = (EPI == EPI_SWIGLU || EPI == EPI_WGRAD_PAIR) ? BN / 2 : BN;
   Tile tl;
   if constexpr (SCHED == SCHED_ROWS) {
-    int64_t rows = p.padded_bins[p.E - 1];
-    if (rows > p.P) rows = p.P;
-    const int64_t num_m = rows / BM;
+    const int64_t num_m = rows_units<MT>(p, s_unit_start);
     const int64_t per_group = (int64_t)kGroupM * p.n_tiles;
     const int64_t g = t / per_group;
     const int64_t first_m = g * kGroupM;
     const int64_t gm = (num_m - first_m) < kGroupM ? (num_m - first_m) : kGroupM;
     const int64_t local = t - g * per_group;
-    const int64_t mt = first_m + local % gm;
+    const int64_t mu = first_m + local % gm;          // M unit
     const int64_t nt = local / gm;
-    tl.row0 = mt * BM;
-    tl.e = expert_of_row(p.padded_bins, p.E, tl.row0);
+    if constexpr (MT == 1) {
+      tl.row0 = mu * BM;
+      tl.e = expert_of_row(p.padded_bins, p.E, tl.row0);
+      tl.halves = 1;
+    } else {
+      // expert = last e with s_unit_start[e] <= mu
+      int lo = 0, hi = p.E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)s_unit_start[mid] <= mu) lo = mid; else hi = mid - 1;
+      }
+      tl.e = lo;
+      const int64_t pstart = tl.e ? p.padded_bins[tl.e - 1] : 0;
+      const int64_t ntile_e = (p.padded_bins[tl.e] - pstart) / BM;
+      const int64_t k = mu - s_unit_start[tl.e];
+      tl.row0 = pstart + k * 2 * BM;
+      tl.halves = (ntile_e - 2 * k) >= 2 ? 2 : 1;
+    }
     tl.m0 = 0;
     tl.n0 = (int)(nt * NOUT);
     tl.nkb = p.kdim / BK;
@@ -116,19 +163,21 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t) {
     const int64_t per_e = (int64_t)p.m_tiles_w * p.n_tiles;
     tl.e = (int)(t / per_e);
     const int64_t r = t - (int64_t)tl.e * per_e;
-    tl.m0 = (int)((r / p.n_tiles) * BM);
+    tl.m0 = (int)((r / p.n_tiles) * BM * MT);
     tl.n0 = (int)((r % p.n_tiles) * NOUT);
     const int64_t lo = tl.e ? p.padded_bins[tl.e - 1] : 0;
     int64_t hi = p.padded_bins[tl.e];
     if (hi > p.P) hi = p.P;
     tl.row0 = lo;
     tl.nkb = hi > lo ? (int)((hi - lo) / BK) : 0;
+    tl.halves = MT;
   } else {
     tl.e = 0;
     tl.row0 = t * BM;
     tl.m0 = 0;
     tl.n0 = 0;
     tl.nkb = p.kdim / BK;
+    tl.halves = 1;
   }
   return tl;
 }
@@ -169,14 +218,158 @@ __device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals
   }
 }
 
-template <int BN, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
+// Epilogue of one 128-row half: TMEM columns [tacc, tacc + BN) of this
+// thread's row -> fused math -> global memory.
+template <int BN, int SCHED, int EPI>
+__device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, uint32_t tacc, int row,
+                                              int part) {
+  const int64_t grow = tl.row0 + row;                 // ROWS/DENSE global row
+  // the two warps of a lane quarter split the columns: part 0 / part 1
+  constexpr int NC = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
+  const int c_begin = part * (NC / 2), c_end = c_begin + NC / 2;
+  if constexpr (EPI == EPI_SWIGLU) {
+    __nv_bfloat16* act = p.out0 + grow * p.ldo + tl.n0;
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; c += 32) {
+      uint32_t g[32], u[32];
+      tmem_ld_32(tacc + c, g);
+      tmem_ld_32(tacc + BN / 2 + c, u);
+      tmem_ld_wait();
+      float a[32], gf[32], uf[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        gf[j] = __uint_as_float(g[j]);
+        uf[j] = __uint_as_float(u[j]);
+        a[j] = silu_f(gf[j]) * uf[j];
+      }
+      store_row_bf16x32(act + c, a);
+      if (p.out1) {
+        store_row_bf16x32(p.out1 + grow * p.ldo + tl.n0 + c, gf);
+        store_row_bf16x32(p.out2 + grow * p.ldo + tl.n0 + c, uf);
+      }
+    }
+  } else if constexpr (EPI == EPI_STORE) {
+    __nv_bfloat16* dst = p.out0 + grow * p.ldo + tl.n0;
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      tmem_ld_wait();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      store_row_bf16x32(dst + c, v);
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+    const int64_t off = grow * p.ldo + tl.n0;
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      float gf[32], uf[32], dg[32], du[32];
+      load_row_bf16x32(p.aux0 + off + c, gf);
+      load_row_bf16x32(p.aux1 + off + c, uf);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float da = __uint_as_float(r[j]);
+        const float sig = 1.f / (1.f + expf(-gf[j]));
+        dg[j] = da * uf[j] * sig * (1.f + gf[j] * (1.f - sig));
+        du[j] = da * gf[j] * sig;
+      }
+      store_row_bf16x32(p.out0 + off + c, dg);
+      store_row_bf16x32(p.out1 + off + c, du);
+    }
+  } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) {
+    const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      tmem_ld_wait();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      if (EPI == EPI_WGRAD_PAIR && c >= BN / 2)
+        store_row_bf16x32(p.out1 + off + (c - BN / 2), v);
+      else
+        store_row_bf16x32(p.out0 + off + c, v);
+    }
+  } else {  // EPI_ROUTER: softmax, top-K, renormalise on this row's E logits
+    if (part != 0) return;
+    constexpr int KMAX = 16;
+    const int E = p.n_mma, K = p.K;
+    const bool live = grow < p.P;
+    float vals[KMAX];
+    int ids[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
+    float m = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < E; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (c + j < E) {
+          const float v = __uint_as_float(r[j]);
+          m = fmaxf(m, v);
+          topk_insert<KMAX>(v, c + j, K, vals, ids);
+          if (live && p.logits) p.logits[grow * E + c + j] = v;
+        }
+      }
+    }
+    if (p.probs) {
+      float Z = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < E; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32(tacc + c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c + j < E) Z += expf(__uint_as_float(r[j]) - m);
+      }
+#pragma unroll 1
+      for (int c = 0; c < E; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32(tacc + c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (live && c + j < E) p.probs[grow * E + c + j] = expf(__uint_as_float(r[j]) - m) / Z;
+      }
+    }
+    if (live) {
+      float S = 0.f, ev[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        ev[j] = (j < K) ? expf(vals[j] - vals[0]) : 0.f;
+        S += ev[j];
+      }
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j < K) {
+          p.top[grow * K + j] = ids[j];
+          p.weights[grow * K + j] = ev[j] / S;
+        }
+      }
+    }
+  }
+}
+
+template <int BN, int MT, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
-  constexpr int B_BYTES = BN * BK * 2;
-  constexpr int STAGE_BYTES = kA_BYTES + B_BYTES;
-  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
-  constexpr uint32_t TMEM_COLS = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
+  using S = Shape<BN, MT>;
+  constexpr int STAGES = S::STAGES;
+  constexpr int STAGE_BYTES = S::STAGE_BYTES;
+  constexpr int A_BYTES = S::A_BYTES;
+  constexpr int ACC_BUFS = S::ACC_BUFS;
+  constexpr int ACC_COLS = S::ACC_COLS;
   static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte swizzle atoms aligned");
   static_assert(STAGES >= 2, "pipeline needs at least two stages");
+  static_assert(MT == 1 || SCHED != SCHED_DENSE, "the router uses single 128-row tiles");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -186,19 +379,44 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
   auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + a); };
-  auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + 2 + a); };
-  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 4);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5));
+  auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + ACC_BUFS + a); };
+  const uint32_t drain_bar = bar_base + 8u * (2 * STAGES + 2 * ACC_BUFS);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * S::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int32_t* s_unit_start = reinterpret_cast<int32_t*>(tmem_holder + 4);   // [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), 4); }
+    for (int a = 0; a < ACC_BUFS; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), kEpiWarps); }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
+  }
+  if (SCHED == SCHED_ROWS && MT == 2 && warp == 2) {
+    // units per expert = ceil(tiles_e / 2); exclusive scan over experts
+    int carry = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int e = e0 + lane;
+      int u = 0;
+      if (e < p.E) {
+        const int64_t lo = e ? p.padded_bins[e - 1] : 0;
+        int64_t hi = p.padded_bins[e];
+        if (hi > p.P) hi = p.P;
+        const int64_t tiles = hi > lo ? (hi - lo) / BM : 0;
+        u = (int)((tiles + 1) / 2);
+      }
+      int incl = u;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < p.E) s_unit_start[e] = carry + incl - u;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_unit_start[p.E] = carry;
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.ta0);
@@ -207,35 +425,36 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     if (SPLIT == SPLIT_K) tma_prefetch_desc(&p.ta1);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_holder), S::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int64_t ntiles = total_tiles<SCHED, BN, EPI>(p);
+  const int64_t ntiles = total_tiles<SCHED, BN, MT, EPI>(p, s_unit_start);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const uint32_t tx = kA_BYTES + (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)B_BYTES);
       bool ok = true;
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = get_tile<SCHED, BN, EPI>(p, t);
+        const Tile tl = get_tile<SCHED, BN, MT, EPI>(p, t, s_unit_start);
+        const uint32_t tx = (uint32_t)tl.halves * BM * BK * 2 +
+                            (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)S::B_BYTES);
         for (int kb = 0; kb < tl.nkb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
           const uint32_t sa = base + stage * STAGE_BYTES;
-          const uint32_t sb = sa + kA_BYTES;
+          const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = full_bar(stage);
           mbar_expect_tx(fb, tx);
           if constexpr (SCHED == SCHED_WGRAD) {
             const int krow = (int)(tl.row0 + (int64_t)kb * BK);
-            // A = X^T tile: two 64-wide MN boxes of the [rows, M] matrix
-            tma_load_2d(sa, &p.ta0, fb, tl.m0, krow);
-            tma_load_2d(sa + 8192, &p.ta0, fb, tl.m0 + 64, krow);
+            // A = X^T: 64-wide MN boxes of the [rows, M] matrix, 2 per half
+#pragma unroll
+            for (int j = 0; j < 2 * MT; ++j) tma_load_2d(sa + j * 8192, &p.ta0, fb, tl.m0 + 64 * j, krow);
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j) {
               if (SPLIT == SPLIT_N && j >= BN / 128)
@@ -249,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
             const CUtensorMap* tb = &p.tb0;
             if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
             tma_load_2d(sa, ta, fb, k, (int)tl.row0);
+            if (MT == 2 && tl.halves == 2) tma_load_2d(sa + BM * BK * 2, ta, fb, k, (int)tl.row0 + BM);
             if constexpr (SCHED == SCHED_DENSE) {
               tma_load_2d(sb, tb, fb, k, 0);
             } else if constexpr (B_MN) {
@@ -268,11 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       }
       if (!ok) {
         // give the loads already issued a bounded chance to land
-        for (int s = 0; s < STAGES; ++s) {
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(full_bar(s), 0) && !mbar_try_wait(full_bar(s), 1) &&
-                 globaltimer() - t0 < 50000000ull) {}
-        }
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 20000000ull) {}
       }
     }
   } else if (warp == 1) {
@@ -286,28 +503,35 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = get_tile<SCHED, BN, EPI>(p, t);
+        const Tile tl = get_tile<SCHED, BN, MT, EPI>(p, t, s_unit_start);
         if (tl.nkb == 0) continue;
         if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
         for (int kb = 0; kb < tl.nkb; ++kb) {
           if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = base + stage * STAGE_BYTES;
-          const uint32_t sb = sa + kA_BYTES;
+          const uint32_t sb = sa + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = A_MN ? desc_mn_sw128(sa + kk * 2048, 8192) : desc_k_sw128(sa + kk * 32);
             const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
-            mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+#pragma unroll
+            for (int h = 0; h < MT; ++h) {
+              if (h < tl.halves) {
+                const uint32_t ah = sa + h * (BM * BK * 2);
+                const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
+                mma_bf16(d_tmem + h * BN, ad, bd, idesc, accum);
+              }
+            }
           }
           mma_commit(empty_bar(stage));      // smem slot free once these MMAs are done
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         mma_commit(tfull_bar(acc));          // accumulator ready for the epilogue
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) {
         mma_commit(drain_bar);
@@ -318,23 +542,28 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                       // TMEM lane quarter of this warp
-    const int row = q * 32 + lane;                // row inside the 128-row tile
+    const int part = (warp - 2) >> 2;             // which half of the columns
+    const int row = q * 32 + lane;                // row inside a 128-row half
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const Tile tl = get_tile<SCHED, BN, EPI>(p, t);
+      const Tile tl = get_tile<SCHED, BN, MT, EPI>(p, t, s_unit_start);
       if constexpr (SCHED == SCHED_WGRAD) {
         if (tl.nkb == 0) {                        // expert with no rows: zero gradient
           const float z[32] = {0.f};
-          if constexpr (EPI == EPI_WGRAD_PAIR) {
-            __nv_bfloat16* d0 = p.out0 + (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
-            __nv_bfloat16* d1 = p.out1 + (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
-#pragma unroll
-            for (int c = 0; c < BN / 2; c += 32) { store_row_bf16x32(d0 + c, z); store_row_bf16x32(d1 + c, z); }
-          } else {
-            __nv_bfloat16* d0 = p.out0 + (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
-#pragma unroll
-            for (int c = 0; c < BN; c += 32) store_row_bf16x32(d0 + c, z);
+#pragma unroll 1
+          for (int h = 0; h < MT; ++h) {
+            const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + h * BM + row) * p.ldo + tl.n0;
+            if constexpr (EPI == EPI_WGRAD_PAIR) {
+#pragma unroll 1
+              for (int c = part * (BN / 4); c < (part + 1) * (BN / 4); c += 32) {
+                store_row_bf16x32(p.out0 + off + c, z);
+                store_row_bf16x32(p.out1 + off + c, z);
+              }
+            } else {
+#pragma unroll 1
+              for (int c = part * (BN / 2); c < (part + 1) * (BN / 2); c += 32) store_row_bf16x32(p.out0 + off + c, z);
+            }
           }
           continue;
         }
@@ -344,142 +573,17 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int64_t grow = tl.row0 + row;         // ROWS/DENSE global row
-
-      if constexpr (EPI == EPI_SWIGLU) {
-        __nv_bfloat16* act = p.out0 + grow * p.ldo + tl.n0;
 #pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld_32(tacc + c, g);
-          tmem_ld_32(tacc + BN / 2 + c, u);
-          tmem_ld_wait();
-          float a[32], gf[32], uf[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            gf[j] = __uint_as_float(g[j]);
-            uf[j] = __uint_as_float(u[j]);
-            a[j] = silu_f(gf[j]) * uf[j];
-          }
-          store_row_bf16x32(act + c, a);
-          if (p.out1) {
-            store_row_bf16x32(p.out1 + grow * p.ldo + tl.n0 + c, gf);
-            store_row_bf16x32(p.out2 + grow * p.ldo + tl.n0 + c, uf);
-          }
-        }
-      } else if constexpr (EPI == EPI_STORE) {
-        __nv_bfloat16* dst = p.out0 + grow * p.ldo + tl.n0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32(tacc + c, r);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          store_row_bf16x32(dst + c, v);
-        }
-      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-        const int64_t off = grow * p.ldo + tl.n0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32(tacc + c, r);
-          float gf[32], uf[32], dg[32], du[32];
-          load_row_bf16x32(p.aux0 + off + c, gf);
-          load_row_bf16x32(p.aux1 + off + c, uf);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float da = __uint_as_float(r[j]);
-            const float sig = 1.f / (1.f + expf(-gf[j]));
-            dg[j] = da * uf[j] * sig * (1.f + gf[j] * (1.f - sig));
-            du[j] = da * gf[j] * sig;
-          }
-          store_row_bf16x32(p.out0 + off + c, dg);
-          store_row_bf16x32(p.out1 + off + c, du);
-        }
-      } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) {
-        const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32(tacc + c, r);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (EPI == EPI_WGRAD_PAIR && c >= BN / 2)
-            store_row_bf16x32(p.out1 + off + (c - BN / 2), v);
-          else
-            store_row_bf16x32(p.out0 + off + c, v);
-        }
-      } else {  // EPI_ROUTER: softmax, top-K, renormalise on this row's E logits
-        constexpr int KMAX = 16;
-        const int E = p.n_mma, K = p.K;
-        const bool live = grow < p.P;
-        float vals[KMAX];
-        int ids[KMAX];
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
-        float m = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < E; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32(tacc + c, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (c + j < E) {
-              const float v = __uint_as_float(r[j]);
-              m = fmaxf(m, v);
-              topk_insert<KMAX>(v, c + j, K, vals, ids);
-              if (live && p.logits) p.logits[grow * E + c + j] = v;
-            }
-          }
-        }
-        if (p.probs) {
-          float Z = 0.f;
-#pragma unroll 1
-          for (int c = 0; c < E; c += 32) {
-            uint32_t r[32];
-            tmem_ld_32(tacc + c, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c + j < E) Z += expf(__uint_as_float(r[j]) - m);
-          }
-#pragma unroll 1
-          for (int c = 0; c < E; c += 32) {
-            uint32_t r[32];
-            tmem_ld_32(tacc + c, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (live && c + j < E) p.probs[grow * E + c + j] = expf(__uint_as_float(r[j]) - m) / Z;
-          }
-        }
-        if (live) {
-          float S = 0.f, ev[KMAX];
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j) {
-            ev[j] = (j < K) ? expf(vals[j] - vals[0]) : 0.f;
-            S += ev[j];
-          }
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j) {
-            if (j < K) {
-              p.top[grow * K + j] = ids[j];
-              p.weights[grow * K + j] = ev[j] / S;
-            }
-          }
-        }
+      for (int h = 0; h < tl.halves; ++h) {
+        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
+        Tile th = tl;
+        if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + h * BM; else th.row0 = tl.row0 + h * BM;
+        epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
@@ -488,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
 }
 
@@ -552,19 +656,17 @@ static int sm_count() {
   return cache[dev];
 }
 
-template <int BN, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
+template <int BN, int MT, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
 static moe_status launch(const char* name, const Params& p, int64_t tiles_upper, cudaStream_t s) {
-  constexpr int STAGE_BYTES = kA_BYTES + BN * BK * 2;
-  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
-  const size_t smem = (size_t)STAGES * STAGE_BYTES + 1024 + 8 * (2 * STAGES + 5) + 16;
-  auto kern = umma_gemm_kernel<BN, SCHED, EPI, A_MN, B_MN, SPLIT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+  using S = Shape<BN, MT>;
+  auto kern = umma_gemm_kernel<BN, MT, SCHED, EPI, A_MN, B_MN, SPLIT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
   }
   int64_t grid = tiles_upper < sm_count() ? tiles_upper : sm_count();
   if (grid < 1) grid = 1;
-  MOE_TRACED(name, s, (kern<<<(unsigned)grid, kThreads, smem, s>>>(p)));
+  MOE_TRACED(name, s, (kern<<<(unsigned)grid, kThreads, S::SMEM, s>>>(p)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -602,7 +704,10 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.out1 = gate_up ? (bf*)gate_up : nullptr;
     p.out2 = gate_up ? (bf*)gate_up + (size_t)P * F : nullptr;
     p.ldo = F;
-    moe_status st = launch<256, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p, (P / BM) * p.n_tiles, s);
+    // 128-row tiles: the SwiGLU epilogue (up to three outputs) stays hidden
+    // behind the next tile's main loop only with two accumulator buffers
+    moe_status st = launch<256, 1, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p,
+                                                                              (P / BM) * p.n_tiles, s);
     if (st != MOE_OK) return st;
   }
   // GEMM2: out = act * W2_e
@@ -615,8 +720,9 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.n_tiles = H / bn;
     p.out0 = (bf*)out;
     p.ldo = H;
-    if (bn == 256) return launch<256, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
-    return launch<128, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
+    if (bn == 256)
+      return launch<256, 2, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
+    return launch<128, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
   }
 }
 
@@ -644,41 +750,48 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.out0 = dG;
     p.out1 = dU;
     p.ldo = F;
-    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, (P / BM) * p.n_tiles, s)
-                   : launch<128, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, (P / BM) * p.n_tiles, s);
+    const int64_t up = (P / BM) * p.n_tiles;
+    // 128-row tiles for the same reason as GEMM1 (the epilogue reads G, U and
+    // writes dG, dU)
+    st = bn == 256 ? launch<256, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s)
+                   : launch<128, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s);
     if (st != MOE_OK) return st;
   }
   // dW2_e = act_e^T * d_out_e   [F, H]
   {
     Params p = blank_params(pb, E, P, status);
     const int bn = (H % 256 == 0) ? 256 : 128;
+    const int mt = (bn == 256 && F % 256 == 0) ? 2 : 1;
     if (!map2d(&p.ta0, act, F, P, F, 64, 64) || !map2d(&p.tb0, d_out, H, P, H, 64, 64)) return MOE_ERR_CUDA;
     p.n_mma = bn;
-    p.m_tiles_w = F / BM;
+    p.m_tiles_w = F / (BM * mt);
     p.n_tiles = H / bn;
     p.out0 = (bf*)dW2;
     p.ldo = H;
     p.out_estride = (int64_t)F * H;
     const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
-    st = bn == 256 ? launch<256, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s)
-                   : launch<128, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
+    if (mt == 2) st = launch<256, 2, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
+    else if (bn == 256) st = launch<256, 1, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
+    else st = launch<128, 1, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
     if (st != MOE_OK) return st;
   }
   // dW1_e | dW3_e = x_perm_e^T * [dG_e | dU_e]   [H, F] each
   {
     Params p = blank_params(pb, E, P, status);
+    const int mt = (H % 256 == 0) ? 2 : 1;
     if (!map2d(&p.ta0, x_perm, H, P, H, 64, 64) || !map2d(&p.tb0, dG, F, P, F, 64, 64) ||
         !map2d(&p.tb1, dU, F, P, F, 64, 64))
       return MOE_ERR_CUDA;
     p.n_mma = 256;
-    p.m_tiles_w = H / BM;
+    p.m_tiles_w = H / (BM * mt);
     p.n_tiles = F / 128;
     p.out0 = (bf*)dW1;
     p.out1 = (bf*)dW3;
     p.ldo = F;
     p.out_estride = (int64_t)H * F;
     const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
-    st = launch<256, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
+    st = mt == 2 ? launch<256, 2, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s)
+                 : launch<256, 1, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
     if (st != MOE_OK) return st;
   }
   // dx_perm = dG * W1_e^T + dU * W3_e^T  (one K = 2F contraction)
@@ -694,8 +807,9 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.n_tiles = H / bn;
     p.out0 = (bf*)dx_perm;
     p.ldo = H;
-    st = bn == 256 ? launch<256, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, (P / BM) * p.n_tiles, s)
-                   : launch<128, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, (P / BM) * p.n_tiles, s);
+    const int64_t up = (P / BM) * p.n_tiles;
+    st = bn == 256 ? launch<256, 2, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s)
+                   : launch<128, 1, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s);
     if (st != MOE_OK) return st;
   }
   return MOE_OK;
@@ -724,7 +838,7 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   p.probs = probs;
   p.top = top;
   p.weights = w;
-  return launch<256, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
+  return launch<256, 1, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
 }
 
 }  // namespace moe

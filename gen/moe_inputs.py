@@ -55,16 +55,17 @@ class MoEShape:
 
 # The five workloads.  Sizes, dtype and the skew intent follow the layer's
 # benchmark description; the bias scales below are input recipe constants:
-#  * fine_grained: sigma = 1.0 makes per-expert counts span from a handful
-#    to several hundred tokens (MoonEP benchmark shapes, section 05, use the
-#    same H=7168, K=8, H'=2048 geometry).
+#  * fine_grained: sigma = 0.75 makes per-expert counts span from a handful
+#    (seed 0: 7) to several hundred tokens (median 163, a few above 1000), so
+#    many groups are a single padded tile (MoonEP benchmark shapes, section
+#    05, use the same H=7168, K=8, H'=2048 geometry).
 #  * skewed_zipf: b_e = -tau * 1.2 * ln(rank_e), a Zipf(s=1.2) popularity
 #    profile over a seeded random expert ranking (MoonEP maxvio, section 01).
 WORKLOADS = {
     "tiny_fp32": MoEShape("tiny_fp32", N=256, H=128, E=4, K=2, F=256, dtype="f32"),
     "mixtral": MoEShape("mixtral", N=4096, H=4096, E=8, K=2, F=14336),
     "fine_grained": MoEShape("fine_grained", N=8192, H=7168, E=256, K=8, F=2048,
-                             skew="normal", skew_param=1.0),
+                             skew="normal", skew_param=0.75),
     "skewed_zipf": MoEShape("skewed_zipf", N=16384, H=2048, E=64, K=6, F=1408,
                             skew="zipf", skew_param=1.0),
     "train_step": MoEShape("train_step", N=16384, H=4096, E=64, K=4, F=2048,
