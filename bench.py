@@ -397,19 +397,20 @@ def _cores():
 
 
 def cpu_baseline(shape, inp=None, budget_s=20.0, o=None):
-    """The oracle, as it stands, on a bounded token sample of the workload."""
+    """The oracle, as it stands, on a bounded token sample of the workload:
+    the sample grows until one oracle pass takes at least half the budget."""
     import numpy as np
     o = o if o is not None else _oracle_inputs(shape, inp)
     rng = np.random.default_rng(0)
-    n = 8
-    t0 = time.perf_counter()
-    _oracle_step(shape, o, np.sort(rng.choice(shape.N, n, replace=False)))
-    t_cal = time.perf_counter() - t0
-    n = int(min(shape.N, max(8, n * (budget_s * 0.7) / max(t_cal, 1e-3))))
-    tok = np.sort(rng.choice(shape.N, n, replace=False))
-    t0 = time.perf_counter()
-    _oracle_step(shape, o, tok)
-    dt = time.perf_counter() - t0
+    n = 16
+    while True:
+        tok = np.sort(rng.choice(shape.N, n, replace=False))
+        t0 = time.perf_counter()
+        _oracle_step(shape, o, tok)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 2 or n >= shape.N:
+            break
+        n = int(min(shape.N, max(2 * n, n * (0.6 * budget_s) / max(dt, 1e-3))))
     return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
             "sample": f"{n} of {shape.N} tokens of {shape.name} ({'fwd+bwd' if shape.training else 'fwd'}), "
                       f"float64 numpy oracle, {dt:.1f} s"}

@@ -26,6 +26,8 @@
 // MOE_DEVERR_TIMEOUT); no TMA multicast is used.
 #include <cuda.h>
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -84,10 +86,10 @@ struct Tile {
 // Compile-time shape of one kernel instance.  MT = 128-row M halves per tile:
 // with MT = 2 two M=128 MMAs share every B tile, so a 256 x BN tile moves
 // (2*128 + BN) rows of operands per k-step instead of (128 + BN) per half.
-template <int BN, int MT>
+template <int BN, int MT, int CG = 1>
 struct Shape {
   static constexpr int A_BYTES = MT * BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = (CG == 2 ? BN / 2 : BN) * BK * 2;   // a pair splits B's columns
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
   static constexpr int ACC_COLS = MT * BN;                       // one accumulator set
@@ -97,6 +99,8 @@ struct Shape {
       USED_COLS <= 32 ? 32 : (USED_COLS <= 64 ? 64 : (USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512)));
   static constexpr int N_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + 8 * N_BARS + 16 + 4 * 260;
+  // 128-row halves per scheduling unit (a CTA's two halves, or a pair's)
+  static constexpr int UNIT = (MT == 2 || CG == 2) ? 2 : 1;
 };
 
 // Rows of the grouped buffers actually used, clamped to the buffers' rows.
@@ -108,16 +112,16 @@ __device__ __forceinline__ int64_t used_rows(const Params& p) {
 // Number of M units for the ROWS schedule: 128-row tiles (MT = 1) or pairs
 // of 128-row tiles of the same expert (MT = 2; an odd last tile of an expert
 // forms a unit of one half).  s_unit_start[e] = first unit of expert e.
-template <int MT>
+template <int UNIT>
 __device__ __forceinline__ int64_t rows_units(const Params& p, const int32_t* s_unit_start) {
-  if constexpr (MT == 1) return used_rows(p) / BM;
+  if constexpr (UNIT == 1) return used_rows(p) / BM;
   return s_unit_start[p.E];
 }
 
-template <int SCHED, int BN, int MT, int EPI>
+template <int SCHED, int BN, int UNIT, int EPI>
 __device__ __forceinline__ int64_t total_tiles(const Params& p, const int32_t* s_unit_start) {
   if constexpr (SCHED == SCHED_ROWS) {
-    return rows_units<MT>(p, s_unit_start) * p.n_tiles;
+    return rows_units<UNIT>(p, s_unit_start) * p.n_tiles;
   } else if constexpr (SCHED == SCHED_WGRAD) {
     return (int64_t)p.E * p.m_tiles_w * p.n_tiles;
   } else {
@@ -125,12 +129,12 @@ __device__ __forceinline__ int64_t total_tiles(const Params& p, const int32_t* s
   }
 }
 
-template <int SCHED, int BN, int MT, int EPI>
+template <int SCHED, int BN, int UNIT, int EPI>
 __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32_t* s_unit_start) {
   constexpr int NOUT = (EPI == EPI_SWIGLU || EPI == EPI_WGRAD_PAIR) ? BN / 2 : BN;
   Tile tl;
   if constexpr (SCHED == SCHED_ROWS) {
-    const int64_t num_m = rows_units<MT>(p, s_unit_start);
+    const int64_t num_m = rows_units<UNIT>(p, s_unit_start);
     const int64_t per_group = (int64_t)kGroupM * p.n_tiles;
     const int64_t g = t / per_group;
     const int64_t first_m = g * kGroupM;
@@ -138,7 +142,7 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32
     const int64_t local = t - g * per_group;
     const int64_t mu = first_m + local % gm;          // M unit
     const int64_t nt = local / gm;
-    if constexpr (MT == 1) {
+    if constexpr (UNIT == 1) {
       tl.row0 = mu * BM;
       tl.e = expert_of_row(p.padded_bins, p.E, tl.row0);
       tl.halves = 1;
@@ -163,14 +167,14 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32
     const int64_t per_e = (int64_t)p.m_tiles_w * p.n_tiles;
     tl.e = (int)(t / per_e);
     const int64_t r = t - (int64_t)tl.e * per_e;
-    tl.m0 = (int)((r / p.n_tiles) * BM * MT);
+    tl.m0 = (int)((r / p.n_tiles) * BM * UNIT);
     tl.n0 = (int)((r % p.n_tiles) * NOUT);
     const int64_t lo = tl.e ? p.padded_bins[tl.e - 1] : 0;
     int64_t hi = p.padded_bins[tl.e];
     if (hi > p.P) hi = p.P;
     tl.row0 = lo;
     tl.nkb = hi > lo ? (int)((hi - lo) / BK) : 0;
-    tl.halves = MT;
+    tl.halves = UNIT;
   } else {
     tl.e = 0;
     tl.row0 = t * BM;
@@ -359,17 +363,25 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
   }
 }
 
-template <int BN, int MT, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
+// CG = 1: one CTA per tile (MT halves of 128 rows).  CG = 2: a cluster of two
+// CTAs per 256-row tile; CTA rank r holds rows [128r, 128r + 128) of A, half of
+// B's columns and its own 128 TMEM lanes of the accumulator; the leader (rank 0)
+// issues the MMAs for both and counts both CTAs' loads on its full barriers.
+template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
-  using S = Shape<BN, MT>;
+  using S = Shape<BN, MT, CG>;
   constexpr int STAGES = S::STAGES;
   constexpr int STAGE_BYTES = S::STAGE_BYTES;
   constexpr int A_BYTES = S::A_BYTES;
+  constexpr int B_BYTES = S::B_BYTES;
   constexpr int ACC_BUFS = S::ACC_BUFS;
   constexpr int ACC_COLS = S::ACC_COLS;
+  constexpr int UNIT = S::UNIT;
+  constexpr bool PAIR = CG == 2;
   static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte swizzle atoms aligned");
   static_assert(STAGES >= 2, "pipeline needs at least two stages");
   static_assert(MT == 1 || SCHED != SCHED_DENSE, "the router uses single 128-row tiles");
+  static_assert(!PAIR || (MT == 1 && SCHED != SCHED_DENSE), "a pair holds one half per CTA");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -386,15 +398,21 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   int32_t* s_unit_start = reinterpret_cast<int32_t*>(tmem_holder + 4);   // [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;          // 0 = leader
+  const int64_t tile0 = PAIR ? (int64_t)cluster_id_x() : (int64_t)blockIdx.x;
+  const int64_t tstep = PAIR ? (int64_t)nclusters_x() : (int64_t)gridDim.x;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-    for (int a = 0; a < ACC_BUFS; ++a) { mbar_init(tfull_bar(a), 1); mbar_init(tempty_bar(a), kEpiWarps); }
+    for (int a = 0; a < ACC_BUFS; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), PAIR ? 2 * kEpiWarps : kEpiWarps);
+    }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
   }
-  if (SCHED == SCHED_ROWS && MT == 2 && warp == 2) {
+  if (SCHED == SCHED_ROWS && UNIT == 2 && warp == 2) {
     // units per expert = ceil(tiles_e / 2); exclusive scan over experts
     int carry = 0;
     for (int e0 = 0; e0 < p.E; e0 += 32) {
@@ -425,14 +443,19 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     if (SPLIT == SPLIT_K) tma_prefetch_desc(&p.ta1);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), S::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), S::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), S::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();   // barriers visible to the peer
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int64_t ntiles = total_tiles<SCHED, BN, MT, EPI>(p, s_unit_start);
+  const int64_t ntiles = total_tiles<SCHED, BN, UNIT, EPI>(p, s_unit_start);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -440,47 +463,84 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = get_tile<SCHED, BN, MT, EPI>(p, t, s_unit_start);
-        const uint32_t tx = (uint32_t)tl.halves * BM * BK * 2 +
-                            (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)S::B_BYTES);
+      for (int64_t t = tile0; t < ntiles && ok; t += tstep) {
+        const Tile tl = get_tile<SCHED, BN, UNIT, EPI>(p, t, s_unit_start);
+        uint32_t tx;
+        if constexpr (PAIR) tx = 2u * (uint32_t)(A_BYTES + B_BYTES);    // both CTAs' loads
+        else tx = (uint32_t)tl.halves * BM * BK * 2 +
+                  (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)B_BYTES);
         for (int kb = 0; kb < tl.nkb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
           const uint32_t sa = base + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t fb = full_bar(stage);
-          mbar_expect_tx(fb, tx);
-          if constexpr (SCHED == SCHED_WGRAD) {
-            const int krow = (int)(tl.row0 + (int64_t)kb * BK);
-            // A = X^T: 64-wide MN boxes of the [rows, M] matrix, 2 per half
+          if constexpr (PAIR) {
+            const uint32_t fb = map_to_rank(full_bar(stage), 0);      // the leader's barrier
+            if (rank == 0) mbar_expect_tx(full_bar(stage), tx);
+            if constexpr (SCHED == SCHED_WGRAD) {
+              const int krow = (int)(tl.row0 + (int64_t)kb * BK);
+              const int m = tl.m0 + BM * (int)rank;
+              tma_load_2d_pair(sa, &p.ta0, fb, m, krow);
+              tma_load_2d_pair(sa + 8192, &p.ta0, fb, m + 64, krow);
 #pragma unroll
-            for (int j = 0; j < 2 * MT; ++j) tma_load_2d(sa + j * 8192, &p.ta0, fb, tl.m0 + 64 * j, krow);
+              for (int j = 0; j < BN / 128; ++j) {
+                if (SPLIT == SPLIT_N)
+                  tma_load_2d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, krow);
+                else
+                  tma_load_2d_pair(sb + j * 8192, &p.tb0, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, krow);
+              }
+            } else {
+              int k = kb * BK;
+              const CUtensorMap* ta = &p.ta0;
+              const CUtensorMap* tb = &p.tb0;
+              if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
+              tma_load_2d_pair(sa, ta, fb, k, (int)tl.row0 + BM * (int)rank);
+              if constexpr (B_MN) {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) {
-              if (SPLIT == SPLIT_N && j >= BN / 128)
-                tma_load_2d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), krow);
-              else
-                tma_load_2d(sb + j * 8192, &p.tb0, fb, tl.n0 + 64 * j, krow);
+                for (int j = 0; j < BN / 128; ++j) {
+                  if (SPLIT == SPLIT_N)
+                    tma_load_3d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k, tl.e);
+                  else
+                    tma_load_3d_pair(sb + j * 8192, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k, tl.e);
+                }
+              } else {
+                tma_load_3d_pair(sb, tb, fb, k, tl.n0 + (BN / 2) * (int)rank, tl.e);
+              }
             }
           } else {
-            int k = kb * BK;
-            const CUtensorMap* ta = &p.ta0;
-            const CUtensorMap* tb = &p.tb0;
-            if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
-            tma_load_2d(sa, ta, fb, k, (int)tl.row0);
-            if (MT == 2 && tl.halves == 2) tma_load_2d(sa + BM * BK * 2, ta, fb, k, (int)tl.row0 + BM);
-            if constexpr (SCHED == SCHED_DENSE) {
-              tma_load_2d(sb, tb, fb, k, 0);
-            } else if constexpr (B_MN) {
+            const uint32_t fb = full_bar(stage);
+            mbar_expect_tx(fb, tx);
+            if constexpr (SCHED == SCHED_WGRAD) {
+              const int krow = (int)(tl.row0 + (int64_t)kb * BK);
+              // A = X^T: 64-wide MN boxes of the [rows, M] matrix, 2 per half
+#pragma unroll
+              for (int j = 0; j < 2 * MT; ++j) tma_load_2d(sa + j * 8192, &p.ta0, fb, tl.m0 + 64 * j, krow);
 #pragma unroll
               for (int j = 0; j < BN / 64; ++j) {
                 if (SPLIT == SPLIT_N && j >= BN / 128)
-                  tma_load_3d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), k, tl.e);
+                  tma_load_2d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), krow);
                 else
-                  tma_load_3d(sb + j * 8192, tb, fb, tl.n0 + 64 * j, k, tl.e);
+                  tma_load_2d(sb + j * 8192, &p.tb0, fb, tl.n0 + 64 * j, krow);
               }
             } else {
-              tma_load_3d(sb, tb, fb, k, tl.n0, tl.e);
+              int k = kb * BK;
+              const CUtensorMap* ta = &p.ta0;
+              const CUtensorMap* tb = &p.tb0;
+              if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
+              tma_load_2d(sa, ta, fb, k, (int)tl.row0);
+              if (MT == 2 && tl.halves == 2) tma_load_2d(sa + BM * BK * 2, ta, fb, k, (int)tl.row0 + BM);
+              if constexpr (SCHED == SCHED_DENSE) {
+                tma_load_2d(sb, tb, fb, k, 0);
+              } else if constexpr (B_MN) {
+#pragma unroll
+                for (int j = 0; j < BN / 64; ++j) {
+                  if (SPLIT == SPLIT_N && j >= BN / 128)
+                    tma_load_3d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), k, tl.e);
+                  else
+                    tma_load_3d(sb + j * 8192, tb, fb, tl.n0 + 64 * j, k, tl.e);
+                }
+              } else {
+                tma_load_3d(sb, tb, fb, k, tl.n0, tl.e);
+              }
             }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -494,16 +554,16 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       const int n_mma = (SCHED == SCHED_DENSE) ? p.n_mma : BN;
-      const uint32_t idesc = idesc_bf16(BM, n_mma, A_MN, B_MN);
+      const uint32_t idesc = idesc_bf16(PAIR ? 2 * BM : BM, n_mma, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = get_tile<SCHED, BN, MT, EPI>(p, t, s_unit_start);
+      for (int64_t t = tile0; t < ntiles && ok; t += tstep) {
+        const Tile tl = get_tile<SCHED, BN, UNIT, EPI>(p, t, s_unit_start);
         if (tl.nkb == 0) continue;
         if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
         tc_fence_after();
@@ -517,24 +577,31 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if constexpr (PAIR) {
+              const uint64_t ad = A_MN ? desc_mn_sw128(sa + kk * 2048, 8192) : desc_k_sw128(sa + kk * 32);
+              mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+            } else {
 #pragma unroll
-            for (int h = 0; h < MT; ++h) {
-              if (h < tl.halves) {
-                const uint32_t ah = sa + h * (BM * BK * 2);
-                const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
-                mma_bf16(d_tmem + h * BN, ad, bd, idesc, accum);
+              for (int h = 0; h < MT; ++h) {
+                if (h < tl.halves) {
+                  const uint32_t ah = sa + h * (BM * BK * 2);
+                  const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
+                  mma_bf16(d_tmem + h * BN, ad, bd, idesc, accum);
+                }
               }
             }
           }
-          mma_commit(empty_bar(stage));      // smem slot free once these MMAs are done
+          // smem slot free (in both CTAs of a pair) once these MMAs are done
+          if constexpr (PAIR) mma_commit_pair(empty_bar(stage), 0x3); else mma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(tfull_bar(acc));          // accumulator ready for the epilogue
+        // accumulator ready for the epilogue(s)
+        if constexpr (PAIR) mma_commit_pair(tfull_bar(acc), 0x3); else mma_commit(tfull_bar(acc));
         if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) {
-        mma_commit(drain_bar);
+        if constexpr (PAIR) mma_commit_pair(drain_bar, 0x1); else mma_commit(drain_bar);
         const uint64_t t0 = globaltimer();
         while (!mbar_try_wait(drain_bar, 0) && globaltimer() - t0 < 50000000ull) {}
       }
@@ -544,16 +611,18 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     const int q = warp & 3;                       // TMEM lane quarter of this warp
     const int part = (warp - 2) >> 2;             // which half of the columns
     const int row = q * 32 + lane;                // row inside a 128-row half
+    const uint32_t tempty_leader0 = PAIR ? map_to_rank(tempty_bar(0), 0) : 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const Tile tl = get_tile<SCHED, BN, MT, EPI>(p, t, s_unit_start);
+    for (int64_t t = tile0; t < ntiles; t += tstep) {
+      const Tile tl = get_tile<SCHED, BN, UNIT, EPI>(p, t, s_unit_start);
       if constexpr (SCHED == SCHED_WGRAD) {
         if (tl.nkb == 0) {                        // expert with no rows: zero gradient
           const float z[32] = {0.f};
 #pragma unroll 1
           for (int h = 0; h < MT; ++h) {
-            const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + h * BM + row) * p.ldo + tl.n0;
+            const int hh = PAIR ? (int)rank : h;
+            const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + hh * BM + row) * p.ldo + tl.n0;
             if constexpr (EPI == EPI_WGRAD_PAIR) {
 #pragma unroll 1
               for (int c = part * (BN / 4); c < (part + 1) * (BN / 4); c += 32) {
@@ -573,26 +642,41 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
+      if constexpr (PAIR) {
+        // this CTA's 128 rows of the 256-row tile; a lone last tile of an
+        // expert has no second half, so the peer stores nothing
+        if ((int)rank < tl.halves) {
+          const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+          Tile th = tl;
+          if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + (int)rank * BM; else th.row0 = tl.row0 + (int)rank * BM;
+          epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part);
+        }
+      } else {
 #pragma unroll 1
-      for (int h = 0; h < tl.halves; ++h) {
-        const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
-        Tile th = tl;
-        if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + h * BM; else th.row0 = tl.row0 + h * BM;
-        epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part);
+        for (int h = 0; h < tl.halves; ++h) {
+          const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
+          Tile th = tl;
+          if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + h * BM; else th.row0 = tl.row0 + h * BM;
+          epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part);
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_remote(tempty_leader0 + 8u * acc);   // the leader's barrier
+        else mbar_arrive(tempty_bar(acc));
+      }
       if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, S::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+    else tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
 }
 
@@ -656,17 +740,55 @@ static int sm_count() {
   return cache[dev];
 }
 
-template <int BN, int MT, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
+template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
 static moe_status launch(const char* name, const Params& p, int64_t tiles_upper, cudaStream_t s) {
-  using S = Shape<BN, MT>;
-  auto kern = umma_gemm_kernel<BN, MT, SCHED, EPI, A_MN, B_MN, SPLIT>;
+  using S = Shape<BN, MT, CG>;
+  auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  int64_t grid = tiles_upper < sm_count() ? tiles_upper : sm_count();
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // Persistent CTAs (or pairs): every one must be resident at once, since each
+  // owns a fixed share of the tiles.  Pairs are placed within a GPC, so ask the
+  // runtime how many fit rather than assuming SMs / 2.
+  int64_t units = sm_count();
+  if (CG == 2) {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+      int n = 0;
+      cfg.gridDim = dim3((unsigned)sm_count(), 1, 1);
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        n = sm_count() / 2;
+      }
+      cached[dev] = n;
+    }
+    units = cached[dev];
+  }
+  int64_t grid = tiles_upper < units ? tiles_upper : units;
   if (grid < 1) grid = 1;
-  MOE_TRACED(name, s, (kern<<<(unsigned)grid, kThreads, S::SMEM, s>>>(p)));
+  cfg.gridDim = dim3((unsigned)(grid * CG), 1, 1);
+  cudaError_t err = cudaSuccess;
+  MOE_TRACED(name, s, (err = cudaLaunchKernelEx(&cfg, kern, p)));
+  if (err != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -687,10 +809,15 @@ using namespace umma;
 
 bool umma_shape_supported(int H, int F) { return H % 128 == 0 && F % 128 == 0 && H >= 128 && F >= 128; }
 
+// Kernel choice per GEMM (measured on B200, training-step and forward
+// workloads): CTA pairs wherever a 256 x 256 tile fits, except the dgrad to x,
+// whose 256-row single-CTA tiles were faster.
+
 moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W3, const void* W2,
                                const int32_t* pb, int E, int H, int F, int64_t P, void* act, void* out,
                                void* gate_up, int* status, cudaStream_t s) {
   typedef __nv_bfloat16 bf;
+  const bool pair = true;
   // GEMM1 + SwiGLU: [G | U] = x_perm * [W1_e | W3_e], act = silu(G) * U
   {
     Params p = blank_params(pb, E, P, status);
@@ -704,10 +831,9 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.out1 = gate_up ? (bf*)gate_up : nullptr;
     p.out2 = gate_up ? (bf*)gate_up + (size_t)P * F : nullptr;
     p.ldo = F;
-    // 128-row tiles: the SwiGLU epilogue (up to three outputs) stays hidden
-    // behind the next tile's main loop only with two accumulator buffers
-    moe_status st = launch<256, 1, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p,
-                                                                              (P / BM) * p.n_tiles, s);
+    const int64_t up = (P / BM) * p.n_tiles;
+    moe_status st = pair ? launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p, up, s)
+                         : launch<256, 1, 1, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p, up, s);
     if (st != MOE_OK) return st;
   }
   // GEMM2: out = act * W2_e
@@ -720,9 +846,10 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.n_tiles = H / bn;
     p.out0 = (bf*)out;
     p.ldo = H;
-    if (bn == 256)
-      return launch<256, 2, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
-    return launch<128, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, (P / BM) * p.n_tiles, s);
+    const int64_t up = (P / BM) * p.n_tiles;
+    if (bn == 256 && pair) return launch<256, 1, 2, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
+    if (bn == 256) return launch<256, 2, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
+    return launch<128, 1, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
   }
 }
 
@@ -736,12 +863,15 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
   const bf* U = G + (size_t)P * F;
   bf* dG = (bf*)d_gate_up;
   bf* dU = dG + (size_t)P * F;
+  const bool pref = true;
   moe_status st;
   // dA = d_out * W2_e^T with the SwiGLU backward in the epilogue
   {
     Params p = blank_params(pb, E, P, status);
     const int bn = (F % 256 == 0) ? 256 : 128;
-    if (!map2d(&p.ta0, d_out, H, P, H, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, bn)) return MOE_ERR_CUDA;
+    const bool pair = pref && bn == 256;
+    if (!map2d(&p.ta0, d_out, H, P, H, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, pair ? bn / 2 : bn))
+      return MOE_ERR_CUDA;
     p.kdim = H;
     p.n_mma = bn;
     p.n_tiles = F / bn;
@@ -751,55 +881,58 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.out1 = dU;
     p.ldo = F;
     const int64_t up = (P / BM) * p.n_tiles;
-    // 128-row tiles for the same reason as GEMM1 (the epilogue reads G, U and
-    // writes dG, dU)
-    st = bn == 256 ? launch<256, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s)
-                   : launch<128, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s);
+    st = pair ? launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s)
+         : bn == 256 ? launch<256, 1, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s)
+                     : launch<128, 1, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s);
     if (st != MOE_OK) return st;
   }
   // dW2_e = act_e^T * d_out_e   [F, H]
   {
     Params p = blank_params(pb, E, P, status);
     const int bn = (H % 256 == 0) ? 256 : 128;
-    const int mt = (bn == 256 && F % 256 == 0) ? 2 : 1;
+    const int unit = (bn == 256 && F % 256 == 0) ? 2 : 1;
     if (!map2d(&p.ta0, act, F, P, F, 64, 64) || !map2d(&p.tb0, d_out, H, P, H, 64, 64)) return MOE_ERR_CUDA;
     p.n_mma = bn;
-    p.m_tiles_w = F / (BM * mt);
+    p.m_tiles_w = F / (BM * unit);
     p.n_tiles = H / bn;
     p.out0 = (bf*)dW2;
     p.ldo = H;
     p.out_estride = (int64_t)F * H;
     const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
-    if (mt == 2) st = launch<256, 2, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
-    else if (bn == 256) st = launch<256, 1, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
-    else st = launch<128, 1, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
+    if (unit == 2 && pref) st = launch<256, 1, 2, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
+    else if (unit == 2) st = launch<256, 2, 1, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
+    else if (bn == 256) st = launch<256, 1, 1, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
+    else st = launch<128, 1, 1, SCHED_WGRAD, EPI_WGRAD, true, true, SPLIT_NONE>("wgrad_w2", p, tiles, s);
     if (st != MOE_OK) return st;
   }
   // dW1_e | dW3_e = x_perm_e^T * [dG_e | dU_e]   [H, F] each
   {
     Params p = blank_params(pb, E, P, status);
-    const int mt = (H % 256 == 0) ? 2 : 1;
+    const int unit = (H % 256 == 0) ? 2 : 1;
     if (!map2d(&p.ta0, x_perm, H, P, H, 64, 64) || !map2d(&p.tb0, dG, F, P, F, 64, 64) ||
         !map2d(&p.tb1, dU, F, P, F, 64, 64))
       return MOE_ERR_CUDA;
     p.n_mma = 256;
-    p.m_tiles_w = H / (BM * mt);
+    p.m_tiles_w = H / (BM * unit);
     p.n_tiles = F / 128;
     p.out0 = (bf*)dW1;
     p.out1 = (bf*)dW3;
     p.ldo = F;
     p.out_estride = (int64_t)H * F;
     const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
-    st = mt == 2 ? launch<256, 2, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s)
-                 : launch<256, 1, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
+    if (unit == 2 && pref) st = launch<256, 1, 2, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
+    else if (unit == 2) st = launch<256, 2, 1, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
+    else st = launch<256, 1, 1, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
     if (st != MOE_OK) return st;
   }
   // dx_perm = dG * W1_e^T + dU * W3_e^T  (one K = 2F contraction)
   {
     Params p = blank_params(pb, E, P, status);
     const int bn = (H % 256 == 0) ? 256 : 128;
+    const bool pair = false;    // see the kernel choice note above
+    const uint32_t box = pair ? bn / 2 : bn;
     if (!map2d(&p.ta0, dG, F, P, F, 64, 128) || !map2d(&p.ta1, dU, F, P, F, 64, 128) ||
-        !map3d(&p.tb0, W1, F, H, E, 64, bn) || !map3d(&p.tb1, W3, F, H, E, 64, bn))
+        !map3d(&p.tb0, W1, F, H, E, 64, box) || !map3d(&p.tb1, W3, F, H, E, 64, box))
       return MOE_ERR_CUDA;
     p.kdim = 2 * F;
     p.ksplit = F;
@@ -808,8 +941,9 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.out0 = (bf*)dx_perm;
     p.ldo = H;
     const int64_t up = (P / BM) * p.n_tiles;
-    st = bn == 256 ? launch<256, 2, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s)
-                   : launch<128, 1, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s);
+    st = pair ? launch<256, 1, 2, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s)
+         : bn == 256 ? launch<256, 2, 1, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s)
+                     : launch<128, 1, 1, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s);
     if (st != MOE_OK) return st;
   }
   return MOE_OK;
@@ -838,7 +972,7 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   p.probs = probs;
   p.top = top;
   p.weights = w;
-  return launch<256, 1, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
+  return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
 }
 
 }  // namespace moe
