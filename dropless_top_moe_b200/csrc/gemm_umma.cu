@@ -222,6 +222,71 @@ __device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals
   }
 }
 
+// Router epilogue for one token row: E fp32 logits in TMEM columns
+// [tacc, tacc + E) -> optional logits / probs, top-K ids (descending, ties to
+// the lower id) and renormalised weights exp(l_k - l_max) / sum_kept.
+template <int KMAX>
+__device__ __forceinline__ void router_row(const Params& p, uint32_t tacc, int64_t grow) {
+  const int E = p.n_mma, K = p.K;
+  const bool live = grow < p.P;
+  float vals[KMAX];
+  int ids[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
+  float m = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < E; c += 32) {
+    uint32_t r[32];
+    tmem_ld_32(tacc + c, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (c + j < E) {
+        const float v = __uint_as_float(r[j]);
+        m = fmaxf(m, v);
+        topk_insert<KMAX>(v, c + j, K, vals, ids);
+        if (live && p.logits) p.logits[grow * E + c + j] = v;
+      }
+    }
+  }
+  if (p.probs) {
+    float Z = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < E; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c + j < E) Z += expf(__uint_as_float(r[j]) - m);
+    }
+#pragma unroll 1
+    for (int c = 0; c < E; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (live && c + j < E) p.probs[grow * E + c + j] = expf(__uint_as_float(r[j]) - m) / Z;
+    }
+  }
+  if (live) {
+    float S = 0.f, ev[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ev[j] = (j < K) ? expf(vals[j] - vals[0]) : 0.f;
+      S += ev[j];
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < K) {
+        p.top[grow * K + j] = ids[j];
+        p.weights[grow * K + j] = ev[j] / S;
+      }
+    }
+  }
+}
+
 // Epilogue of one 128-row half: TMEM columns [tacc, tacc + BN) of this
 // thread's row -> fused math -> global memory.
 template <int BN, int SCHED, int EPI>
@@ -301,72 +366,11 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
     }
   } else {  // EPI_ROUTER: softmax, top-K, renormalise on this row's E logits
     if (part != 0) return;
-    constexpr int KMAX = 16;
-    const int E = p.n_mma, K = p.K;
-    const bool live = grow < p.P;
-    float vals[KMAX];
-    int ids[KMAX];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
-    float m = -INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < E; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32(tacc + c, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (c + j < E) {
-          const float v = __uint_as_float(r[j]);
-          m = fmaxf(m, v);
-          topk_insert<KMAX>(v, c + j, K, vals, ids);
-          if (live && p.logits) p.logits[grow * E + c + j] = v;
-        }
-      }
-    }
-    if (p.probs) {
-      float Z = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < E; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32(tacc + c, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c + j < E) Z += expf(__uint_as_float(r[j]) - m);
-      }
-#pragma unroll 1
-      for (int c = 0; c < E; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32(tacc + c, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (live && c + j < E) p.probs[grow * E + c + j] = expf(__uint_as_float(r[j]) - m) / Z;
-      }
-    }
-    if (live) {
-      float S = 0.f, ev[KMAX];
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        ev[j] = (j < K) ? expf(vals[j] - vals[0]) : 0.f;
-        S += ev[j];
-      }
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (j < K) {
-          p.top[grow * K + j] = ids[j];
-          p.weights[grow * K + j] = ev[j] / S;
-        }
-      }
-    }
+    if (p.K <= 8) router_row<8>(p, tacc, grow);
+    else router_row<16>(p, tacc, grow);
   }
 }
 
-// CG = 1: one CTA per tile (MT halves of 128 rows).  CG = 2: a cluster of two
-// CTAs per 256-row tile; CTA rank r holds rows [128r, 128r + 128) of A, half of
-// B's columns and its own 128 TMEM lanes of the accumulator; the leader (rank 0)
-// issues the MMAs for both and counts both CTAs' loads on its full barriers.
 template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
   using S = Shape<BN, MT, CG>;
@@ -528,7 +532,9 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
               if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
               tma_load_2d(sa, ta, fb, k, (int)tl.row0);
               if (MT == 2 && tl.halves == 2) tma_load_2d(sa + BM * BK * 2, ta, fb, k, (int)tl.row0 + BM);
-              if constexpr (SCHED == SCHED_DENSE) {
+              if constexpr (SCHED == SCHED_DENSE && B_MN) {
+                for (int j = 0; j < p.n_mma / 64; ++j) tma_load_2d(sb + j * 8192, tb, fb, 64 * j, k);
+              } else if constexpr (SCHED == SCHED_DENSE) {
                 tma_load_2d(sb, tb, fb, k, 0);
               } else if constexpr (B_MN) {
 #pragma unroll
@@ -960,11 +966,18 @@ size_t route_umma_scratch(int H, int E) { return (size_t)E * H * 2; }
 
 moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K, float* logits,
                       float* probs, int32_t* top, float* w, void* scratch, int* status, cudaStream_t s) {
-  // B operand K-major: W_r^T [E, H] kept in the workspace
-  moe_status st = transpose_matrix(W_r, H, E, MOE_BF16, scratch, s);
-  if (st != MOE_OK) return st;
   Params p = blank_params(nullptr, 1, N, status);
-  if (!map2d(&p.ta0, x, H, N, H, 64, 128) || !map2d(&p.tb0, scratch, H, E, H, 64, E)) return MOE_ERR_CUDA;
+  if (!map2d(&p.ta0, x, H, N, H, 64, 128)) return MOE_ERR_CUDA;
+  const bool mn = E % 64 == 0;
+  if (mn) {
+    // B operand MN-major straight from W_r [H, E]: 64-expert boxes
+    if (!map2d(&p.tb0, W_r, E, H, E, 64, 64)) return MOE_ERR_CUDA;
+  } else {
+    // B operand K-major: W_r^T [E, H] kept in the workspace
+    moe_status st = transpose_matrix(W_r, H, E, MOE_BF16, scratch, s);
+    if (st != MOE_OK) return st;
+    if (!map2d(&p.tb0, scratch, H, E, H, 64, E)) return MOE_ERR_CUDA;
+  }
   p.kdim = H;
   p.n_mma = E;
   p.K = K;
@@ -972,6 +985,7 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   p.probs = probs;
   p.top = top;
   p.weights = w;
+  if (mn) return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER, false, true, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
   return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
 }
 

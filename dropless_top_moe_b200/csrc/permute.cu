@@ -132,16 +132,31 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ out, const fl
       if (p >= 0) {
         const T* o = out + (size_t)p * H;
         T* d = d_out + (size_t)p * H;
-        for (int v = lane; v < nvec; v += 32) {
-          float gf[V], of[V], df[V];
-          Vec<T>::to_float(ld_nc_v4(g + (size_t)v * V), gf);
-          Vec<T>::to_float(ld_nc_v4(o + (size_t)v * V), of);
+        for (int v0 = lane; v0 < nvec; v0 += 32 * kSeg) {
+          uint4 gv[kSeg], ov[kSeg];          // issue all loads of the segment first
 #pragma unroll
-          for (int j = 0; j < V; ++j) {
-            dot = fmaf(gf[j], of[j], dot);
-            df[j] = w * gf[j];
+          for (int u = 0; u < kSeg; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < nvec) {
+              gv[u] = ld_nc_v4(g + (size_t)v * V);
+              ov[u] = ld_nc_v4(o + (size_t)v * V);
+            }
           }
-          st_v4(d + (size_t)v * V, Vec<T>::from_float(df));
+#pragma unroll
+          for (int u = 0; u < kSeg; ++u) {
+            const int v = v0 + 32 * u;
+            if (v < nvec) {
+              float gf[V], of[V], df[V];
+              Vec<T>::to_float(gv[u], gf);
+              Vec<T>::to_float(ov[u], of);
+#pragma unroll
+              for (int j = 0; j < V; ++j) {
+                dot = fmaf(gf[j], of[j], dot);
+                df[j] = w * gf[j];
+              }
+              st_v4(d + (size_t)v * V, Vec<T>::from_float(df));
+            }
+          }
         }
       }
       dot = warp_sum(dot);
@@ -256,13 +271,29 @@ router_wgrad_partial_kernel(const float* __restrict__ dlogit, const T* __restric
   float acc[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) acc[j] = 0.f;
-  for (int64_t r = r0; r < r1; ++r) {
-    const int i = indices[sstart + r];
-    const float dl = dlogit[i];
-    float f[V];
-    Vec<T>::to_float(ld_nc_v4(x + (size_t)(i / K) * H + h0), f);
+  constexpr int U = 4;                      // rows in flight; summed in increasing r
+  for (int64_t r = r0; r < r1; r += U) {
+    int idx[U];
+    float dl[U];
+    uint4 xv[U];
 #pragma unroll
-    for (int j = 0; j < V; ++j) acc[j] = fmaf(dl, f[j], acc[j]);
+    for (int u = 0; u < U; ++u) idx[u] = (r + u < r1) ? indices[sstart + r + u] : -1;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (idx[u] >= 0) {
+        dl[u] = dlogit[idx[u]];
+        xv[u] = ld_nc_v4(x + (size_t)(idx[u] / K) * H + h0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (idx[u] >= 0) {
+        float f[V];
+        Vec<T>::to_float(xv[u], f);
+#pragma unroll
+        for (int j = 0; j < V; ++j) acc[j] = fmaf(dl[u], f[j], acc[j]);
+      }
+    }
   }
   float* dst = part + m * H + h0;
 #pragma unroll
