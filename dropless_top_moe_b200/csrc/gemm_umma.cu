@@ -227,7 +227,7 @@ __device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals
 // the lower id) and renormalised weights exp(l_k - l_max) / sum_kept.
 template <int KMAX>
 __device__ __forceinline__ void router_row(const Params& p, uint32_t tacc, int64_t grow) {
-  const int E = p.n_mma, K = p.K;
+  const int E = p.E, K = p.K;     // MMA columns beyond E (padding to 16) are ignored
   const bool live = grow < p.P;
   float vals[KMAX];
   int ids[KMAX];
@@ -959,27 +959,30 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
 
 bool route_umma_supported(int N, int H, int E, int K) {
   (void)N;
-  return E >= 16 && E <= 256 && E % 16 == 0 && K <= 16 && H % 64 == 0;
+  return E >= 1 && E <= 256 && K <= 16 && H % 64 == 0;
 }
 
-size_t route_umma_scratch(int H, int E) { return (size_t)E * H * 2; }
+size_t route_umma_scratch(int H, int E) { return (size_t)round_up(E < 16 ? 16 : E, 16) * H * 2; }
 
 moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K, float* logits,
                       float* probs, int32_t* top, float* w, void* scratch, int* status, cudaStream_t s) {
-  Params p = blank_params(nullptr, 1, N, status);
+  Params p = blank_params(nullptr, E, N, status);
   if (!map2d(&p.ta0, x, H, N, H, 64, 128)) return MOE_ERR_CUDA;
   const bool mn = E % 64 == 0;
+  // MMA N: E rounded up to 16 (the smallest M = 128 MMA width); the extra
+  // columns read zeros (out-of-bounds rows of the K-major map) and are ignored
+  const int n_mma = E < 16 ? 16 : (int)round_up(E, 16);
   if (mn) {
     // B operand MN-major straight from W_r [H, E]: 64-expert boxes
     if (!map2d(&p.tb0, W_r, E, H, E, 64, 64)) return MOE_ERR_CUDA;
   } else {
     // B operand K-major: W_r^T [E, H] kept in the workspace
-    moe_status st = transpose_matrix(W_r, H, E, MOE_BF16, scratch, s);
+    moe_status st = transpose_matrix(W_r, H, E, MOE_BF16, scratch, s, n_mma);   // rows E.. are 0
     if (st != MOE_OK) return st;
-    if (!map2d(&p.tb0, scratch, H, E, H, 64, E)) return MOE_ERR_CUDA;
+    if (!map2d(&p.tb0, scratch, H, n_mma, H, 64, (uint32_t)n_mma)) return MOE_ERR_CUDA;
   }
   p.kdim = H;
-  p.n_mma = E;
+  p.n_mma = n_mma;
   p.K = K;
   p.logits = logits;
   p.probs = probs;

@@ -31,7 +31,8 @@ moe_status combine_rows(const void* out, const float* w, const int32_t* pos, int
 moe_status combine_bwd_rows(const void* dy, const void* out, const float* w, const int32_t* pos,
                             const int32_t* bins, const int32_t* pb, int N, int K, int H, int E,
                             moe_dtype dt, float* dw, float* dlogit, void* d_out, cudaStream_t s);
-moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s);
+moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s,
+                            int C_pad = 0);
 size_t unpermute_router_bwd_scratch(int H, int E, int64_t P);
 moe_status unpermute_router_bwd(const void* dx_perm, const float* dlogit, const void* x,
                                 const void* W_r, const int32_t* top, const int32_t* pos,

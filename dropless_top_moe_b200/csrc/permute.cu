@@ -171,19 +171,20 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ out, const fl
   zero_pad_rows<T>(bins, padded_bins, E, H, d_out);
 }
 
-// W_rT[e][h] = W_r[h][e], through a shared-memory tile.
+// outT[c][r] = in[r][c] for c < C, and 0 for C <= c < C_pad (zero rows that
+// pad a transposed operand to an MMA width), through a shared-memory tile.
 template <typename T>
-__global__ void transpose_kernel(const T* __restrict__ in, int R, int C, T* __restrict__ outT) {
+__global__ void transpose_kernel(const T* __restrict__ in, int R, int C, int C_pad, T* __restrict__ outT) {
   __shared__ T tile[32][33];
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
     const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < R && c < C) tile[i][threadIdx.x] = in[(size_t)r * C + c];
+    if (r < R && c < C_pad) tile[i][threadIdx.x] = c < C ? in[(size_t)r * C + c] : from_f<T>(0.f);
   }
   __syncthreads();
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
     const int c = c0 + i, r = r0 + threadIdx.x;
-    if (r < R && c < C) outT[(size_t)c * R + r] = tile[threadIdx.x][i];
+    if (r < R && c < C_pad) outT[(size_t)c * R + r] = tile[threadIdx.x][i];
   }
 }
 
@@ -267,24 +268,33 @@ router_wgrad_partial_kernel(const float* __restrict__ dlogit, const T* __restric
   const int64_t r0 = row0 - pstart;                       // rank of the tile's first row
   const int64_t r1 = (r0 + kTile < cnt) ? r0 + kTile : cnt;
   const int h0 = (blockIdx.y * blockDim.x + threadIdx.x) * V;
-  if (h0 >= H) return;
   float acc[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) acc[j] = 0.f;
-  constexpr int U = 4;                      // rows in flight; summed in increasing r
-  for (int64_t r = r0; r < r1; r += U) {
+  // the tile's assignment ids and their dlogits, staged once per block
+  __shared__ int s_row[kTile];
+  __shared__ float s_dl[kTile];
+  for (int q = threadIdx.x; q < kTile; q += blockDim.x) {
+    const int64_t r = r0 + q;
+    const int i = r < r1 ? indices[sstart + r] : -1;
+    s_row[q] = i >= 0 ? i / K : -1;
+    s_dl[q] = i >= 0 ? dlogit[i] : 0.f;
+  }
+  __syncthreads();
+  if (h0 >= H) return;
+  constexpr int U = 8;                      // rows in flight; summed in increasing r
+  for (int q0 = 0; q0 < (int)(r1 - r0); q0 += U) {
     int idx[U];
     float dl[U];
     uint4 xv[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) idx[u] = (r + u < r1) ? indices[sstart + r + u] : -1;
-#pragma unroll
     for (int u = 0; u < U; ++u) {
-      if (idx[u] >= 0) {
-        dl[u] = dlogit[idx[u]];
-        xv[u] = ld_nc_v4(x + (size_t)(idx[u] / K) * H + h0);
-      }
+      idx[u] = (q0 + u < (int)(r1 - r0)) ? s_row[q0 + u] : -1;
+      dl[u] = s_dl[q0 + u < kTile ? q0 + u : 0];
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (idx[u] >= 0) xv[u] = ld_nc_v4(x + (size_t)idx[u] * H + h0);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (idx[u] >= 0) {
@@ -369,13 +379,16 @@ moe_status combine_bwd_rows(const void* dy, const void* out, const float* w, con
              : combine_bwd_t<__nv_bfloat16>(dy, out, w, pos, bins, pb, N, K, H, E, dw, dlogit, d_out, s);
 }
 
-moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s) {
-  dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R, 32)), block(32, 8);
+moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s,
+                            int C_pad) {
+  if (C_pad < C) C_pad = C;
+  dim3 grid((unsigned)cdiv(C_pad, 32), (unsigned)cdiv(R, 32)), block(32, 8);
   if (dt == MOE_F32)
-    MOE_TRACED("transpose", s, (transpose_kernel<float><<<grid, block, 0, s>>>((const float*)in, R, C, (float*)outT)));
+    MOE_TRACED("transpose", s, (transpose_kernel<float><<<grid, block, 0, s>>>((const float*)in, R, C, C_pad,
+                                                                                (float*)outT)));
   else
-    MOE_TRACED("transpose", s, (transpose_kernel<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)in, R, C,
-                                                           (__nv_bfloat16*)outT)));
+    MOE_TRACED("transpose", s, (transpose_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+                                   (const __nv_bfloat16*)in, R, C, C_pad, (__nv_bfloat16*)outT)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

@@ -22,9 +22,10 @@ route_simt_kernel(const T* __restrict__ x, const T* __restrict__ W_r, int N, int
                   int32_t* __restrict__ top_experts, float* __restrict__ weights) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   T* wrT = reinterpret_cast<T*>(smem_raw);          // [E][H]
+  // transposed staging with h fastest across threads: conflict-free smem writes
   for (int idx = threadIdx.x; idx < H * E; idx += blockDim.x) {
-    const int h = idx / E, e = idx - h * E;
-    wrT[(size_t)e * H + h] = W_r[idx];
+    const int e = idx / H, h = idx - e * H;
+    wrT[idx] = W_r[(size_t)h * E + e];
   }
   __syncthreads();
 

@@ -24,6 +24,8 @@ ROUTE_SHAPES = [
     small_shape("r_bf16_e64_k1", N=260, H=128, E=64, K=1),
     small_shape("r_f32_k_eq_e", N=130, H=64, E=4, K=4, dtype="f32"),
     small_shape("r_bf16_zipf", N=640, H=256, E=64, K=6, skew="zipf", skew_param=1.0),
+    small_shape("r_bf16_e4", N=300, H=128, E=4, K=2),
+    small_shape("r_bf16_e100", N=333, H=256, E=100, K=5),
 ]
 
 
