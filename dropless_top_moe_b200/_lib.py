@@ -44,6 +44,7 @@ SIGNATURES = {
     "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
                             P, P, P, P, P, P, SZ, P]),
     "moe_dispatch_meta_noalloc": (I32, [P, I32, I32, I32, P, P, P, P, P, P, P]),
+    "moe_sum_rank_ordered": (I32, [P, I32, I64, I32, C.c_float, P, P]),
     "moe_trace_attach": (I32, [P, I32, P, P]),
     "moe_trace_detach": (I32, []),
 }

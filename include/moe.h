@@ -242,6 +242,16 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                          int32_t F, moe_dtype dt, void* dx, void* dW_r, void* dW1, void* dW3,
                          void* dW2, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Local step of a deterministic data-parallel gradient all-reduce (replicas of
+ * the layer on several GPUs each hold gradients of their own tokens; a
+ * trainer sums them).  shards: [n_ranks, numel] contiguous (dt), one row per
+ * rank in rank order, as an all-to-all of equal shards delivers them;
+ * out[j] = scale * sum_{r = 0..n_ranks-1} shards[r][j], summed in increasing r
+ * in fp32 and rounded once, so every rank gets identical bits.  numel must be
+ * a multiple of 8 (bf16) or 4 (fp32). */
+moe_status moe_sum_rank_ordered(const void* shards, int32_t n_ranks, int64_t numel, moe_dtype dt,
+                                float scale, void* out, moe_stream_t stream);
+
 /* Per-launch timing.  While attached, every kernel launch made by any entry
  * point records events[2*i] on its stream just before launch i and
  * events[2*i+1] just after it, stores a static kernel name in labels[i]

@@ -174,3 +174,18 @@ def test_grouped_swiglu_matches_oracle(dtype, H, F, E, counts):
             Gr = Xd[start:end] @ om.f64(W1[e].cpu())
             assert_scaled(gu[0, start:end], Gr, dtype, f"G[{e}]")
         start = end
+
+
+@pytest.mark.parametrize("dt,n,numel", [(torch.bfloat16, 8, 1 << 20), (torch.float32, 3, 4096 * 3),
+                                        (torch.bfloat16, 1, 64)])
+def test_sum_rank_ordered_matches_ordered_fp32_sum(dt, n, numel):
+    from dropless_top_moe_b200._lib import call, MOE_BF16, MOE_F32
+    g = torch.Generator(device="cuda").manual_seed(n)
+    shards = torch.randn(n, numel, generator=g, device="cuda").to(dt)
+    out = torch.empty(numel, dtype=dt, device="cuda")
+    call("moe_sum_rank_ordered", shards.data_ptr(), n, numel, MOE_BF16 if dt == torch.bfloat16 else MOE_F32,
+         1.0 / n, out.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    acc = torch.zeros(numel, dtype=torch.float32, device="cuda")
+    for r in range(n):
+        acc += shards[r].float()
+    assert torch.equal(out, (acc * (1.0 / n)).to(dt))
