@@ -277,10 +277,26 @@ def dense_mixture(x, W_r, W1, W3, W2) -> np.ndarray:
     return y
 
 
+# ------------------------------------------------- load-balancing loss ---
+
+def aux_loss(probs, top_experts, alpha: float, N_total: int | None = None) -> float:
+    """Switch-style auxiliary load-balancing loss (icman sec. 4.2):
+    alpha * E * sum_i f_i * P_i with f_i = share of the N*K assignments routed
+    to expert i and P_i = mean over tokens of the router probability of i.
+    With perfectly balanced routing and uniform probabilities it equals alpha."""
+    p = np.asarray(probs, np.float64)
+    te = np.asarray(top_experts)
+    N, E = p.shape
+    K = te.shape[1]
+    f = np.bincount(te.reshape(-1), minlength=E) / (N * K)
+    P = p.sum(axis=0) / N
+    return float(alpha * E * np.sum(f * P))
+
+
 # -------------------------------------------------------------- backward ---
 
 def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
-                 tokens=None) -> dict:
+                 tokens=None, aux_alpha: float = 0.0, aux_grad: float = 1.0) -> dict:
     """Gradients of sum(y * dy) by the chain rule of the forward definition.
 
     Per token t and slot k with expert e (forward g = x W1_e, u = x W3_e,
@@ -294,6 +310,9 @@ def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
       softmax: dlogits = p * (dp - <dp, p>);  dW_r += x^T dlogits;  dx += dlogits W_r^T
     `tokens` restricts every sum to a subset of tokens (the weight gradients
     are then those of the sub-batch).
+    With aux_alpha != 0 the objective also carries aux_grad * aux_loss (of the
+    whole batch): the counts f_i are piecewise constant, so the extra gradient
+    flows through P_i = mean_t p_t,i only: dp_t,i += aux_grad*alpha*E*f_i/N.
     """
     xv, dyv = f64(x), f64(dy)
     r = routing if routing is not None else route(x, W_r, K)
@@ -335,6 +354,9 @@ def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
     dp_kept = dw / S - np.sum(dw * p_kept, axis=1, keepdims=True) / S ** 2
     dp = np.zeros_like(probs)
     np.put_along_axis(dp, te.astype(np.int64), dp_kept, axis=1)
+    if aux_alpha != 0.0:
+        f_all = np.bincount(np.asarray(r["top_experts"]).reshape(-1), minlength=E) / (N * K)
+        dp = dp + aux_grad * aux_alpha * E * f_all[None, :] / N
     dlogits = probs * (dp - np.sum(dp * probs, axis=1, keepdims=True))
     dW_r = xs.T @ dlogits
     dx += dlogits @ W_rv.T
@@ -342,6 +364,12 @@ def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
             "dw": dw, "dlogits": dlogits, "tokens": tok}
 
 
-def loss_sum(x, W_r, W1, W3, W2, K, dy) -> float:
-    """sum(y * dy) with routing recomputed; used by the finite-difference pins."""
-    return float(np.sum(moe_forward(x, W_r, W1, W3, W2, K)["y"] * f64(dy)))
+def loss_sum(x, W_r, W1, W3, W2, K, dy, aux_alpha: float = 0.0, aux_grad: float = 1.0) -> float:
+    """sum(y * dy) (+ aux_grad * aux_loss) with routing recomputed; used by the
+    finite-difference pins."""
+    out = moe_forward(x, W_r, W1, W3, W2, K)
+    v = float(np.sum(out["y"] * f64(dy)))
+    if aux_alpha != 0.0:
+        r = out["routing"]
+        v += aux_grad * aux_loss(r["probs"], r["top_experts"], aux_alpha)
+    return v

@@ -267,3 +267,31 @@ def test_generator_is_deterministic_and_skew_column():
     for k in a:
         assert torch.equal(a[k], b[k])
     assert torch.all(a["x"][:, 0] == 1)
+
+
+# ----------------------------------------------------- load-balancing loss
+
+def test_aux_loss_closed_forms():
+    N, E, K = 64, 8, 2
+    probs = np.full((N, E), 1.0 / E)
+    te = np.stack([[(2 * t) % E, (2 * t + 1) % E] for t in range(N)])
+    assert om.aux_loss(probs, te, 0.01) == pytest.approx(0.01, rel=1e-14)   # balanced: alpha
+    # everything on experts 0 and 1 with certainty-like probabilities: alpha * E / 2 * (P0 + P1)
+    p2 = np.zeros((N, E)); p2[:, 0] = 0.6; p2[:, 1] = 0.4
+    te2 = np.tile([[0, 1]], (N, 1))
+    assert om.aux_loss(p2, te2, 0.1) == pytest.approx(0.1 * E * (0.5 * 0.6 + 0.5 * 0.4), rel=1e-14)
+
+
+@pytest.mark.parametrize("E,K", [(4, 2), (6, 3)])
+def test_backward_with_aux_loss_matches_central_differences(E, K):
+    shp, inp = small(N=7, H=8, E=E, K=K, F=12, seed=40 + E)
+    P = {k: om.f64(v).copy() for k, v in inp.items()}
+    alpha, g = 0.37, 1.7
+    grads = om.moe_backward(P["x"], P["W_r"], P["W1"], P["W3"], P["W2"], K, P["dy"],
+                            aux_alpha=alpha, aux_grad=g)
+    f = lambda: om.loss_sum(P["x"], P["W_r"], P["W1"], P["W3"], P["W2"], K, P["dy"], alpha, g)
+    for name, gk in (("x", "dx"), ("W_r", "dW_r")):
+        arr = P[name]
+        for idx in np.ndindex(arr.shape):
+            num = _fd(f, arr, idx, 1e-6)
+            assert abs(num - grads[gk][idx]) <= 1e-6 * (1 + abs(num)), (name, idx, num, grads[gk][idx])
