@@ -16,7 +16,7 @@ MOE_DEVERR_EXPERT_ID, MOE_DEVERR_TIMEOUT, MOE_DEVERR_ROWS = 1, 2, 4
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA"}
 
-P, I32, I64, SZ = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
+P, I32, I64, SZ, FL = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t, C.c_float
 
 # name -> (restype, argtypes); mirrors include/moe.h one to one
 SIGNATURES = {
@@ -25,7 +25,8 @@ SIGNATURES = {
     "moe_route_workspace_size": (SZ, [I32, I32, I32, I32, I32]),
     "moe_dispatch_meta_workspace_size": (SZ, [I32, I32, I32]),
     "moe_grouped_workspace_size": (SZ, []),
-    "moe_unpermute_router_bwd_workspace_size": (SZ, [I32, I32, I64]),
+    "moe_unpermute_router_bwd_workspace_size": (SZ, [I32, I32, I32, I64]),
+    "moe_aux_loss_workspace_size": (SZ, [I32, I32]),
     "moe_workspace_size": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
     "moe_workspace_init": (I32, [P, SZ, P]),
     "moe_get_device_status": (I32, [P, P, P]),
@@ -37,14 +38,15 @@ SIGNATURES = {
     "moe_combine_bwd": (I32, [P, P, P, P, P, P, I32, I32, I32, I32, I32, P, P, P, P]),
     "moe_grouped_swiglu_bwd": (I32, [P, P, P, P, P, P, P, P, I32, I32, I32, I64, I32,
                                      P, P, P, P, P, P, SZ, P]),
-    "moe_unpermute_router_bwd": (I32, [P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I64, I32,
-                                       P, P, P, SZ, P]),
-    "moe_layer_fwd": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P,
-                            P, SZ, P]),
-    "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
+    "moe_unpermute_router_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, FL, FL, I32, I32, I32, I32, I64,
+                                       I32, P, P, P, SZ, P]),
+    "moe_aux_loss": (I32, [P, P, I32, I32, I32, FL, P, P, P, SZ, P]),
+    "moe_layer_fwd": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, FL, P, P, P, P, P,
+                            P, P, P, SZ, P]),
+    "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, FL, FL,
                             P, P, P, P, P, P, SZ, P]),
     "moe_dispatch_meta_noalloc": (I32, [P, I32, I32, I32, P, P, P, P, P, P, P]),
-    "moe_sum_rank_ordered": (I32, [P, I32, I64, I32, C.c_float, P, P]),
+    "moe_sum_rank_ordered": (I32, [P, I32, I64, I32, FL, P, P]),
     "moe_trace_attach": (I32, [P, I32, P, P]),
     "moe_trace_detach": (I32, []),
 }

@@ -49,6 +49,9 @@ struct LayerWs {
   void* dx_perm;
   float* dlogit;
   void* ur_scratch;
+  float* probs;      // router probabilities (written when the aux loss is on)
+  void* aux_scratch;
+  void* dense_scratch;   // training only: dense router backward
   size_t total;
 };
 
@@ -72,6 +75,8 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int t
   w.route_scratch = take(route_scratch_bytes(H, E, dt));
   w.meta_scratch = take(meta_workspace_bytes(NK, E));
   w.pos = (int32_t*)take(NK * 4);
+  w.probs = (float*)take((size_t)N * E * 4);
+  w.aux_scratch = take(aux_loss_scratch(N, E));
   w.x_perm = take(P * H * eb);
   w.act = take(P * F * eb);
   w.out = take(P * H * eb);
@@ -82,6 +87,7 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int t
     w.dx_perm = take(P * H * eb);
     w.dlogit = (float*)take(NK * 4);
     w.ur_scratch = take(unpermute_router_bwd_scratch(H, E, P));
+    w.dense_scratch = take(dense_router_bwd_scratch(N, H, E));
   }
   w.total = off;
   return w;
@@ -145,8 +151,13 @@ size_t moe_dispatch_meta_workspace_size(int32_t N, int32_t K, int32_t E) {
 
 size_t moe_grouped_workspace_size(void) { return al256(kStatusBytes); }
 
-size_t moe_unpermute_router_bwd_workspace_size(int32_t H, int32_t E, int64_t P) {
-  return al256(kStatusBytes) + al256(unpermute_router_bwd_scratch(H, E, P));
+size_t moe_unpermute_router_bwd_workspace_size(int32_t N, int32_t H, int32_t E, int64_t P) {
+  return al256(kStatusBytes) + al256(unpermute_router_bwd_scratch(H, E, P)) +
+         al256(dense_router_bwd_scratch(N, H, E));
+}
+
+size_t moe_aux_loss_workspace_size(int32_t N, int32_t E) {
+  return al256(kStatusBytes) + al256(aux_loss_scratch(N, E));
 }
 
 size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
@@ -262,26 +273,42 @@ moe_status moe_grouped_swiglu_bwd(const void* d_out, const void* x_perm, const v
 moe_status moe_unpermute_router_bwd(const void* dx_perm, const float* dlogit, const void* x,
                                     const void* W_r, const int32_t* top_experts, const int32_t* pos,
                                     const int32_t* indices, const int32_t* bins,
-                                    const int32_t* padded_bins, int32_t N, int32_t H, int32_t E,
-                                    int32_t K, int64_t P, moe_dtype dt, void* dx, void* dW_r, void* ws,
-                                    size_t ws_bytes, moe_stream_t stream) {
+                                    const int32_t* padded_bins, const float* probs, float aux_alpha,
+                                    float aux_grad, int32_t N, int32_t H, int32_t E, int32_t K, int64_t P,
+                                    moe_dtype dt, void* dx, void* dW_r, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
   if (P < 0 || P % kTile != 0) return MOE_ERR_INVALID_ARG;
   const void* ptrs[] = {dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins, dx, dW_r};
   for (const void* q : ptrs)
     if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < moe_unpermute_router_bwd_workspace_size(H, E, P))
-    return MOE_ERR_WORKSPACE;
+  const bool aux = aux_alpha != 0.0f && N > 0;
+  if (aux && !probs) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_unpermute_router_bwd_workspace_size(N, H, E, P)) return MOE_ERR_WORKSPACE;
+  char* scratch = (char*)ws + al256(kStatusBytes);
+  if (aux)
+    return dense_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, bins, probs, N, H, E, K, dt, aux_alpha,
+                            aux_grad, dx, dW_r, scratch + al256(unpermute_router_bwd_scratch(H, E, P)),
+                            (cudaStream_t)stream);
   return unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins, N,
-                              H, E, K, P, dt, dx, dW_r, (char*)ws + al256(kStatusBytes),
-                              (cudaStream_t)stream);
+                              H, E, K, P, dt, dx, dW_r, scratch, (cudaStream_t)stream);
+}
+
+moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int32_t K, int32_t E,
+                        float alpha, float* loss, float* P, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (N < 0 || K <= 0 || E <= 0 || K > E) return MOE_ERR_INVALID_ARG;
+  if (E > 256) return MOE_ERR_UNSUPPORTED;
+  if (!bins || !loss || (N > 0 && !probs)) return MOE_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < moe_aux_loss_workspace_size(N, E)) return MOE_ERR_WORKSPACE;
+  return aux_loss_fwd(probs, bins, N, K, E, alpha, loss, P, (char*)ws + al256(kStatusBytes),
+                      (cudaStream_t)stream);
 }
 
 moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const void* W3, const void* W2,
                          int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
-                         int32_t training, void* y, int32_t* top_experts, float* weights,
-                         int32_t* indices, int32_t* bins, int32_t* padded_bins, void* ws,
-                         size_t ws_bytes, moe_stream_t stream) {
+                         int32_t training, float aux_alpha, float* aux_loss, void* y,
+                         int32_t* top_experts, float* weights, int32_t* indices, int32_t* bins,
+                         int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
   MOE_TRY(check_ffn(H, F, dt));
   const void* ptrs[] = {x, W_r, W1, W3, W2, y, top_experts, weights, indices, bins, padded_bins};
@@ -292,10 +319,13 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
   cudaStream_t s = (cudaStream_t)stream;
   LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
-  MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, nullptr, top_experts, weights, w.route_scratch,
-                    w.status, s));
+  const bool aux = aux_alpha != 0.0f;
+  if (aux && !aux_loss) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, aux ? w.probs : nullptr, top_experts, weights,
+                    w.route_scratch, w.status, s));
   MOE_TRY(dispatch_meta(top_experts, (int64_t)N * K, E, indices, nullptr, bins, padded_bins, w.pos,
                         w.meta_scratch, w.status, s));
+  if (aux) MOE_TRY(aux_loss_fwd(w.probs, bins, N, K, E, aux_alpha, aux_loss, nullptr, w.aux_scratch, s));
   if (N == 0) return MOE_OK;
   MOE_TRY(permute_rows(x, w.pos, bins, padded_bins, N, H, E, K, dt, w.x_perm, s));
   MOE_TRY(swiglu_any(w.x_perm, W1, W3, W2, padded_bins, E, H, F, P, dt, w.act, w.out,
@@ -307,9 +337,9 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
 moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const void* W1, const void* W3,
                          const void* W2, const int32_t* top_experts, const float* weights,
                          const int32_t* indices, const int32_t* bins, const int32_t* padded_bins,
-                         int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt, void* dx,
-                         void* dW_r, void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
-                         moe_stream_t stream) {
+                         int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
+                         float aux_alpha, float aux_grad, void* dx, void* dW_r, void* dW1, void* dW3,
+                         void* dW2, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
   MOE_TRY(check_ffn(H, F, dt));
   const void* ptrs[] = {dy, x, W_r, W1, W3, W2, top_experts, weights, indices, bins, padded_bins,
@@ -325,8 +355,12 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                            w.dlogit, w.d_out, s));
   MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, w.gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
                          w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s));
-  MOE_TRY(unpermute_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, indices, bins,
-                               padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, s));
+  if (aux_alpha != 0.0f && N > 0)
+    MOE_TRY(dense_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, bins, w.probs, N, H, E, K, dt,
+                             aux_alpha, aux_grad, dx, dW_r, w.dense_scratch, s));
+  else
+    MOE_TRY(unpermute_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, indices, bins,
+                                 padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, s));
   return MOE_OK;
 }
 

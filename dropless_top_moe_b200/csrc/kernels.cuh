@@ -40,6 +40,16 @@ moe_status unpermute_router_bwd(const void* dx_perm, const float* dlogit, const 
                                 int N, int H, int E, int K, int64_t P, moe_dtype dt, void* dx,
                                 void* dWr, void* scratch, cudaStream_t s);
 
+// aux.cu - load-balancing loss and the dense router backward it needs
+size_t aux_loss_scratch(int N, int E);
+size_t dense_router_bwd_scratch(int N, int H, int E);
+moe_status aux_loss_fwd(const float* probs, const int32_t* bins, int N, int K, int E, float alpha, float* loss,
+                        float* P, void* scratch, cudaStream_t s);
+moe_status dense_router_bwd(const void* dx_perm, const float* dlogit, const void* x, const void* W_r,
+                            const int32_t* top, const int32_t* pos, const int32_t* bins, const float* probs,
+                            int N, int H, int E, int K, moe_dtype dt, float aux_alpha, float aux_grad,
+                            void* dx, void* dWr, void* scratch, cudaStream_t s);
+
 // gemm_simt.cu - fp32 grouped GEMMs
 moe_status grouped_swiglu_simt(const void* x_perm, const void* W1, const void* W3, const void* W2,
                                const int32_t* pb, int E, int H, int F, int64_t P, moe_dtype dt,

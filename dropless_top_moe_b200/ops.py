@@ -162,20 +162,33 @@ def moe_grouped_swiglu_bwd(d_out, x_perm, act, gate_up, W1, W3, W2, padded_bins,
 
 
 def moe_unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins,
-                             ws=None):
+                             probs=None, aux_alpha: float = 0.0, aux_grad: float = 1.0, ws=None):
     N, H = x.shape
     E = W_r.shape[1]
     K = top_experts.shape[1]
     P = dx_perm.shape[0]
     dev = x.device
     if ws is None:
-        ws = workspace(load().moe_unpermute_router_bwd_workspace_size(H, E, P), dev)
+        ws = workspace(load().moe_unpermute_router_bwd_workspace_size(N, H, E, P), dev)
     dx = torch.empty(N, H, dtype=x.dtype, device=dev)
     dW_r = torch.empty(H, E, dtype=x.dtype, device=dev)
     call("moe_unpermute_router_bwd", _p(dx_perm), _p(dlogit), _p(x), _p(W_r), _p(top_experts), _p(pos),
-         _p(indices), _p(bins), _p(padded_bins), N, H, E, K, P, _dt(x), _p(dx), _p(dW_r),
-         ws.data_ptr(), ws.numel(), _stream())
+         _p(indices), _p(bins), _p(padded_bins), _p(probs), float(aux_alpha), float(aux_grad), N, H, E, K, P,
+         _dt(x), _p(dx), _p(dW_r), ws.data_ptr(), ws.numel(), _stream())
     return dx, dW_r
+
+
+def moe_aux_loss(probs, bins, K: int, alpha: float, ws=None):
+    """Load-balancing loss alpha * E * sum_i f_i * P_i; returns (loss [1], P [E])."""
+    N, E = probs.shape
+    dev = probs.device
+    if ws is None:
+        ws = workspace(load().moe_aux_loss_workspace_size(N, E), dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    P = torch.empty(E, dtype=torch.float32, device=dev)
+    call("moe_aux_loss", _p(probs), _p(bins), N, K, E, float(alpha), _p(loss), _p(P), ws.data_ptr(),
+         ws.numel(), _stream())
+    return loss, P
 
 
 class MoELayer:
@@ -186,9 +199,10 @@ class MoELayer:
     """
 
     def __init__(self, N: int, H: int, E: int, K: int, F: int, dtype=torch.bfloat16,
-                 training: bool = False, device="cuda"):
+                 training: bool = False, device="cuda", aux_alpha: float = 0.0):
         self.N, self.H, self.E, self.K, self.F = N, H, E, K, F
         self.dtype, self.training = dtype, training
+        self.aux_alpha = float(aux_alpha)
         self.device = torch.device(device)
         self.dt = _DT[dtype]
         nbytes = load().moe_workspace_size(N, H, E, K, F, self.dt, int(training))
@@ -202,12 +216,14 @@ class MoELayer:
         self.indices = torch.empty(N * K, dtype=torch.int32, device=dev)
         self.bins = torch.empty(E, dtype=torch.int32, device=dev)
         self.padded_bins = torch.empty(E, dtype=torch.int32, device=dev)
+        self.aux_loss = torch.zeros(1, dtype=torch.float32, device=dev)
         self._grads = None
 
     def forward(self, x, W_r, W1, W3, W2, y=None):
         y = self.y if y is None else y
         call("moe_layer_fwd", _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), self.N, self.H, self.E, self.K,
-             self.F, self.dt, int(self.training), _p(y), _p(self.top_experts), _p(self.weights),
+             self.F, self.dt, int(self.training), self.aux_alpha, _p(self.aux_loss), _p(y),
+             _p(self.top_experts), _p(self.weights),
              _p(self.indices), _p(self.bins), _p(self.padded_bins), self.ws.data_ptr(),
              self.ws.numel(), _stream())
         return y
@@ -223,13 +239,15 @@ class MoELayer:
                            "dW2": torch.empty(E, F, H, dtype=dt, device=dev)}
         return self._grads
 
-    def backward(self, dy, x, W_r, W1, W3, W2, grads=None):
+    def backward(self, dy, x, W_r, W1, W3, W2, grads=None, aux_grad: float = 1.0):
+        """Gradients of sum(y * dy) (+ aux_grad * aux_loss when aux_alpha != 0)."""
         if not self.training:
             raise RuntimeError("layer was built with training=False")
         g = self.grad_buffers() if grads is None else grads
         call("moe_layer_bwd", _p(dy), _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), _p(self.top_experts),
              _p(self.weights), _p(self.indices), _p(self.bins), _p(self.padded_bins), self.N, self.H,
-             self.E, self.K, self.F, self.dt, _p(g["dx"]), _p(g["dW_r"]), _p(g["dW1"]), _p(g["dW3"]),
+             self.E, self.K, self.F, self.dt, self.aux_alpha, float(aux_grad), _p(g["dx"]), _p(g["dW_r"]),
+             _p(g["dW1"]), _p(g["dW3"]),
              _p(g["dW2"]), self.ws.data_ptr(), self.ws.numel(), _stream())
         return g
 

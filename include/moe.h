@@ -209,38 +209,65 @@ moe_status moe_grouped_swiglu_bwd(const void* d_out, const void* x_perm, const v
  *   dW_r[:, e] = sum over assignments i of expert e, in sorted order, of
  *                dlogit_i * x[token(i)]
  * (sums in fixed order, fp32).  indices/bins/padded_bins from
- * moe_dispatch_meta; P = rows of dx_perm.  ws: moe_unpermute_router_bwd_workspace_size.
+ * moe_dispatch_meta; P = rows of dx_perm.
+ * With aux_alpha != 0 the router also receives the gradient of
+ * aux_grad * L_aux (see moe_aux_loss): every logit gets
+ *   a[t,e] = aux_grad*aux_alpha*E/N * probs[t,e] * (f_e - sum_i f_i probs[t,i]),
+ * f_e = count_e / (N*K), and the router terms use the dense
+ * D = a + (dlogit scattered to the kept experts):
+ *   dx[t] = sum_k dx_perm[pos[t*K+k]] + sum_e D[t,e] W_r[:,e],  dW_r = x^T D
+ * (fixed-order fp32 reductions); probs [N,E] float32 is then required.
+ * ws: moe_unpermute_router_bwd_workspace_size bytes.
  *   dx [N,H]; dW_r [H,E] (dt). */
-size_t moe_unpermute_router_bwd_workspace_size(int32_t H, int32_t E, int64_t P);
+size_t moe_unpermute_router_bwd_workspace_size(int32_t N, int32_t H, int32_t E, int64_t P);
 moe_status moe_unpermute_router_bwd(const void* dx_perm, const float* dlogit, const void* x,
                                     const void* W_r, const int32_t* top_experts,
                                     const int32_t* pos, const int32_t* indices,
-                                    const int32_t* bins, const int32_t* padded_bins, int32_t N,
+                                    const int32_t* bins, const int32_t* padded_bins,
+                                    const float* probs, float aux_alpha, float aux_grad, int32_t N,
                                     int32_t H, int32_t E, int32_t K, int64_t P, moe_dtype dt,
                                     void* dx, void* dW_r, void* ws, size_t ws_bytes,
                                     moe_stream_t stream);
+
+/* Auxiliary load-balancing loss ("MoE computation principle and execution",
+ * sec. 4.2): *loss = alpha * E * sum_i f_i * P_i with f_i = count_i / (N*K)
+ * (count_i from bins) and P_i = mean over tokens of probs[:, i].  Column sums
+ * run over 256-token chunks in increasing order, then over the chunks in
+ * order, then a fixed pairwise tree over experts: deterministic.
+ *   probs [N,E] float32 (moe_route's probs); bins [E]; loss: device float;
+ *   P: NULL or device float [E] receiving P_i.  ws: moe_aux_loss_workspace_size. */
+size_t moe_aux_loss_workspace_size(int32_t N, int32_t E);
+moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int32_t K, int32_t E,
+                        float alpha, float* loss, float* P, void* ws, size_t ws_bytes,
+                        moe_stream_t stream);
 
 /* Whole layer forward: route -> dispatch_meta -> permute -> grouped SwiGLU
  * -> combine, all on `stream`, no host synchronisation.
  *   y [N,H] (dt); top_experts [N,K]; weights [N,K]; indices [N*K];
  *   bins, padded_bins [E] (all outputs required).
+ *   aux_alpha != 0 also computes the load-balancing loss into *aux_loss (a
+ *   device float, see moe_aux_loss) and keeps the router probabilities in the
+ *   workspace for the backward pass; aux_alpha = 0 skips both.
  * ws: moe_workspace_size(..., training) bytes; with training != 0 it keeps
  * what moe_layer_bwd reads. */
 moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const void* W3,
                          const void* W2, int32_t N, int32_t H, int32_t E, int32_t K, int32_t F,
-                         moe_dtype dt, int32_t training, void* y, int32_t* top_experts,
-                         float* weights, int32_t* indices, int32_t* bins, int32_t* padded_bins,
-                         void* ws, size_t ws_bytes, moe_stream_t stream);
+                         moe_dtype dt, int32_t training, float aux_alpha, float* aux_loss, void* y,
+                         int32_t* top_experts, float* weights, int32_t* indices, int32_t* bins,
+                         int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Whole layer backward for the forward run last with this workspace
  * (training != 0).  dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F],
- * dW2 [E,F,H], all dt, overwritten. */
+ * dW2 [E,F,H], all dt, overwritten.  aux_alpha must equal the forward's;
+ * when non-zero, aux_grad = dObjective/dL_aux scales the load-balancing
+ * loss's gradient, which is added to the router's (dense router backward). */
 moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const void* W1,
                          const void* W3, const void* W2, const int32_t* top_experts,
                          const float* weights, const int32_t* indices, const int32_t* bins,
                          const int32_t* padded_bins, int32_t N, int32_t H, int32_t E, int32_t K,
-                         int32_t F, moe_dtype dt, void* dx, void* dW_r, void* dW1, void* dW3,
-                         void* dW2, void* ws, size_t ws_bytes, moe_stream_t stream);
+                         int32_t F, moe_dtype dt, float aux_alpha, float aux_grad, void* dx,
+                         void* dW_r, void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
+                         moe_stream_t stream);
 
 /* Local step of a deterministic data-parallel gradient all-reduce (replicas of
  * the layer on several GPUs each hold gradients of their own tokens; a

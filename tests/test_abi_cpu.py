@@ -76,7 +76,8 @@ def test_route_rejects_bad_shapes(lib):
 
 
 def test_layer_rejects_bad_arguments(lib):
-    args = [FAKE] * 5 + [64, 128, 4, 2, 256, MOE_BF16, 0] + [FAKE] * 6
+    # x W_r W1 W3 W2 | N H E K F dt training aux_alpha aux_loss | y top w idx bins pbins
+    args = [FAKE] * 5 + [64, 128, 4, 2, 256, MOE_BF16, 0, 0.0, None] + [FAKE] * 6
     assert lib.moe_layer_fwd(*args, FAKE, 1024, None) == MOE_ERR_WORKSPACE
     bad = list(args)
     bad[0] = None
@@ -86,6 +87,9 @@ def test_layer_rejects_bad_arguments(lib):
     assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_UNSUPPORTED
     bad = list(args)
     bad[8] = 5     # K > E
+    assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_INVALID_ARG
+    bad = list(args)
+    bad[12] = 0.01  # aux loss requested without an output pointer
     assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_INVALID_ARG
 
 

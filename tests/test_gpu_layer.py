@@ -135,3 +135,40 @@ def test_layer_is_bitwise_deterministic():
                     [g[k].clone() for k in ("dx", "dW_r", "dW1", "dW3", "dW2")])
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+AUX = [small_shape("aux_f32", N=256, H=64, E=8, K=2, F=96, dtype="f32", training=True),
+       small_shape("aux_bf16", N=700, H=256, E=64, K=4, F=256, training=True),
+       small_shape("aux_bf16_e8", N=333, H=128, E=8, K=2, F=128, training=True)]
+
+
+@pytest.mark.parametrize("shape", AUX, ids=lambda s: s.name)
+def test_layer_with_load_balancing_loss(shape):
+    alpha, g = 0.01, 1.7
+    c = make_case(shape, seed=8, with_dy=True)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=True, aux_alpha=alpha)
+    layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    grads = layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"], aux_grad=g)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    check_routing_and_meta(layer, shape, ref)
+    la = om.aux_loss(ref["probs"], ref["top_experts"], alpha)
+    assert abs(layer.aux_loss.item() - la) <= 1e-4 * abs(la)
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                         c["dy"].cpu(), routing=ref, aux_alpha=alpha, aux_grad=g)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(grads[k], gr[k], shape.dtype, k)
+
+
+def test_aux_loss_stage_matches_oracle():
+    shape = small_shape("aux_stage", N=1000, H=256, E=64, K=6, skew="zipf", skew_param=1.0)
+    c = make_case(shape, seed=9)
+    r = moe.moe_route(c["x"], c["W_r"], shape.K, want_probs=True)
+    m = moe.moe_dispatch_meta(r["top_experts"], shape.E)
+    loss, P = moe.moe_aux_loss(r["probs"], m["bins"], shape.K, 0.05)
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    la = om.aux_loss(ref["probs"], ref["top_experts"], 0.05)
+    assert abs(loss.item() - la) <= 1e-4 * abs(la)
+    assert_scaled(P, ref["probs"].mean(axis=0), "f32", "P")
