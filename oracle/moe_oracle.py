@@ -138,11 +138,35 @@ def round_up(n, m: int = TILE):
     return ((np.asarray(n, dtype=np.int64) + m - 1) // m) * m
 
 
-def dispatch_meta(top_experts, E: int) -> dict:
+def capacity_from_factor(N: int, E: int, capacity_factor: float) -> int:
+    """Per-expert capacity as the icman page states it (sec. 3.4):
+    ceil(N / E * capacity_factor), N the tokens of the batch."""
+    import math
+    return int(math.ceil(N / E * capacity_factor))
+
+
+def kept_mask(top_experts, E: int, capacity: int) -> np.ndarray:
+    """Token-dropping variant: each expert keeps its first `capacity`
+    assignments in increasing flat id t*K + k and drops the rest
+    (capacity 0 = dropless, everything kept)."""
+    te = np.asarray(top_experts)
+    flat = te.reshape(-1)
+    keep = np.ones(flat.size, dtype=bool)
+    if capacity > 0:
+        seen = np.zeros(E, dtype=np.int64)
+        for i, e in enumerate(flat):
+            if seen[e] >= capacity:
+                keep[i] = False
+            seen[e] += 1
+    return keep.reshape(te.shape)
+
+
+def dispatch_meta(top_experts, E: int, capacity: int = 0) -> dict:
     """Sort / histogram / cumsum / round-up / cumsum (MegaBlocks sec. 2.1, 2.3).
 
     Flat assignment id i = t*K + k.  The sort is a counting sort that visits i
-    in increasing order, so it is stable.
+    in increasing order, so it is stable.  With capacity > 0 only the kept
+    assignments (kept_mask) are counted and placed; dropped ones get pos -1.
       hist[e]        number of assignments to expert e
       bins[e]        inclusive cumsum of hist
       padded_bins[e] inclusive cumsum of round_up(hist, 128)
@@ -150,19 +174,24 @@ def dispatch_meta(top_experts, E: int) -> dict:
       bin_ids[j]     expert of indices[j]
       pos[i]         padded row of assignment i
     """
+    keep = kept_mask(top_experts, E, capacity).reshape(-1)
     te = np.asarray(top_experts, dtype=np.int64).reshape(-1)
     hist = np.zeros(E, dtype=np.int64)
-    for e in te:
-        hist[e] += 1
+    for e, kp in zip(te, keep):
+        if kp:
+            hist[e] += 1
     bins = np.cumsum(hist)
     padded_bins = np.cumsum(round_up(hist))
     sorted_start = bins - hist
     padded_start = padded_bins - round_up(hist)
     fill = np.zeros(E, dtype=np.int64)
-    indices = np.zeros(te.size, dtype=np.int64)
-    bin_ids = np.zeros(te.size, dtype=np.int64)
-    pos = np.zeros(te.size, dtype=np.int64)
+    n_kept = int(hist.sum())
+    indices = np.zeros(n_kept, dtype=np.int64)
+    bin_ids = np.zeros(n_kept, dtype=np.int64)
+    pos = np.full(te.size, -1, dtype=np.int64)
     for i, e in enumerate(te):
+        if not keep[i]:
+            continue
         r = fill[e]
         fill[e] += 1
         indices[sorted_start[e] + r] = i
@@ -241,16 +270,20 @@ def combine(O, weights, pos, N: int, K: int):
 
 
 def moe_forward(x, W_r, W1, W3, W2, K: int, routing: dict | None = None,
-                tokens=None) -> dict:
+                tokens=None, capacity: int = 0) -> dict:
     """Whole layer, written as the per-expert loop of the LLaMA MoE tutorial
     (sec. 2.3): for each expert find its (token, slot) pairs, run the expert
     on those tokens and index-add the weighted outputs.
 
     `routing` may carry a precomputed route(); `tokens` restricts y to a subset
     of token ids (y for token t depends only on x[t] once routing is fixed).
+    capacity > 0 gives the token-dropping variant: dropped (token, expert)
+    pairs contribute nothing (icman sec. 3.4; kept_mask for which are kept).
     """
     r = routing if routing is not None else route(x, W_r, K)
     te, w = r["top_experts"], r["weights"]
+    if capacity > 0:
+        w = np.where(kept_mask(te, W1.shape[0], capacity), w, 0.0)
     xv = f64(x)
     N = xv.shape[0]
     tok = np.arange(N) if tokens is None else np.asarray(tokens, dtype=np.int64)
@@ -296,7 +329,8 @@ def aux_loss(probs, top_experts, alpha: float, N_total: int | None = None) -> fl
 # -------------------------------------------------------------- backward ---
 
 def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
-                 tokens=None, aux_alpha: float = 0.0, aux_grad: float = 1.0) -> dict:
+                 tokens=None, aux_alpha: float = 0.0, aux_grad: float = 1.0,
+                 capacity: int = 0) -> dict:
     """Gradients of sum(y * dy) by the chain rule of the forward definition.
 
     Per token t and slot k with expert e (forward g = x W1_e, u = x W3_e,
@@ -321,6 +355,7 @@ def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
     E, _, F = W1.shape
     W_rv = f64(W_r)
     te, w, probs = r["top_experts"][tok], r["weights"][tok], r["probs"][tok]
+    kept = kept_mask(r["top_experts"], E, capacity)[tok]   # all True when dropless
     xs, dys = xv[tok], dyv[tok]
     n = tok.size
     dx = np.zeros((n, H))
@@ -329,7 +364,7 @@ def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
     dW2 = np.zeros((E, F, H))
     dw = np.zeros((n, K))
     for e in range(E):
-        rows, slots = np.nonzero(te == e)
+        rows, slots = np.nonzero((te == e) & kept)
         if rows.size == 0:
             continue
         W1e, W3e, W2e = f64(W1[e]), f64(W3[e]), f64(W2[e])
@@ -364,10 +399,11 @@ def moe_backward(x, W_r, W1, W3, W2, K: int, dy, routing: dict | None = None,
             "dw": dw, "dlogits": dlogits, "tokens": tok}
 
 
-def loss_sum(x, W_r, W1, W3, W2, K, dy, aux_alpha: float = 0.0, aux_grad: float = 1.0) -> float:
+def loss_sum(x, W_r, W1, W3, W2, K, dy, aux_alpha: float = 0.0, aux_grad: float = 1.0,
+             capacity: int = 0) -> float:
     """sum(y * dy) (+ aux_grad * aux_loss) with routing recomputed; used by the
     finite-difference pins."""
-    out = moe_forward(x, W_r, W1, W3, W2, K)
+    out = moe_forward(x, W_r, W1, W3, W2, K, capacity=capacity)
     v = float(np.sum(out["y"] * f64(dy)))
     if aux_alpha != 0.0:
         r = out["routing"]

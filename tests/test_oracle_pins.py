@@ -295,3 +295,57 @@ def test_backward_with_aux_loss_matches_central_differences(E, K):
         for idx in np.ndindex(arr.shape):
             num = _fd(f, arr, idx, 1e-6)
             assert abs(num - grads[gk][idx]) <= 1e-6 * (1 + abs(num)), (name, idx, num, grads[gk][idx])
+
+
+# ------------------------------------------------------ token-dropping variant
+
+def test_capacity_large_enough_equals_dropless():
+    shp, inp = small(N=60, E=4, K=2)
+    a = om.moe_forward(inp["x"], inp["W_r"], inp["W1"], inp["W3"], inp["W2"], 2)["y"]
+    b = om.moe_forward(inp["x"], inp["W_r"], inp["W1"], inp["W3"], inp["W2"], 2, capacity=10 ** 6)["y"]
+    np.testing.assert_array_equal(a, b)
+
+
+def test_capacity_keeps_first_assignments_brute_force():
+    te = np.array([[0, 1], [1, 0], [0, 2], [2, 0], [1, 2]])
+    # expert 0 sees flat ids 0, 3, 4, 7; expert 1: 1, 2, 8; expert 2: 5, 6, 9
+    keep = om.kept_mask(te, 3, 2)
+    np.testing.assert_array_equal(keep, [[1, 1], [1, 1], [0, 1], [1, 0], [0, 0]])
+    m = om.dispatch_meta(te, 3, capacity=2)
+    np.testing.assert_array_equal(m["hist"], [2, 2, 2])
+    np.testing.assert_array_equal(m["indices"], [0, 3, 1, 2, 5, 6])
+    np.testing.assert_array_equal(m["pos"], [0, 128, 129, 1, -1, 256, 257, -1, -1, -1])
+    assert om.capacity_from_factor(1000, 8, 1.25) == 157     # ceil(1000 / 8 * 1.25)
+
+
+def test_capacity_layer_equals_masked_sum():
+    """With dropping, y is the per-expert loop restricted to kept pairs."""
+    shp, inp = small(N=90, E=4, K=2)
+    r = om.route(inp["x"], inp["W_r"], 2)
+    cap = 30
+    y = om.moe_forward(inp["x"], inp["W_r"], inp["W1"], inp["W3"], inp["W2"], 2, routing=r, capacity=cap)["y"]
+    keep = om.kept_mask(r["top_experts"], 4, cap)
+    x = om.f64(inp["x"])
+    ref = np.zeros_like(x)
+    for t in range(90):
+        for k in range(2):
+            if keep[t, k]:
+                e = r["top_experts"][t, k]
+                ref[t] += r["weights"][t, k] * om.swiglu_ffn(x[t:t + 1], om.f64(inp["W1"][e]),
+                                                             om.f64(inp["W3"][e]), om.f64(inp["W2"][e]))[0]
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_backward_with_capacity_matches_central_differences():
+    shp, inp = small(N=8, H=8, E=3, K=2, F=12, seed=77)
+    P = {k: om.f64(v).copy() for k, v in inp.items()}
+    cap = 4       # 16 assignments over 3 experts: some experts overflow
+    r = om.route(P["x"], P["W_r"], 2)
+    assert not om.kept_mask(r["top_experts"], 3, cap).all()
+    grads = om.moe_backward(P["x"], P["W_r"], P["W1"], P["W3"], P["W2"], 2, P["dy"], capacity=cap)
+    f = lambda: om.loss_sum(P["x"], P["W_r"], P["W1"], P["W3"], P["W2"], 2, P["dy"], capacity=cap)
+    for name, gk in (("x", "dx"), ("W_r", "dW_r"), ("W1", "dW1"), ("W2", "dW2")):
+        arr = P[name]
+        for idx in list(np.ndindex(arr.shape))[::3]:
+            num = _fd(f, arr, idx, 1e-6)
+            assert abs(num - grads[gk][idx]) <= 1e-6 * (1 + abs(num)), (name, idx, num, grads[gk][idx])
