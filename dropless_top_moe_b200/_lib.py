@@ -31,7 +31,7 @@ SIGNATURES = {
     "moe_workspace_init": (I32, [P, SZ, P]),
     "moe_get_device_status": (I32, [P, P, P]),
     "moe_route": (I32, [P, P, I32, I32, I32, I32, I32, P, P, P, P, P, SZ, P]),
-    "moe_dispatch_meta": (I32, [P, I32, I32, I32, P, P, P, P, P, P, SZ, P]),
+    "moe_dispatch_meta": (I32, [P, I32, I32, I32, I32, P, P, P, P, P, P, SZ, P]),
     "moe_permute": (I32, [P, P, P, P, I32, I32, I32, I32, I32, P, P]),
     "moe_grouped_swiglu": (I32, [P, P, P, P, P, I32, I32, I32, I64, I32, P, P, P, P, SZ, P]),
     "moe_combine": (I32, [P, P, P, I32, I32, I32, I32, P, P]),
@@ -41,10 +41,10 @@ SIGNATURES = {
     "moe_unpermute_router_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, FL, FL, I32, I32, I32, I32, I64,
                                        I32, P, P, P, SZ, P]),
     "moe_aux_loss": (I32, [P, P, I32, I32, I32, FL, P, P, P, SZ, P]),
-    "moe_layer_fwd": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, FL, P, P, P, P, P,
-                            P, P, P, SZ, P]),
-    "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, FL, FL,
-                            P, P, P, P, P, P, SZ, P]),
+    "moe_layer_fwd": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, FL, P, P, P, P,
+                            P, P, P, P, SZ, P]),
+    "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, FL,
+                            FL, P, P, P, P, P, P, SZ, P]),
     "moe_dispatch_meta_noalloc": (I32, [P, I32, I32, I32, P, P, P, P, P, P, P]),
     "moe_sum_rank_ordered": (I32, [P, I32, I64, I32, FL, P, P]),
     "moe_trace_attach": (I32, [P, I32, P, P]),

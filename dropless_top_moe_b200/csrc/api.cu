@@ -195,15 +195,16 @@ moe_status moe_route(const void* x, const void* W_r, int32_t N, int32_t H, int32
 }
 
 moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, int32_t E,
-                             int32_t* indices, int32_t* bin_ids, int32_t* bins, int32_t* padded_bins,
-                             int32_t* pos, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  if (N < 0 || K <= 0 || E <= 0 || K > E) return MOE_ERR_INVALID_ARG;
+                             int32_t capacity, int32_t* indices, int32_t* bin_ids, int32_t* bins,
+                             int32_t* padded_bins, int32_t* pos, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+  if (N < 0 || K <= 0 || E <= 0 || K > E || capacity < 0) return MOE_ERR_INVALID_ARG;
   if (E > 256) return MOE_ERR_UNSUPPORTED;
   if (!padded_bins || (N > 0 && (!top_experts || !pos))) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < moe_dispatch_meta_workspace_size(N, K, E)) return MOE_ERR_WORKSPACE;
   char* base = (char*)ws;
   return dispatch_meta(top_experts, (int64_t)N * K, E, indices, bin_ids, bins, padded_bins, pos,
-                       base + al256(kStatusBytes), (int*)ws, (cudaStream_t)stream);
+                       base + al256(kStatusBytes), (int*)ws, (cudaStream_t)stream, capacity);
 }
 
 moe_status moe_permute(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* padded_bins,
@@ -306,7 +307,7 @@ moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int3
 
 moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const void* W3, const void* W2,
                          int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
-                         int32_t training, float aux_alpha, float* aux_loss, void* y,
+                         int32_t training, int32_t capacity, float aux_alpha, float* aux_loss, void* y,
                          int32_t* top_experts, float* weights, int32_t* indices, int32_t* bins,
                          int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
@@ -320,11 +321,11 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
   LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
   const bool aux = aux_alpha != 0.0f;
-  if (aux && !aux_loss) return MOE_ERR_INVALID_ARG;
+  if ((aux && !aux_loss) || capacity < 0) return MOE_ERR_INVALID_ARG;
   MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, aux ? w.probs : nullptr, top_experts, weights,
                     w.route_scratch, w.status, s));
   MOE_TRY(dispatch_meta(top_experts, (int64_t)N * K, E, indices, nullptr, bins, padded_bins, w.pos,
-                        w.meta_scratch, w.status, s));
+                        w.meta_scratch, w.status, s, capacity));
   if (aux) MOE_TRY(aux_loss_fwd(w.probs, bins, N, K, E, aux_alpha, aux_loss, nullptr, w.aux_scratch, s));
   if (N == 0) return MOE_OK;
   MOE_TRY(permute_rows(x, w.pos, bins, padded_bins, N, H, E, K, dt, w.x_perm, s));
@@ -338,8 +339,9 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                          const void* W2, const int32_t* top_experts, const float* weights,
                          const int32_t* indices, const int32_t* bins, const int32_t* padded_bins,
                          int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
-                         float aux_alpha, float aux_grad, void* dx, void* dW_r, void* dW1, void* dW3,
-                         void* dW2, void* ws, size_t ws_bytes, moe_stream_t stream) {
+                         int32_t capacity, float aux_alpha, float aux_grad, void* dx, void* dW_r,
+                         void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
   MOE_TRY(check_ffn(H, F, dt));
   const void* ptrs[] = {dy, x, W_r, W1, W3, W2, top_experts, weights, indices, bins, padded_bins,
@@ -355,7 +357,9 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                            w.dlogit, w.d_out, s));
   MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, w.gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
                          w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s));
-  if (aux_alpha != 0.0f && N > 0)
+  // the sparse router backward walks the kept assignments only; the aux loss
+  // and dropped assignments need every (token, expert) logit: dense path
+  if ((aux_alpha != 0.0f || capacity > 0) && N > 0)
     MOE_TRY(dense_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, bins, w.probs, N, H, E, K, dt,
                              aux_alpha, aux_grad, dx, dW_r, w.dense_scratch, s));
   else

@@ -21,7 +21,7 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
 size_t meta_workspace_bytes(int64_t NK, int E);
 moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices, int32_t* bin_ids,
                          int32_t* bins, int32_t* padded_bins, int32_t* pos, void* scratch,
-                         int* status, cudaStream_t s);
+                         int* status, cudaStream_t s, int capacity = 0);
 
 // permute.cu
 moe_status permute_rows(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* pb,

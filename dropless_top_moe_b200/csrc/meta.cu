@@ -42,7 +42,7 @@ meta_count_kernel(const int32_t* __restrict__ top, int64_t NK, int E, int32_t* _
 
 // One block of 256 threads (E <= 256).
 __global__ void __launch_bounds__(256)
-meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
+meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E, int capacity,
                  int32_t* __restrict__ bins, int32_t* __restrict__ padded_bins,
                  int32_t* __restrict__ sorted_start, int32_t* __restrict__ padded_start) {
   __shared__ int s_a[256], s_b[256];
@@ -55,6 +55,8 @@ meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
       total += v;
     }
   }
+  // token-dropping variant: only the first `capacity` assignments are kept
+  if (capacity > 0 && total > capacity) total = capacity;
   const int padded = (int)round_up(total, kTile);
   s_a[e] = (e < E) ? total : 0;
   s_b[e] = (e < E) ? padded : 0;
@@ -77,7 +79,7 @@ meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
 }
 
 __global__ void __launch_bounds__(kMetaPlaceThreads)
-meta_place_kernel(const int32_t* __restrict__ top, int64_t NK, int E,
+meta_place_kernel(const int32_t* __restrict__ top, int64_t NK, int E, int capacity,
                   const int32_t* __restrict__ chunk_offsets, const int32_t* __restrict__ sorted_start,
                   const int32_t* __restrict__ padded_start, int32_t* __restrict__ indices,
                   int32_t* __restrict__ bin_ids, int32_t* __restrict__ pos) {
@@ -113,10 +115,15 @@ meta_place_kernel(const int32_t* __restrict__ top, int64_t NK, int E,
     __syncthreads();
     if (i < NK) {
       if (e >= 0) {
+        // rank among all of expert e's assignments, in flat-id order
         const int rank = s_base[e] + s_warp[warp * E + e] + rank_w;
-        if (indices) indices[sorted_start[e] + rank] = (int32_t)i;
-        if (bin_ids) bin_ids[sorted_start[e] + rank] = e;
-        pos[i] = padded_start[e] + rank;
+        if (capacity > 0 && rank >= capacity) {
+          pos[i] = -1;                      // dropped: beyond the expert's capacity
+        } else {
+          if (indices) indices[sorted_start[e] + rank] = (int32_t)i;
+          if (bin_ids) bin_ids[sorted_start[e] + rank] = e;
+          pos[i] = padded_start[e] + rank;
+        }
       } else {
         pos[i] = -1;
       }
@@ -134,20 +141,20 @@ size_t meta_workspace_bytes(int64_t NK, int E) {
 
 moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices, int32_t* bin_ids,
                          int32_t* bins, int32_t* padded_bins, int32_t* pos, void* scratch,
-                         int* status, cudaStream_t s) {
+                         int* status, cudaStream_t s, int capacity) {
   const int n_chunks = (int)cdiv(NK > 0 ? NK : 1, kMetaChunk);
   int32_t* chunk_counts = (int32_t*)scratch;
   int32_t* sorted_start = chunk_counts + (size_t)n_chunks * E;
   int32_t* padded_start = sorted_start + E;
   MOE_TRACED("meta_count", s, (meta_count_kernel<<<n_chunks, 256, E * sizeof(int), s>>>(top, NK, E, chunk_counts, status)));
   MOE_LAUNCH_CHECK();
-  MOE_TRACED("meta_scan", s, (meta_scan_kernel<<<1, 256, 0, s>>>(chunk_counts, n_chunks, E, bins, padded_bins, sorted_start,
+  MOE_TRACED("meta_scan", s, (meta_scan_kernel<<<1, 256, 0, s>>>(chunk_counts, n_chunks, E, capacity, bins, padded_bins, sorted_start,
                                      padded_start)));
   MOE_LAUNCH_CHECK();
   if (NK > 0) {
     const size_t smem = (size_t)(kMetaPlaceThreads / 32 + 2) * E * sizeof(int);
     cudaFuncSetAttribute(meta_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    MOE_TRACED("meta_place", s, (meta_place_kernel<<<n_chunks, kMetaPlaceThreads, smem, s>>>(top, NK, E, chunk_counts,
+    MOE_TRACED("meta_place", s, (meta_place_kernel<<<n_chunks, kMetaPlaceThreads, smem, s>>>(top, NK, E, capacity, chunk_counts,
                                                                 sorted_start, padded_start, indices,
                                                                 bin_ids, pos)));
     MOE_LAUNCH_CHECK();

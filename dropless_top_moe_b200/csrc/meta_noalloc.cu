@@ -52,5 +52,5 @@ extern "C" moe_status moe_dispatch_meta_noalloc(const int32_t* top_experts, int3
   // The count kernel writes every chunk count (zeros included) and the scan
   // writes every start, so nothing in the array needs clearing first.
   return moe::dispatch_meta(top_experts, NK, E, indices, bin_ids, bins, padded_bins, pos,
-                            g_scratch_addr[dev], status, (cudaStream_t)stream);
+                            g_scratch_addr[dev], status, (cudaStream_t)stream, 0);
 }

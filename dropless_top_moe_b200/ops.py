@@ -78,7 +78,7 @@ def moe_route(x, W_r, K: int, want_logits: bool = False, want_probs: bool = Fals
     return out
 
 
-def moe_dispatch_meta(top_experts, E: int, ws=None) -> dict:
+def moe_dispatch_meta(top_experts, E: int, ws=None, capacity: int = 0) -> dict:
     N, K = top_experts.shape
     dev = top_experts.device
     if ws is None:
@@ -88,7 +88,7 @@ def moe_dispatch_meta(top_experts, E: int, ws=None) -> dict:
     out["bins"] = torch.empty(E, dtype=torch.int32, device=dev)
     out["padded_bins"] = torch.empty(E, dtype=torch.int32, device=dev)
     out["ws"] = ws
-    call("moe_dispatch_meta", _p(top_experts), N, K, E, _p(out["indices"]), _p(out["bin_ids"]),
+    call("moe_dispatch_meta", _p(top_experts), N, K, E, int(capacity), _p(out["indices"]), _p(out["bin_ids"]),
          _p(out["bins"]), _p(out["padded_bins"]), _p(out["pos"]), ws.data_ptr(), ws.numel(),
          _stream())
     return out
@@ -199,10 +199,11 @@ class MoELayer:
     """
 
     def __init__(self, N: int, H: int, E: int, K: int, F: int, dtype=torch.bfloat16,
-                 training: bool = False, device="cuda", aux_alpha: float = 0.0):
+                 training: bool = False, device="cuda", aux_alpha: float = 0.0, capacity: int = 0):
         self.N, self.H, self.E, self.K, self.F = N, H, E, K, F
         self.dtype, self.training = dtype, training
         self.aux_alpha = float(aux_alpha)
+        self.capacity = int(capacity)   # 0 = dropless
         self.device = torch.device(device)
         self.dt = _DT[dtype]
         nbytes = load().moe_workspace_size(N, H, E, K, F, self.dt, int(training))
@@ -222,7 +223,7 @@ class MoELayer:
     def forward(self, x, W_r, W1, W3, W2, y=None):
         y = self.y if y is None else y
         call("moe_layer_fwd", _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), self.N, self.H, self.E, self.K,
-             self.F, self.dt, int(self.training), self.aux_alpha, _p(self.aux_loss), _p(y),
+             self.F, self.dt, int(self.training), self.capacity, self.aux_alpha, _p(self.aux_loss), _p(y),
              _p(self.top_experts), _p(self.weights),
              _p(self.indices), _p(self.bins), _p(self.padded_bins), self.ws.data_ptr(),
              self.ws.numel(), _stream())
@@ -246,7 +247,8 @@ class MoELayer:
         g = self.grad_buffers() if grads is None else grads
         call("moe_layer_bwd", _p(dy), _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), _p(self.top_experts),
              _p(self.weights), _p(self.indices), _p(self.bins), _p(self.padded_bins), self.N, self.H,
-             self.E, self.K, self.F, self.dt, self.aux_alpha, float(aux_grad), _p(g["dx"]), _p(g["dW_r"]),
+             self.E, self.K, self.F, self.dt, self.capacity, self.aux_alpha, float(aux_grad), _p(g["dx"]),
+             _p(g["dW_r"]),
              _p(g["dW1"]), _p(g["dW3"]),
              _p(g["dW2"]), self.ws.data_ptr(), self.ws.numel(), _stream())
         return g

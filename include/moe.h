@@ -113,6 +113,11 @@ moe_status moe_route(const void* x, const void* W_r, int32_t N, int32_t H, int32
 
 /* Dispatch metadata (MegaBlocks sec. 2.1/2.3): stable sort of the N*K flat
  * assignment ids by expert, histogram, inclusive cumsums.
+ *   capacity: 0 = dropless.  > 0 gives the token-dropping variant (icman
+ *   sec. 3.4): each expert keeps its first `capacity` assignments in flat-id
+ *   order and drops the rest; counts, bins, padded_bins and indices then
+ *   cover kept assignments only (indices holds bins[E-1] entries) and dropped
+ *   assignments get pos -1.
  *   top_experts [N*K] int32 in [0,E).
  *   indices [N*K]  flat ids in expert order (stable: increasing id within an expert)
  *   bin_ids [N*K]  expert of indices[j]
@@ -123,11 +128,12 @@ moe_status moe_route(const void* x, const void* W_r, int32_t N, int32_t H, int32
  * Any output pointer except padded_bins and pos may be NULL.  Ids outside
  * [0,E) set MOE_DEVERR_EXPERT_ID; their pos is -1 and they are skipped. */
 moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, int32_t E,
-                             int32_t* indices, int32_t* bin_ids, int32_t* bins,
+                             int32_t capacity, int32_t* indices, int32_t* bin_ids, int32_t* bins,
                              int32_t* padded_bins, int32_t* pos, void* ws, size_t ws_bytes,
                              moe_stream_t stream);
 
-/* Dispatch metadata for callers that cannot allocate device memory.  The
+/* Dispatch metadata for callers that cannot allocate device memory (dropless,
+ * capacity 0).  The
  * pages have no counterpart to this entry point.  Some callers cannot call
  * cudaMalloc: code embedded in another runtime that owns all device memory
  * and gives its plugins no allocator, or a latency-critical path where an
@@ -245,6 +251,8 @@ moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int3
  * -> combine, all on `stream`, no host synchronisation.
  *   y [N,H] (dt); top_experts [N,K]; weights [N,K]; indices [N*K];
  *   bins, padded_bins [E] (all outputs required).
+ *   capacity: 0 = dropless; > 0 = token-dropping variant (see
+ *   moe_dispatch_meta): dropped (token, expert) pairs add nothing to y.
  *   aux_alpha != 0 also computes the load-balancing loss into *aux_loss (a
  *   device float, see moe_aux_loss) and keeps the router probabilities in the
  *   workspace for the backward pass; aux_alpha = 0 skips both.
@@ -252,20 +260,24 @@ moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int3
  * what moe_layer_bwd reads. */
 moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const void* W3,
                          const void* W2, int32_t N, int32_t H, int32_t E, int32_t K, int32_t F,
-                         moe_dtype dt, int32_t training, float aux_alpha, float* aux_loss, void* y,
+                         moe_dtype dt, int32_t training, int32_t capacity, float aux_alpha,
+                         float* aux_loss, void* y,
                          int32_t* top_experts, float* weights, int32_t* indices, int32_t* bins,
                          int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Whole layer backward for the forward run last with this workspace
  * (training != 0).  dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F],
- * dW2 [E,F,H], all dt, overwritten.  aux_alpha must equal the forward's;
+ * dW2 [E,F,H], all dt, overwritten.  capacity and aux_alpha must equal the
+ * forward's (dropped pairs still pass gradient to the router through the
+ * renormalised weights);
  * when non-zero, aux_grad = dObjective/dL_aux scales the load-balancing
  * loss's gradient, which is added to the router's (dense router backward). */
 moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const void* W1,
                          const void* W3, const void* W2, const int32_t* top_experts,
                          const float* weights, const int32_t* indices, const int32_t* bins,
                          const int32_t* padded_bins, int32_t N, int32_t H, int32_t E, int32_t K,
-                         int32_t F, moe_dtype dt, float aux_alpha, float aux_grad, void* dx,
+                         int32_t F, moe_dtype dt, int32_t capacity, float aux_alpha, float aux_grad,
+                         void* dx,
                          void* dW_r, void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 

@@ -76,8 +76,8 @@ def test_route_rejects_bad_shapes(lib):
 
 
 def test_layer_rejects_bad_arguments(lib):
-    # x W_r W1 W3 W2 | N H E K F dt training aux_alpha aux_loss | y top w idx bins pbins
-    args = [FAKE] * 5 + [64, 128, 4, 2, 256, MOE_BF16, 0, 0.0, None] + [FAKE] * 6
+    # x W_r W1 W3 W2 | N H E K F dt training capacity aux_alpha aux_loss | y top w idx bins pbins
+    args = [FAKE] * 5 + [64, 128, 4, 2, 256, MOE_BF16, 0, 0, 0.0, None] + [FAKE] * 6
     assert lib.moe_layer_fwd(*args, FAKE, 1024, None) == MOE_ERR_WORKSPACE
     bad = list(args)
     bad[0] = None
@@ -89,15 +89,17 @@ def test_layer_rejects_bad_arguments(lib):
     bad[8] = 5     # K > E
     assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_INVALID_ARG
     bad = list(args)
-    bad[12] = 0.01  # aux loss requested without an output pointer
+    bad[13] = 0.01  # aux loss requested without an output pointer
     assert lib.moe_layer_fwd(*bad, FAKE, 1 << 40, None) == MOE_ERR_INVALID_ARG
 
 
 def test_meta_and_grouped_reject_bad_arguments(lib):
-    assert lib.moe_dispatch_meta(FAKE, 10, 3, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
+    assert lib.moe_dispatch_meta(FAKE, 10, 3, 2, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
                                  None) == MOE_ERR_INVALID_ARG
-    assert lib.moe_dispatch_meta(FAKE, 10, 2, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+    assert lib.moe_dispatch_meta(FAKE, 10, 2, 4, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
                                  None) == MOE_ERR_WORKSPACE
+    assert lib.moe_dispatch_meta(FAKE, 10, 2, 4, -1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20,
+                                 None) == MOE_ERR_INVALID_ARG
     # P must be a multiple of 128
     assert lib.moe_grouped_swiglu(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, 100, MOE_BF16, FAKE, FAKE,
                                   None, FAKE, 4096, None) == MOE_ERR_INVALID_ARG

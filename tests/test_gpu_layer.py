@@ -172,3 +172,48 @@ def test_aux_loss_stage_matches_oracle():
     la = om.aux_loss(ref["probs"], ref["top_experts"], 0.05)
     assert abs(loss.item() - la) <= 1e-4 * abs(la)
     assert_scaled(P, ref["probs"].mean(axis=0), "f32", "P")
+
+
+CAP = [small_shape("cap_f32", N=256, H=64, E=8, K=2, F=96, dtype="f32", training=True),
+       small_shape("cap_bf16_zipf", N=900, H=256, E=16, K=4, F=256, skew="zipf", skew_param=1.0,
+                   training=True)]
+
+
+@pytest.mark.parametrize("shape", CAP, ids=lambda s: s.name)
+def test_layer_token_dropping_variant(shape):
+    cap = om.capacity_from_factor(shape.N, shape.E, 1.0)      # icman sec. 3.4 with factor 1
+    c = make_case(shape, seed=12, with_dy=True)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=True, capacity=cap)
+    y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"]).clone()
+    g = layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    np.testing.assert_array_equal(layer.top_experts.cpu().numpy(), ref["top_experts"])
+    m = om.dispatch_meta(ref["top_experts"], shape.E, capacity=cap)
+    assert m["hist"].sum() < shape.N * shape.K          # something was dropped
+    np.testing.assert_array_equal(layer.bins.cpu().numpy(), m["bins"])
+    np.testing.assert_array_equal(layer.padded_bins.cpu().numpy(), m["padded_bins"])
+    np.testing.assert_array_equal(layer.indices.cpu().numpy()[:m["indices"].size], m["indices"])
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                        routing=ref, capacity=cap)["y"]
+    assert_scaled(y, yr, shape.dtype, "y")
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                         c["dy"].cpu(), routing=ref, capacity=cap)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(g[k], gr[k], shape.dtype, k)
+
+
+def test_dispatch_meta_capacity_bit_exact():
+    g = torch.Generator().manual_seed(21)
+    te = torch.stack([torch.randperm(16, generator=g)[:3] for _ in range(3000)]).to(torch.int32)
+    te[:1500, 0] = 5                                    # overflow expert 5
+    for cap in (1, 100, 600, 10 ** 6):
+        m = moe.moe_dispatch_meta(te.cuda(), 16, capacity=cap)
+        ref = om.dispatch_meta(te.numpy(), 16, capacity=cap)
+        n = ref["indices"].size
+        for k in ("bins", "padded_bins", "pos"):
+            np.testing.assert_array_equal(m[k].cpu().numpy(), ref[k], err_msg=f"{k} cap={cap}")
+        for k in ("indices", "bin_ids"):
+            np.testing.assert_array_equal(m[k].cpu().numpy()[:n], ref[k], err_msg=f"{k} cap={cap}")
