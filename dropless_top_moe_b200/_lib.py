@@ -43,8 +43,8 @@ SIGNATURES = {
     "moe_aux_loss": (I32, [P, P, I32, I32, I32, FL, P, P, P, SZ, P]),
     "moe_layer_fwd": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, FL, P, P, P, P,
                             P, P, P, P, SZ, P]),
-    "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, FL,
-                            FL, P, P, P, P, P, P, SZ, P]),
+    "moe_layer_bwd": (I32, [P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32,
+                            FL, FL, P, P, P, P, P, P, SZ, P]),
     "moe_dispatch_meta_noalloc": (I32, [P, I32, I32, I32, P, P, P, P, P, P, P]),
     "moe_sum_rank_ordered": (I32, [P, I32, I64, I32, FL, P, P]),
     "moe_trace_attach": (I32, [P, I32, P, P]),

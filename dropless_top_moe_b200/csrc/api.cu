@@ -81,7 +81,8 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int t
   w.act = take(P * F * eb);
   w.out = take(P * H * eb);
   if (training) {
-    w.gate_up = take(2 * P * F * eb);
+    // training == 2 (memory-optimised) keeps no G, U between the passes
+    w.gate_up = training == 1 ? take(2 * P * F * eb) : nullptr;
     w.d_out = take(P * H * eb);
     w.d_gate_up = take(2 * P * F * eb);
     w.dx_perm = take(P * H * eb);
@@ -330,7 +331,7 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
   if (N == 0) return MOE_OK;
   MOE_TRY(permute_rows(x, w.pos, bins, padded_bins, N, H, E, K, dt, w.x_perm, s));
   MOE_TRY(swiglu_any(w.x_perm, W1, W3, W2, padded_bins, E, H, F, P, dt, w.act, w.out,
-                     training ? w.gate_up : nullptr, w.status, s));
+                     training == 1 ? w.gate_up : nullptr, w.status, s));
   MOE_TRY(combine_rows(w.out, weights, w.pos, N, K, H, dt, y, s));
   return MOE_OK;
 }
@@ -339,8 +340,8 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                          const void* W2, const int32_t* top_experts, const float* weights,
                          const int32_t* indices, const int32_t* bins, const int32_t* padded_bins,
                          int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
-                         int32_t capacity, float aux_alpha, float aux_grad, void* dx, void* dW_r,
-                         void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
+                         int32_t training, int32_t capacity, float aux_alpha, float aux_grad, void* dx,
+                         void* dW_r, void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
                          moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
   MOE_TRY(check_ffn(H, F, dt));
@@ -348,14 +349,29 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                         dx, dW_r, dW1, dW3, dW2};
   for (const void* q : ptrs)
     if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
-  const size_t need = moe_workspace_size(N, H, E, K, F, dt, 1);
+  if (training != 1 && training != 2) return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_workspace_size(N, H, E, K, F, dt, training);
   if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
-  LayerWs w = carve(ws, N, H, E, K, F, dt, 1);
+  LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
+  void* gate_up = w.gate_up;
+  if (training == 2) {
+    // recompute G, U (same kernel and inputs as the forward: identical bits)
+    // into the dG, dU scratch; the SwiGLU backward then runs in place there
+    gate_up = w.d_gate_up;
+    const size_t eb = elem_bytes(dt);
+    void* G = w.d_gate_up;
+    void* U = (char*)w.d_gate_up + (size_t)P * F * eb;
+    if (dt == MOE_F32)
+      MOE_TRY(gate_up_simt(w.x_perm, W1, W3, padded_bins, E, H, F, P, G, U, s));
+    else
+      MOE_TRY(gemm1_umma(w.x_perm, W1, W3, padded_bins, E, H, F, P, nullptr, G, U, w.status, s,
+                         "gate_up_recompute"));
+  }
   MOE_TRY(combine_bwd_rows(dy, w.out, weights, w.pos, bins, padded_bins, N, K, H, E, dt, nullptr,
                            w.dlogit, w.d_out, s));
-  MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, w.gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
+  MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
                          w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s));
   // the sparse router backward walks the kept assignments only; the aux loss
   // and dropped assignments need every (token, expert) logit: dense path

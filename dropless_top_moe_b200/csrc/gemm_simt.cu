@@ -91,7 +91,7 @@ gemm_rows_simt_kernel(const T* __restrict__ A0, const T* __restrict__ A1, int64_
         C0[o] = from_f<T>(acc[i][j]);
       } else if (EPI == SIMT_SWIGLU) {
         const float g = acc[i][j], u = acc2[i][j];
-        C0[o] = from_f<T>(silu_f(g) * u);
+        if (C0) C0[o] = from_f<T>(silu_f(g) * u);
         if (C1) C1[o] = from_f<T>(g);
         if (C2) C2[o] = from_f<T>(u);
       } else {  // SIMT_SWIGLU_BWD: acc = dA, aux0 = G, aux1 = U
@@ -227,6 +227,22 @@ moe_status grouped_swiglu_bwd_simt(const void* d_out, const void* x_perm, const 
   if (dt != MOE_F32) return MOE_ERR_UNSUPPORTED;
   return swiglu_bwd_simt_t<float>(d_out, x_perm, act, gate_up, W1, W3, W2, pb, E, H, F, P, d_gate_up,
                                   dW1, dW3, dW2, dx_perm, s);
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// G, U = X W1_e, X W3_e only (the backward's recompute of the saved gates).
+moe_status gate_up_simt(const void* x_perm, const void* W1, const void* W3, const int32_t* pb, int E, int H,
+                        int F, int64_t P, void* G, void* U, cudaStream_t s) {
+  typedef float T;
+  dim3 g1((unsigned)cdiv(F, kSB), (unsigned)(P / kSB));
+  MOE_TRACED("simt_gate_up_recompute", s, (gemm_rows_simt_kernel<T, SIMT_SWIGLU><<<g1, 256, 0, s>>>(
+      (const T*)x_perm, nullptr, H, (const T*)W1, (const T*)W3, (int64_t)H * F, F, 1, pb, E, H, F,
+      nullptr, (T*)G, (T*)U, F, nullptr, nullptr)));
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
 }
 
 }  // namespace moe

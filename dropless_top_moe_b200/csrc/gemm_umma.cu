@@ -297,7 +297,7 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
   constexpr int NC = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
   const int c_begin = part * (NC / 2), c_end = c_begin + NC / 2;
   if constexpr (EPI == EPI_SWIGLU) {
-    __nv_bfloat16* act = p.out0 + grow * p.ldo + tl.n0;
+    // out0 = act (NULL when only G and U are wanted: backward recompute)
 #pragma unroll 1
     for (int c = c_begin; c < c_end; c += 32) {
       uint32_t g[32], u[32];
@@ -311,7 +311,7 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
         uf[j] = __uint_as_float(u[j]);
         a[j] = silu_f(gf[j]) * uf[j];
       }
-      store_row_bf16x32(act + c, a);
+      if (p.out0) store_row_bf16x32(p.out0 + grow * p.ldo + tl.n0 + c, a);
       if (p.out1) {
         store_row_bf16x32(p.out1 + grow * p.ldo + tl.n0 + c, gf);
         store_row_bf16x32(p.out2 + grow * p.ldo + tl.n0 + c, uf);
@@ -819,31 +819,40 @@ bool umma_shape_supported(int H, int F) { return H % 128 == 0 && F % 128 == 0 &&
 // workloads): CTA pairs wherever a 256 x 256 tile fits, except the dgrad to x,
 // whose 256-row single-CTA tiles were faster.
 
+// [G | U] = x_perm * [W1_e | W3_e] per group; act = silu(G) * U.  act, G and U
+// may each be NULL (the backward's recompute asks for G and U only).
+moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const int32_t* pb, int E, int H,
+                      int F, int64_t P, void* act, void* G, void* U, int* status, cudaStream_t s,
+                      const char* name) {
+  typedef __nv_bfloat16 bf;
+  Params p = blank_params(pb, E, P, status);
+  if (!map2d(&p.ta0, x_perm, H, P, H, 64, 128) || !map3d(&p.tb0, W1, F, H, E, 64, 64) ||
+      !map3d(&p.tb1, W3, F, H, E, 64, 64))
+    return MOE_ERR_CUDA;
+  p.kdim = H;
+  p.n_mma = 256;
+  p.n_tiles = F / 128;
+  p.out0 = (bf*)act;
+  p.out1 = (bf*)G;
+  p.out2 = (bf*)U;
+  p.ldo = F;
+  const int64_t up = (P / BM) * p.n_tiles;
+  return launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>(name, p, up, s);
+}
+
 moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W3, const void* W2,
                                const int32_t* pb, int E, int H, int F, int64_t P, void* act, void* out,
                                void* gate_up, int* status, cudaStream_t s) {
   typedef __nv_bfloat16 bf;
   const bool pair = true;
   // GEMM1 + SwiGLU: [G | U] = x_perm * [W1_e | W3_e], act = silu(G) * U
-  {
-    Params p = blank_params(pb, E, P, status);
-    if (!map2d(&p.ta0, x_perm, H, P, H, 64, 128) || !map3d(&p.tb0, W1, F, H, E, 64, 64) ||
-        !map3d(&p.tb1, W3, F, H, E, 64, 64))
-      return MOE_ERR_CUDA;
-    p.kdim = H;
-    p.n_mma = 256;
-    p.n_tiles = F / 128;
-    p.out0 = (bf*)act;
-    p.out1 = gate_up ? (bf*)gate_up : nullptr;
-    p.out2 = gate_up ? (bf*)gate_up + (size_t)P * F : nullptr;
-    p.ldo = F;
-    const int64_t up = (P / BM) * p.n_tiles;
-    moe_status st = pair ? launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p, up, s)
-                         : launch<256, 1, 1, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu", p, up, s);
-    if (st != MOE_OK) return st;
-  }
+  moe_status st = gemm1_umma(x_perm, W1, W3, pb, E, H, F, P, act,
+                             gate_up ? (bf*)gate_up : nullptr,
+                             gate_up ? (bf*)gate_up + (size_t)P * F : nullptr, status, s, "gemm1_swiglu");
+  if (st != MOE_OK) return st;
   // GEMM2: out = act * W2_e
   {
+    (void)pair;
     Params p = blank_params(pb, E, P, status);
     const int bn = (H % 256 == 0) ? 256 : 128;
     if (!map2d(&p.ta0, act, F, P, F, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, 64)) return MOE_ERR_CUDA;

@@ -60,7 +60,13 @@ moe_status grouped_swiglu_bwd_simt(const void* d_out, const void* x_perm, const 
                                    moe_dtype dt, void* d_gate_up, void* dW1, void* dW3, void* dW2,
                                    void* dx_perm, cudaStream_t s);
 
+moe_status gate_up_simt(const void* x_perm, const void* W1, const void* W3, const int32_t* pb, int E, int H,
+                        int F, int64_t P, void* G, void* U, cudaStream_t s);
+
 // gemm_umma.cu - bf16 tcgen05 grouped GEMMs
+moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const int32_t* pb, int E, int H,
+                      int F, int64_t P, void* act, void* G, void* U, int* status, cudaStream_t s,
+                      const char* name);
 bool umma_shape_supported(int H, int F);
 moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W3, const void* W2,
                                const int32_t* pb, int E, int H, int F, int64_t P, void* act,

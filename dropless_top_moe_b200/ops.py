@@ -201,12 +201,14 @@ class MoELayer:
     def __init__(self, N: int, H: int, E: int, K: int, F: int, dtype=torch.bfloat16,
                  training: bool = False, device="cuda", aux_alpha: float = 0.0, capacity: int = 0):
         self.N, self.H, self.E, self.K, self.F = N, H, E, K, F
-        self.dtype, self.training = dtype, training
+        self.dtype, self.training = dtype, bool(training)
+        # training: False/0 forward only; True/1 keep G, U; 2 recompute them in backward
+        self.mode = 0 if not training else (2 if training == 2 else 1)
         self.aux_alpha = float(aux_alpha)
         self.capacity = int(capacity)   # 0 = dropless
         self.device = torch.device(device)
         self.dt = _DT[dtype]
-        nbytes = load().moe_workspace_size(N, H, E, K, F, self.dt, int(training))
+        nbytes = load().moe_workspace_size(N, H, E, K, F, self.dt, self.mode)
         if nbytes == 0:
             raise _lib.MoEError("moe_workspace_size", _lib.MOE_ERR_UNSUPPORTED)
         self.ws = workspace(nbytes, self.device)
@@ -223,7 +225,7 @@ class MoELayer:
     def forward(self, x, W_r, W1, W3, W2, y=None):
         y = self.y if y is None else y
         call("moe_layer_fwd", _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), self.N, self.H, self.E, self.K,
-             self.F, self.dt, int(self.training), self.capacity, self.aux_alpha, _p(self.aux_loss), _p(y),
+             self.F, self.dt, self.mode, self.capacity, self.aux_alpha, _p(self.aux_loss), _p(y),
              _p(self.top_experts), _p(self.weights),
              _p(self.indices), _p(self.bins), _p(self.padded_bins), self.ws.data_ptr(),
              self.ws.numel(), _stream())
@@ -247,7 +249,8 @@ class MoELayer:
         g = self.grad_buffers() if grads is None else grads
         call("moe_layer_bwd", _p(dy), _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), _p(self.top_experts),
              _p(self.weights), _p(self.indices), _p(self.bins), _p(self.padded_bins), self.N, self.H,
-             self.E, self.K, self.F, self.dt, self.capacity, self.aux_alpha, float(aux_grad), _p(g["dx"]),
+             self.E, self.K, self.F, self.dt, self.mode, self.capacity, self.aux_alpha, float(aux_grad),
+             _p(g["dx"]),
              _p(g["dW_r"]),
              _p(g["dW1"]), _p(g["dW3"]),
              _p(g["dW2"]), self.ws.data_ptr(), self.ws.numel(), _stream())

@@ -87,8 +87,11 @@ int64_t moe_padded_rows_max(int32_t N, int32_t E, int32_t K);
 size_t moe_route_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, moe_dtype dt);
 size_t moe_dispatch_meta_workspace_size(int32_t N, int32_t K, int32_t E);
 size_t moe_grouped_workspace_size(void);
-/* Whole layer.  training != 0 adds the activations the backward pass reads
- * (the same workspace must then be passed to moe_layer_bwd unchanged). */
+/* Whole layer.  training: 0 = forward only; 1 = keep what the backward pass
+ * reads, including the SwiGLU gate and up projections G, U; 2 = memory-
+ * optimised training: G and U are not kept (2*P*F elements less) and the
+ * backward recomputes them (+4*N*K*H*F FLOPs).  The same workspace must then
+ * be passed to moe_layer_bwd unchanged. */
 size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F,
                           moe_dtype dt, int32_t training);
 
@@ -266,7 +269,8 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
                          int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Whole layer backward for the forward run last with this workspace
- * (training != 0).  dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F],
+ * (training 1 or 2, the forward's value; with 2 the gate and up projections
+ * G, U are recomputed here by the forward's own GEMM kernel, bit-identical).  dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F],
  * dW2 [E,F,H], all dt, overwritten.  capacity and aux_alpha must equal the
  * forward's (dropped pairs still pass gradient to the router through the
  * renormalised weights);
@@ -276,8 +280,8 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                          const void* W3, const void* W2, const int32_t* top_experts,
                          const float* weights, const int32_t* indices, const int32_t* bins,
                          const int32_t* padded_bins, int32_t N, int32_t H, int32_t E, int32_t K,
-                         int32_t F, moe_dtype dt, int32_t capacity, float aux_alpha, float aux_grad,
-                         void* dx,
+                         int32_t F, moe_dtype dt, int32_t training, int32_t capacity, float aux_alpha,
+                         float aux_grad, void* dx,
                          void* dW_r, void* dW1, void* dW3, void* dW2, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 

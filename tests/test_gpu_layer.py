@@ -217,3 +217,26 @@ def test_dispatch_meta_capacity_bit_exact():
             np.testing.assert_array_equal(m[k].cpu().numpy(), ref[k], err_msg=f"{k} cap={cap}")
         for k in ("indices", "bin_ids"):
             np.testing.assert_array_equal(m[k].cpu().numpy()[:n], ref[k], err_msg=f"{k} cap={cap}")
+
+
+@pytest.mark.parametrize("shape", [small_shape("memopt_bf16", N=800, H=256, E=16, K=4, F=384, training=True),
+                                   small_shape("memopt_f32", N=200, H=64, E=4, K=2, F=96, dtype="f32",
+                                               training=True)], ids=lambda s: s.name)
+def test_memory_optimised_backward_is_bit_identical(shape):
+    """training=2 keeps no gate/up projections and recomputes them in the
+    backward with the forward's own kernel: same bits as training=1, less
+    workspace."""
+    c = make_case(shape, seed=13, with_dy=True)
+    outs = {}
+    for mode in (1, 2):
+        layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                             training=mode)
+        y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"]).clone()
+        g = {k: v.clone() for k, v in layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"]).items()}
+        torch.cuda.synchronize()
+        assert layer.status() == 0
+        outs[mode] = (y, g, layer.ws.numel())
+    assert outs[2][2] < outs[1][2]
+    assert torch.equal(outs[1][0], outs[2][0])
+    for k in outs[1][1]:
+        assert torch.equal(outs[1][1][k], outs[2][1][k]), k
