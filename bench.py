@@ -45,6 +45,11 @@ def parse_args():
     ap.add_argument("--workload", default="train_step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--train-mode", type=int, default=1, choices=[1, 2],
+                    help="1: keep the SwiGLU gates for the backward; 2: recompute them (less memory)")
+    ap.add_argument("--aux-alpha", type=float, default=0.0, help="load-balancing loss weight (0 = off)")
+    ap.add_argument("--capacity-factor", type=float, default=0.0,
+                    help="token-dropping variant: per-expert capacity ceil(N/E*cf) (0 = dropless)")
     ap.add_argument("--tokens", type=int, default=0, help="override N (small profiling cases)")
     ap.add_argument("--experts", type=int, default=0, help="override E (small profiling cases)")
     return ap.parse_args()
@@ -198,8 +203,13 @@ def run_ours(args, rank, world, local_rank):
         inp["x"] = token_rows(shape, shape.N, _gen(1000 + rank, dev), dev)
         if shape.training:
             inp["dy"] = torch.randn(shape.N, shape.H, generator=_gen(2000 + rank, dev), device=dev).to(shape.torch_dtype)
+    import math
+    # capacity per expert = ceil(N*K/E * cf): cf = 1 is the balanced load
+    capacity = (int(math.ceil(shape.N * shape.K / shape.E * args.capacity_factor))
+                if args.capacity_factor > 0 else 0)
+    train_mode = args.train_mode if shape.training else 0
     layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
-                         training=shape.training, device=dev)
+                         training=train_mode, device=dev, aux_alpha=args.aux_alpha, capacity=capacity)
     grads = layer.grad_buffers() if shape.training else None
 
     def step():
@@ -270,7 +280,12 @@ def run_ours(args, rank, world, local_rank):
         tot, n = per.get(name, (0.0, 0))
         per[name] = (tot + d, n + 1)
     padded_rows = int(layer.padded_bins[-1].item())
-    fl = flops_by_kernel(shape)
+    # algorithmic work counts the assignments actually computed (all N*K when
+    # dropless; the kept ones in the token-dropping variant)
+    kept = int(layer.bins[-1].item())
+    work = shape.with_(K=1, N=kept) if capacity else shape
+    fl = flops_by_kernel(work)
+    fl["route_umma"] = 2 * shape.N * shape.H * shape.E
     by = bytes_by_kernel(shape, padded_rows)
     peaks, peak_src = load_peaks()
     kernels = {}
@@ -306,9 +321,13 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"{shape.name}: N={shape.N} H={shape.H} E={shape.E} top_k={shape.K} "
                                f"F={shape.F} SwiGLU, {'forward+backward' if shape.training else 'forward'}",
                    "tokens_per_step_per_gpu": shape.N, "parallelism": f"replicas x{world}",
+                   "variant": {"train_mode": train_mode, "aux_alpha": args.aux_alpha,
+                               "capacity": capacity or "dropless"},
                    "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
                          (3 * shape.E * shape.H * shape.F * 2 / 1e9)},
-        "tflops": round(layer_flops(shape) / (ms_max * 1e-3) / 1e12, 1),
+        "tflops": round((layer_flops(work) - (2 * work.N * work.H * work.E) * (3 if shape.training else 1)
+                         + (2 * shape.N * shape.H * shape.E) * (3 if shape.training else 1))
+                        / (ms_max * 1e-3) / 1e12, 1),
         "roofline": roof, "kernels": kernels, "gpu_launches": count.value,
         "launches_per_step": per_step, "device_status": status, "clocks": clk,
     }

@@ -138,11 +138,12 @@ def round_up(n, m: int = TILE):
     return ((np.asarray(n, dtype=np.int64) + m - 1) // m) * m
 
 
-def capacity_from_factor(N: int, E: int, capacity_factor: float) -> int:
-    """Per-expert capacity as the icman page states it (sec. 3.4):
-    ceil(N / E * capacity_factor), N the tokens of the batch."""
+def capacity_from_factor(N: int, E: int, capacity_factor: float, K: int = 1) -> int:
+    """Per-expert capacity ceil(N*K / E * capacity_factor) (icman sec. 3.4
+    writes ceil(N / E * cf) and says cf = 1 is the perfectly uniform case,
+    which holds for top-K routing only when N counts the N*K assignments)."""
     import math
-    return int(math.ceil(N / E * capacity_factor))
+    return int(math.ceil(N * K / E * capacity_factor))
 
 
 def kept_mask(top_experts, E: int, capacity: int) -> np.ndarray:

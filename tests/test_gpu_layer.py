@@ -181,7 +181,7 @@ CAP = [small_shape("cap_f32", N=256, H=64, E=8, K=2, F=96, dtype="f32", training
 
 @pytest.mark.parametrize("shape", CAP, ids=lambda s: s.name)
 def test_layer_token_dropping_variant(shape):
-    cap = om.capacity_from_factor(shape.N, shape.E, 1.0)      # icman sec. 3.4 with factor 1
+    cap = om.capacity_from_factor(shape.N, shape.E, 1.0, shape.K)   # icman sec. 3.4, factor 1
     c = make_case(shape, seed=12, with_dy=True)
     layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
                          training=True, capacity=cap)

@@ -316,6 +316,7 @@ def test_capacity_keeps_first_assignments_brute_force():
     np.testing.assert_array_equal(m["indices"], [0, 3, 1, 2, 5, 6])
     np.testing.assert_array_equal(m["pos"], [0, 128, 129, 1, -1, 256, 257, -1, -1, -1])
     assert om.capacity_from_factor(1000, 8, 1.25) == 157     # ceil(1000 / 8 * 1.25)
+    assert om.capacity_from_factor(1000, 8, 1.0, K=2) == 250  # balanced top-2 load per expert
 
 
 def test_capacity_layer_equals_masked_sum():
