@@ -59,7 +59,15 @@ size_t route_scratch_bytes(int H, int E, moe_dtype dt) {
   return dt == MOE_BF16 ? route_umma_scratch(H, E) : 0;
 }
 
-LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int training) {
+// training: mode 0 / 1 / 2 in the low bits, MOE_LAYER_GATHER_ROWS (bf16 only) on top
+bool layer_flags_ok(int32_t training, moe_dtype dt) {
+  if ((training & ~(3 | MOE_LAYER_GATHER_ROWS)) != 0 || (training & 3) == 3) return false;
+  return !(training & MOE_LAYER_GATHER_ROWS) || dt == MOE_BF16;
+}
+
+LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int flags) {
+  const int training = flags & 3;
+  const bool gather = (flags & MOE_LAYER_GATHER_ROWS) != 0;
   LayerWs w;
   memset(&w, 0, sizeof(w));
   char* p = (char*)base;
@@ -77,7 +85,7 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int t
   w.pos = (int32_t*)take(NK * 4);
   w.probs = (float*)take((size_t)N * E * 4);
   w.aux_scratch = take(aux_loss_scratch(N, E));
-  w.x_perm = take(P * H * eb);
+  w.x_perm = gather ? nullptr : take(P * H * eb);   // gathered rows need no permuted copy
   w.act = take(P * F * eb);
   w.out = take(P * H * eb);
   if (training) {
@@ -107,21 +115,22 @@ moe_status route_any(const void* x, const void* W_r, int N, int H, int E, int K,
 
 moe_status swiglu_any(const void* x_perm, const void* W1, const void* W3, const void* W2,
                       const int32_t* pb, int E, int H, int F, int64_t P, moe_dtype dt, void* act,
-                      void* out, void* gate_up, int* status, cudaStream_t s) {
+                      void* out, void* gate_up, int* status, cudaStream_t s, const RowGather* ga = nullptr) {
   if (dt == MOE_F32)
     return grouped_swiglu_simt(x_perm, W1, W3, W2, pb, E, H, F, P, dt, act, out, gate_up, s);
-  return grouped_swiglu_umma(x_perm, W1, W3, W2, pb, E, H, F, P, act, out, gate_up, status, s);
+  return grouped_swiglu_umma(x_perm, W1, W3, W2, pb, E, H, F, P, act, out, gate_up, status, s, ga);
 }
 
 moe_status swiglu_bwd_any(const void* d_out, const void* x_perm, const void* act, const void* gate_up,
                           const void* W1, const void* W3, const void* W2, const int32_t* pb, int E,
                           int H, int F, int64_t P, moe_dtype dt, void* d_gate_up, void* dW1,
-                          void* dW3, void* dW2, void* dx_perm, int* status, cudaStream_t s) {
+                          void* dW3, void* dW2, void* dx_perm, int* status, cudaStream_t s,
+                          const RowGather* ga = nullptr) {
   if (dt == MOE_F32)
     return grouped_swiglu_bwd_simt(d_out, x_perm, act, gate_up, W1, W3, W2, pb, E, H, F, P, dt,
                                    d_gate_up, dW1, dW3, dW2, dx_perm, s);
   return grouped_swiglu_bwd_umma(d_out, x_perm, act, gate_up, W1, W3, W2, pb, E, H, F, P, d_gate_up,
-                                 dW1, dW3, dW2, dx_perm, status, s);
+                                 dW1, dW3, dW2, dx_perm, status, s, ga);
 }
 
 }  // namespace
@@ -163,7 +172,7 @@ size_t moe_aux_loss_workspace_size(int32_t N, int32_t E) {
 
 size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
                           int32_t training) {
-  if (check_shape(N, H, E, K, dt) != MOE_OK || F <= 0) return 0;
+  if (check_shape(N, H, E, K, dt) != MOE_OK || F <= 0 || !layer_flags_ok(training, dt)) return 0;
   return carve(nullptr, N, H, E, K, F, dt, training).total;
 }
 
@@ -316,11 +325,14 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
   const void* ptrs[] = {x, W_r, W1, W3, W2, y, top_experts, weights, indices, bins, padded_bins};
   for (const void* q : ptrs)
     if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  if (!layer_flags_ok(training, dt)) return MOE_ERR_INVALID_ARG;
   const size_t need = moe_workspace_size(N, H, E, K, F, dt, training);
   if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
+  const bool gather = (training & MOE_LAYER_GATHER_ROWS) != 0;
+  training &= 3;
   const bool aux = aux_alpha != 0.0f;
   if ((aux && !aux_loss) || capacity < 0) return MOE_ERR_INVALID_ARG;
   MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, aux ? w.probs : nullptr, top_experts, weights,
@@ -329,9 +341,10 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
                         w.meta_scratch, w.status, s, capacity));
   if (aux) MOE_TRY(aux_loss_fwd(w.probs, bins, N, K, E, aux_alpha, aux_loss, nullptr, w.aux_scratch, s));
   if (N == 0) return MOE_OK;
-  MOE_TRY(permute_rows(x, w.pos, bins, padded_bins, N, H, E, K, dt, w.x_perm, s));
+  const RowGather ga = {x, indices, bins, N, K};
+  if (!gather) MOE_TRY(permute_rows(x, w.pos, bins, padded_bins, N, H, E, K, dt, w.x_perm, s));
   MOE_TRY(swiglu_any(w.x_perm, W1, W3, W2, padded_bins, E, H, F, P, dt, w.act, w.out,
-                     training == 1 ? w.gate_up : nullptr, w.status, s));
+                     training == 1 ? w.gate_up : nullptr, w.status, s, gather ? &ga : nullptr));
   MOE_TRY(combine_rows(w.out, weights, w.pos, N, K, H, dt, y, s));
   return MOE_OK;
 }
@@ -349,12 +362,15 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                         dx, dW_r, dW1, dW3, dW2};
   for (const void* q : ptrs)
     if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
-  if (training != 1 && training != 2) return MOE_ERR_INVALID_ARG;
+  if (!layer_flags_ok(training, dt) || ((training & 3) != 1 && (training & 3) != 2)) return MOE_ERR_INVALID_ARG;
   const size_t need = moe_workspace_size(N, H, E, K, F, dt, training);
   if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
+  const RowGather ga = {x, indices, bins, N, K};
+  const bool gather = (training & MOE_LAYER_GATHER_ROWS) != 0;
+  training &= 3;
   void* gate_up = w.gate_up;
   if (training == 2) {
     // recompute G, U (same kernel and inputs as the forward: identical bits)
@@ -367,12 +383,12 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
       MOE_TRY(gate_up_simt(w.x_perm, W1, W3, padded_bins, E, H, F, P, G, U, s));
     else
       MOE_TRY(gemm1_umma(w.x_perm, W1, W3, padded_bins, E, H, F, P, nullptr, G, U, w.status, s,
-                         "gate_up_recompute"));
+                         "gate_up_recompute", gather ? &ga : nullptr));
   }
   MOE_TRY(combine_bwd_rows(dy, w.out, weights, w.pos, bins, padded_bins, N, K, H, E, dt, nullptr,
                            w.dlogit, w.d_out, s));
   MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
-                         w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s));
+                         w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s, gather ? &ga : nullptr));
   // the sparse router backward walks the kept assignments only; the aux loss
   // and dropped assignments need every (token, expert) logit: dense path
   if ((aux_alpha != 0.0f || capacity > 0) && N > 0)

@@ -59,6 +59,14 @@ struct Params {
   int n_mma;          // MMA N (== BN except DENSE, where it is E)
   int n_tiles;        // tiles along N
   int m_tiles_w;      // WGRAD: tiles along M
+  int group_m;        // ROWS: M units per raster group
+  // Gathered A (GA kernels): ta0 maps the token matrix [g_N, kdim or M] with
+  // one-row boxes; padded row r of expert e holds token
+  // g_indices[g_bins[e-1] + r - padded_bins[e-1]] / g_K, pad rows read zeros
+  const int32_t* g_indices;
+  const int32_t* g_bins;
+  int g_K;
+  int g_N;
   __nv_bfloat16* out0;
   __nv_bfloat16* out1;
   __nv_bfloat16* out2;
@@ -99,8 +107,8 @@ struct Shape {
       USED_COLS <= 32 ? 32 : (USED_COLS <= 64 ? 64 : (USED_COLS <= 128 ? 128 : (USED_COLS <= 256 ? 256 : 512)));
   static constexpr int N_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + 8 * N_BARS + 16 + 4 * 260;
-  // 128-row halves per scheduling unit (a CTA's two halves, or a pair's)
-  static constexpr int UNIT = (MT == 2 || CG == 2) ? 2 : 1;
+  // 128-row tiles per scheduling unit: MT per CTA, times 2 for a pair
+  static constexpr int UNIT = MT * CG;
 };
 
 // Rows of the grouped buffers actually used, clamped to the buffers' rows.
@@ -109,9 +117,9 @@ __device__ __forceinline__ int64_t used_rows(const Params& p) {
   return rows > p.P ? p.P : rows;
 }
 
-// Number of M units for the ROWS schedule: 128-row tiles (MT = 1) or pairs
-// of 128-row tiles of the same expert (MT = 2; an odd last tile of an expert
-// forms a unit of one half).  s_unit_start[e] = first unit of expert e.
+// Number of M units for the ROWS schedule: 128-row tiles (UNIT = 1) or
+// groups of UNIT consecutive 128-row tiles of the same expert (the last unit
+// of an expert may hold fewer).  s_unit_start[e] = first unit of expert e.
 template <int UNIT>
 __device__ __forceinline__ int64_t rows_units(const Params& p, const int32_t* s_unit_start) {
   if constexpr (UNIT == 1) return used_rows(p) / BM;
@@ -135,10 +143,10 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32
   Tile tl;
   if constexpr (SCHED == SCHED_ROWS) {
     const int64_t num_m = rows_units<UNIT>(p, s_unit_start);
-    const int64_t per_group = (int64_t)kGroupM * p.n_tiles;
+    const int64_t per_group = (int64_t)p.group_m * p.n_tiles;
     const int64_t g = t / per_group;
-    const int64_t first_m = g * kGroupM;
-    const int64_t gm = (num_m - first_m) < kGroupM ? (num_m - first_m) : kGroupM;
+    const int64_t first_m = g * p.group_m;
+    const int64_t gm = (num_m - first_m) < p.group_m ? (num_m - first_m) : p.group_m;
     const int64_t local = t - g * per_group;
     const int64_t mu = first_m + local % gm;          // M unit
     const int64_t nt = local / gm;
@@ -157,8 +165,8 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32
       const int64_t pstart = tl.e ? p.padded_bins[tl.e - 1] : 0;
       const int64_t ntile_e = (p.padded_bins[tl.e] - pstart) / BM;
       const int64_t k = mu - s_unit_start[tl.e];
-      tl.row0 = pstart + k * 2 * BM;
-      tl.halves = (ntile_e - 2 * k) >= 2 ? 2 : 1;
+      tl.row0 = pstart + k * UNIT * BM;
+      tl.halves = (int)((ntile_e - UNIT * k) >= UNIT ? UNIT : (ntile_e - UNIT * k));
     }
     tl.m0 = 0;
     tl.n0 = (int)(nt * NOUT);
@@ -371,7 +379,60 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
   }
 }
 
-template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
+// B tile of one k block into sb; k is the k offset (ROWS / DENSE) or the
+// group row (WGRAD); tb is the map to read (SPLIT_K picks it per k block).
+// In a pair each CTA fetches its half of B's columns (SPLIT_N: W1 | W3).
+template <int BN, int CG, int SCHED, bool B_MN, int SPLIT>
+__device__ __forceinline__ void load_b(const Params& p, const Tile& tl, uint32_t sb, uint32_t fb,
+                                       uint32_t rank, int k, const CUtensorMap* tb) {
+  if constexpr (CG == 2) {
+    if constexpr (SCHED == SCHED_WGRAD) {
+#pragma unroll
+      for (int j = 0; j < BN / 128; ++j) {
+        if (SPLIT == SPLIT_N)
+          tma_load_2d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k);
+        else
+          tma_load_2d_pair(sb + j * 8192, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k);
+      }
+    } else if constexpr (B_MN) {
+#pragma unroll
+      for (int j = 0; j < BN / 128; ++j) {
+        if (SPLIT == SPLIT_N)
+          tma_load_3d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k, tl.e);
+        else
+          tma_load_3d_pair(sb + j * 8192, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k, tl.e);
+      }
+    } else {
+      tma_load_3d_pair(sb, tb, fb, k, tl.n0 + (BN / 2) * (int)rank, tl.e);
+    }
+  } else {
+    if constexpr (SCHED == SCHED_WGRAD) {
+#pragma unroll
+      for (int j = 0; j < BN / 64; ++j) {
+        if (SPLIT == SPLIT_N && j >= BN / 128)
+          tma_load_2d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), k);
+        else
+          tma_load_2d(sb + j * 8192, tb, fb, tl.n0 + 64 * j, k);
+      }
+    } else if constexpr (SCHED == SCHED_DENSE && B_MN) {
+      for (int j = 0; j < p.n_mma / 64; ++j) tma_load_2d(sb + j * 8192, tb, fb, 64 * j, k);
+    } else if constexpr (SCHED == SCHED_DENSE) {
+      tma_load_2d(sb, tb, fb, k, 0);
+    } else if constexpr (B_MN) {
+#pragma unroll
+      for (int j = 0; j < BN / 64; ++j) {
+        if (SPLIT == SPLIT_N && j >= BN / 128)
+          tma_load_3d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), k, tl.e);
+        else
+          tma_load_3d(sb + j * 8192, tb, fb, tl.n0 + 64 * j, k, tl.e);
+      }
+    } else {
+      tma_load_3d(sb, tb, fb, k, tl.n0, tl.e);
+    }
+  }
+}
+
+template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT, bool GA>
 __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
   using S = Shape<BN, MT, CG>;
   constexpr int STAGES = S::STAGES;
@@ -385,7 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte swizzle atoms aligned");
   static_assert(STAGES >= 2, "pipeline needs at least two stages");
   static_assert(MT == 1 || SCHED != SCHED_DENSE, "the router uses single 128-row tiles");
-  static_assert(!PAIR || (MT == 1 && SCHED != SCHED_DENSE), "a pair holds one half per CTA");
+  static_assert(!PAIR || SCHED != SCHED_DENSE, "the router uses single CTAs");
+  static_assert(!GA || (SCHED == SCHED_ROWS && !A_MN && SPLIT != SPLIT_K) || (SCHED == SCHED_WGRAD && A_MN),
+                "row gathers feed K-major A of ROWS or MN-major A of WGRAD");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -416,8 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     fence_barrier_init();
     fence_proxy_async();
   }
-  if (SCHED == SCHED_ROWS && UNIT == 2 && warp == 2) {
-    // units per expert = ceil(tiles_e / 2); exclusive scan over experts
+  if (SCHED == SCHED_ROWS && UNIT > 1 && warp == 2) {
+    // units per expert = ceil(tiles_e / UNIT); exclusive scan over experts
     int carry = 0;
     for (int e0 = 0; e0 < p.E; e0 += 32) {
       const int e = e0 + lane;
@@ -427,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
         int64_t hi = p.padded_bins[e];
         if (hi > p.P) hi = p.P;
         const int64_t tiles = hi > lo ? (hi - lo) / BM : 0;
-        u = (int)((tiles + 1) / 2);
+        u = (int)((tiles + UNIT - 1) / UNIT);
       }
       int incl = u;
 #pragma unroll
@@ -463,14 +526,98 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if constexpr (GA) {
+      // A rows gathered from the token matrix: each lane gathers four rows
+      // (ROWS: rows 4*lane.. of each 128-row half; WGRAD: k rows 4*(lane%16)..
+      // of column box lane/16); lane 0 arms the barrier and loads B
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      const int g = lane & 15, jb = lane >> 4;
+      for (int64_t t = tile0; t < ntiles && ok; t += tstep) {
+        const Tile tl = get_tile<SCHED, BN, UNIT, EPI>(p, t, s_unit_start);
+        const int64_t pstart = tl.e ? p.padded_bins[tl.e - 1] : 0;
+        const int32_t bstart = tl.e ? p.g_bins[tl.e - 1] : 0;
+        const int64_t cnt = (int64_t)p.g_bins[tl.e] - bstart;
+        auto tok_of = [&](int64_t r) -> int {
+          const int64_t j = r - pstart;
+          return j < cnt ? p.g_indices[bstart + j] / p.g_K : p.g_N;
+        };
+        const int n_mma_h = PAIR ? (tl.halves + 1) / 2 : tl.halves;
+        uint32_t tx;
+        if constexpr (PAIR) tx = 2u * (uint32_t)(n_mma_h * BM * BK * 2 + B_BYTES);
+        else tx = (uint32_t)tl.halves * BM * BK * 2 + (uint32_t)B_BYTES;
+        int tk[MT][4];      // ROWS: this lane's four tokens of each half
+        int nx[4];          // WGRAD: this lane's four tokens of the next k block
+        if constexpr (SCHED == SCHED_ROWS) {
+#pragma unroll
+          for (int h = 0; h < MT; ++h) {
+            const int hh = PAIR ? 2 * h + (int)rank : h;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              tk[h][i] = h < n_mma_h ? tok_of(tl.row0 + hh * BM + 4 * lane + i) : p.g_N;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) nx[i] = tl.nkb > 0 ? tok_of(tl.row0 + 4 * g + i) : p.g_N;
+        }
+        for (int kb = 0; kb < tl.nkb; ++kb) {
+          int w_ok = 1;
+          if (lane == 0)
+            w_ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kTimeoutNs) ? 1 : 0;
+          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+          if (!w_ok) { ok = false; break; }
+          const uint32_t sa = base + stage * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+          const uint32_t fb = PAIR ? map_to_rank(full_bar(stage), 0) : full_bar(stage);
+          const int kc = SCHED == SCHED_WGRAD ? (int)(tl.row0 + (int64_t)kb * BK) : kb * BK;
+          if (lane == 0) {
+            if (!PAIR || rank == 0) mbar_expect_tx(full_bar(stage), tx);
+            load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, kc, &p.tb0);
+          }
+          if constexpr (SCHED == SCHED_WGRAD) {
+            int cur[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cur[i] = nx[i];
+            for (int h = 0; h < n_mma_h; ++h) {
+              const int hh = PAIR ? 2 * h + (int)rank : h;
+              const uint32_t dst = sa + h * (BM * BK * 2) + jb * 8192 + g * 512;
+              const int m = tl.m0 + BM * hh + 64 * jb;
+              if constexpr (PAIR) tma_gather4_pair(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
+              else tma_gather4(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
+            }
+            if (kb + 1 < tl.nkb) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) nx[i] = tok_of((int64_t)kc + BK + 4 * g + i);
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < MT; ++h) {
+              if (h < n_mma_h) {
+                const uint32_t dst = sa + h * (BM * BK * 2) + lane * 512;
+                if constexpr (PAIR) tma_gather4_pair(dst, &p.ta0, fb, kc, tk[h][0], tk[h][1], tk[h][2], tk[h][3]);
+                else tma_gather4(dst, &p.ta0, fb, kc, tk[h][0], tk[h][1], tk[h][2], tk[h][3]);
+              }
+            }
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 20000000ull) {}
+      }
+    } else if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int64_t t = tile0; t < ntiles && ok; t += tstep) {
         const Tile tl = get_tile<SCHED, BN, UNIT, EPI>(p, t, s_unit_start);
+        // MMAs of this tile: with a pair, MMA h covers tiles 2h and 2h+1 of the
+        // unit (one per CTA) and runs when tile 2h exists
+        const int n_mma_h = PAIR ? (tl.halves + 1) / 2 : tl.halves;
         uint32_t tx;
-        if constexpr (PAIR) tx = 2u * (uint32_t)(A_BYTES + B_BYTES);    // both CTAs' loads
+        if constexpr (PAIR) tx = 2u * (uint32_t)(n_mma_h * BM * BK * 2 + B_BYTES);   // both CTAs' loads
         else tx = (uint32_t)tl.halves * BM * BK * 2 +
                   (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)B_BYTES);
         for (int kb = 0; kb < tl.nkb; ++kb) {
@@ -482,33 +629,20 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
             if (rank == 0) mbar_expect_tx(full_bar(stage), tx);
             if constexpr (SCHED == SCHED_WGRAD) {
               const int krow = (int)(tl.row0 + (int64_t)kb * BK);
-              const int m = tl.m0 + BM * (int)rank;
-              tma_load_2d_pair(sa, &p.ta0, fb, m, krow);
-              tma_load_2d_pair(sa + 8192, &p.ta0, fb, m + 64, krow);
-#pragma unroll
-              for (int j = 0; j < BN / 128; ++j) {
-                if (SPLIT == SPLIT_N)
-                  tma_load_2d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, krow);
-                else
-                  tma_load_2d_pair(sb + j * 8192, &p.tb0, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, krow);
+              for (int h = 0; h < n_mma_h; ++h) {
+                const int m = tl.m0 + BM * (2 * h + (int)rank);
+                tma_load_2d_pair(sa + h * (BM * BK * 2), &p.ta0, fb, m, krow);
+                tma_load_2d_pair(sa + h * (BM * BK * 2) + 8192, &p.ta0, fb, m + 64, krow);
               }
+              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, krow, &p.tb0);
             } else {
               int k = kb * BK;
               const CUtensorMap* ta = &p.ta0;
               const CUtensorMap* tb = &p.tb0;
               if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
-              tma_load_2d_pair(sa, ta, fb, k, (int)tl.row0 + BM * (int)rank);
-              if constexpr (B_MN) {
-#pragma unroll
-                for (int j = 0; j < BN / 128; ++j) {
-                  if (SPLIT == SPLIT_N)
-                    tma_load_3d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k, tl.e);
-                  else
-                    tma_load_3d_pair(sb + j * 8192, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k, tl.e);
-                }
-              } else {
-                tma_load_3d_pair(sb, tb, fb, k, tl.n0 + (BN / 2) * (int)rank, tl.e);
-              }
+              for (int h = 0; h < n_mma_h; ++h)
+                tma_load_2d_pair(sa + h * (BM * BK * 2), ta, fb, k, (int)tl.row0 + BM * (2 * h + (int)rank));
+              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, k, tb);
             }
           } else {
             const uint32_t fb = full_bar(stage);
@@ -518,13 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
               // A = X^T: 64-wide MN boxes of the [rows, M] matrix, 2 per half
 #pragma unroll
               for (int j = 0; j < 2 * MT; ++j) tma_load_2d(sa + j * 8192, &p.ta0, fb, tl.m0 + 64 * j, krow);
-#pragma unroll
-              for (int j = 0; j < BN / 64; ++j) {
-                if (SPLIT == SPLIT_N && j >= BN / 128)
-                  tma_load_2d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), krow);
-                else
-                  tma_load_2d(sb + j * 8192, &p.tb0, fb, tl.n0 + 64 * j, krow);
-              }
+              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, 0u, krow, &p.tb0);
             } else {
               int k = kb * BK;
               const CUtensorMap* ta = &p.ta0;
@@ -532,21 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
               if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
               tma_load_2d(sa, ta, fb, k, (int)tl.row0);
               if (MT == 2 && tl.halves == 2) tma_load_2d(sa + BM * BK * 2, ta, fb, k, (int)tl.row0 + BM);
-              if constexpr (SCHED == SCHED_DENSE && B_MN) {
-                for (int j = 0; j < p.n_mma / 64; ++j) tma_load_2d(sb + j * 8192, tb, fb, 64 * j, k);
-              } else if constexpr (SCHED == SCHED_DENSE) {
-                tma_load_2d(sb, tb, fb, k, 0);
-              } else if constexpr (B_MN) {
-#pragma unroll
-                for (int j = 0; j < BN / 64; ++j) {
-                  if (SPLIT == SPLIT_N && j >= BN / 128)
-                    tma_load_3d(sb + j * 8192, &p.tb1, fb, tl.n0 + 64 * (j - BN / 128), k, tl.e);
-                  else
-                    tma_load_3d(sb + j * 8192, tb, fb, tl.n0 + 64 * j, k, tl.e);
-                }
-              } else {
-                tma_load_3d(sb, tb, fb, k, tl.n0, tl.e);
-              }
+              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, 0u, k, tb);
             }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -584,8 +698,14 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
             const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             if constexpr (PAIR) {
-              const uint64_t ad = A_MN ? desc_mn_sw128(sa + kk * 2048, 8192) : desc_k_sw128(sa + kk * 32);
-              mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+#pragma unroll
+              for (int h = 0; h < MT; ++h) {
+                if (2 * h < tl.halves) {
+                  const uint32_t ah = sa + h * (BM * BK * 2);
+                  const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
+                  mma_bf16_pair(d_tmem + h * BN, ad, bd, idesc, accum);
+                }
+              }
             } else {
 #pragma unroll
               for (int h = 0; h < MT; ++h) {
@@ -627,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           const float z[32] = {0.f};
 #pragma unroll 1
           for (int h = 0; h < MT; ++h) {
-            const int hh = PAIR ? (int)rank : h;
+            const int hh = PAIR ? 2 * h + (int)rank : h;
             const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + hh * BM + row) * p.ldo + tl.n0;
             if constexpr (EPI == EPI_WGRAD_PAIR) {
 #pragma unroll 1
@@ -649,12 +769,15 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       if (!ok) break;
       tc_fence_after();
       if constexpr (PAIR) {
-        // this CTA's 128 rows of the 256-row tile; a lone last tile of an
-        // expert has no second half, so the peer stores nothing
-        if ((int)rank < tl.halves) {
-          const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+        // this CTA's tiles 2h + rank of the unit; tiles past the expert's end
+        // (a short last unit) are computed on garbage rows and not stored
+#pragma unroll 1
+        for (int h = 0; h < MT; ++h) {
+          const int j = 2 * h + (int)rank;
+          if (j >= tl.halves) continue;
+          const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
           Tile th = tl;
-          if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + (int)rank * BM; else th.row0 = tl.row0 + (int)rank * BM;
+          if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + j * BM; else th.row0 = tl.row0 + j * BM;
           epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part);
         }
       } else {
@@ -710,6 +833,7 @@ static bool map2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t oute
                   uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
+
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_elems * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
@@ -746,10 +870,12 @@ static int sm_count() {
   return cache[dev];
 }
 
-template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT>
-static moe_status launch(const char* name, const Params& p, int64_t tiles_upper, cudaStream_t s) {
+template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT, bool GA = false>
+static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upper, cudaStream_t s) {
   using S = Shape<BN, MT, CG>;
-  auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT>;
+  Params p = p_in;
+  if (p.group_m <= 0) p.group_m = S::UNIT >= 4 ? (kGroupM * 2) / S::UNIT : kGroupM;
+  auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -799,6 +925,13 @@ static moe_status launch(const char* name, const Params& p, int64_t tiles_upper,
   return MOE_OK;
 }
 
+static void set_gather(Params* p, const RowGather* ga) {
+  p->g_indices = ga->indices;
+  p->g_bins = ga->bins;
+  p->g_K = ga->K;
+  p->g_N = ga->N;
+}
+
 static Params blank_params(const int32_t* pb, int E, int64_t P, int* status) {
   Params p;
   memset(&p, 0, sizeof(p));
@@ -823,12 +956,13 @@ bool umma_shape_supported(int H, int F) { return H % 128 == 0 && F % 128 == 0 &&
 // may each be NULL (the backward's recompute asks for G and U only).
 moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const int32_t* pb, int E, int H,
                       int F, int64_t P, void* act, void* G, void* U, int* status, cudaStream_t s,
-                      const char* name) {
+                      const char* name, const RowGather* ga) {
   typedef __nv_bfloat16 bf;
   Params p = blank_params(pb, E, P, status);
-  if (!map2d(&p.ta0, x_perm, H, P, H, 64, 128) || !map3d(&p.tb0, W1, F, H, E, 64, 64) ||
-      !map3d(&p.tb1, W3, F, H, E, 64, 64))
+  const bool a_ok = ga ? map2d(&p.ta0, ga->x, H, ga->N, H, 64, 1) : map2d(&p.ta0, x_perm, H, P, H, 64, 128);
+  if (!a_ok || !map3d(&p.tb0, W1, F, H, E, 64, 64) || !map3d(&p.tb1, W3, F, H, E, 64, 64))
     return MOE_ERR_CUDA;
+  if (ga) set_gather(&p, ga);
   p.kdim = H;
   p.n_mma = 256;
   p.n_tiles = F / 128;
@@ -837,18 +971,19 @@ moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const 
   p.out2 = (bf*)U;
   p.ldo = F;
   const int64_t up = (P / BM) * p.n_tiles;
+  if (ga) return launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N, true>(name, p, up, s);
   return launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>(name, p, up, s);
 }
 
 moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W3, const void* W2,
                                const int32_t* pb, int E, int H, int F, int64_t P, void* act, void* out,
-                               void* gate_up, int* status, cudaStream_t s) {
+                               void* gate_up, int* status, cudaStream_t s, const RowGather* ga) {
   typedef __nv_bfloat16 bf;
   const bool pair = true;
   // GEMM1 + SwiGLU: [G | U] = x_perm * [W1_e | W3_e], act = silu(G) * U
   moe_status st = gemm1_umma(x_perm, W1, W3, pb, E, H, F, P, act,
                              gate_up ? (bf*)gate_up : nullptr,
-                             gate_up ? (bf*)gate_up + (size_t)P * F : nullptr, status, s, "gemm1_swiglu");
+                             gate_up ? (bf*)gate_up + (size_t)P * F : nullptr, status, s, "gemm1_swiglu", ga);
   if (st != MOE_OK) return st;
   // GEMM2: out = act * W2_e
   {
@@ -872,7 +1007,7 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
                                    const void* gate_up, const void* W1, const void* W3, const void* W2,
                                    const int32_t* pb, int E, int H, int F, int64_t P, void* d_gate_up,
                                    void* dW1, void* dW3, void* dW2, void* dx_perm, int* status,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, const RowGather* ga) {
   typedef __nv_bfloat16 bf;
   const bf* G = (const bf*)gate_up;
   const bf* U = G + (size_t)P * F;
@@ -924,9 +1059,10 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
   {
     Params p = blank_params(pb, E, P, status);
     const int unit = (H % 256 == 0) ? 2 : 1;
-    if (!map2d(&p.ta0, x_perm, H, P, H, 64, 64) || !map2d(&p.tb0, dG, F, P, F, 64, 64) ||
-        !map2d(&p.tb1, dU, F, P, F, 64, 64))
+    const bool a_ok = ga ? map2d(&p.ta0, ga->x, H, ga->N, H, 64, 1) : map2d(&p.ta0, x_perm, H, P, H, 64, 64);
+    if (!a_ok || !map2d(&p.tb0, dG, F, P, F, 64, 64) || !map2d(&p.tb1, dU, F, P, F, 64, 64))
       return MOE_ERR_CUDA;
+    if (ga) set_gather(&p, ga);
     p.n_mma = 256;
     p.m_tiles_w = H / (BM * unit);
     p.n_tiles = F / 128;
@@ -935,7 +1071,9 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.ldo = F;
     p.out_estride = (int64_t)H * F;
     const int64_t tiles = (int64_t)E * p.m_tiles_w * p.n_tiles;
-    if (unit == 2 && pref) st = launch<256, 1, 2, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
+    if (ga && unit == 2) st = launch<256, 1, 2, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N, true>("wgrad_w1_w3", p, tiles, s);
+    else if (ga) st = launch<256, 1, 1, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N, true>("wgrad_w1_w3", p, tiles, s);
+    else if (unit == 2 && pref) st = launch<256, 1, 2, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
     else if (unit == 2) st = launch<256, 2, 1, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
     else st = launch<256, 1, 1, SCHED_WGRAD, EPI_WGRAD_PAIR, true, true, SPLIT_N>("wgrad_w1_w3", p, tiles, s);
     if (st != MOE_OK) return st;

@@ -64,17 +64,30 @@ moe_status gate_up_simt(const void* x_perm, const void* W1, const void* W3, cons
                         int F, int64_t P, void* G, void* U, cudaStream_t s);
 
 // gemm_umma.cu - bf16 tcgen05 grouped GEMMs
+//
+// Row gather in place of x_perm: the GEMMs that read the permuted tokens
+// (GEMM1 and the dW1/dW3 weight gradient) can fetch padded row r of expert e
+// straight from x as token indices[bins[e-1] + r - padded_bins[e-1]] / K
+// (pad rows read zeros), so the permuted copy is never written.
+struct RowGather {
+  const void* x;            // [N, H] tokens
+  const int32_t* indices;   // sorted flat assignment ids (dispatch metadata)
+  const int32_t* bins;      // inclusive cumsum of per-expert (kept) counts
+  int N;
+  int K;
+};
 moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const int32_t* pb, int E, int H,
                       int F, int64_t P, void* act, void* G, void* U, int* status, cudaStream_t s,
-                      const char* name);
+                      const char* name, const RowGather* ga = nullptr);
 bool umma_shape_supported(int H, int F);
 moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W3, const void* W2,
                                const int32_t* pb, int E, int H, int F, int64_t P, void* act,
-                               void* out, void* gate_up, int* status, cudaStream_t s);
+                               void* out, void* gate_up, int* status, cudaStream_t s,
+                               const RowGather* ga = nullptr);
 moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const void* act,
                                    const void* gate_up, const void* W1, const void* W3,
                                    const void* W2, const int32_t* pb, int E, int H, int F, int64_t P,
                                    void* d_gate_up, void* dW1, void* dW3, void* dW2, void* dx_perm,
-                                   int* status, cudaStream_t s);
+                                   int* status, cudaStream_t s, const RowGather* ga = nullptr);
 
 }  // namespace moe

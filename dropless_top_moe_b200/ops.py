@@ -199,11 +199,14 @@ class MoELayer:
     """
 
     def __init__(self, N: int, H: int, E: int, K: int, F: int, dtype=torch.bfloat16,
-                 training: bool = False, device="cuda", aux_alpha: float = 0.0, capacity: int = 0):
+                 training: bool = False, device="cuda", aux_alpha: float = 0.0, capacity: int = 0,
+                 gather_rows: bool = False):
         self.N, self.H, self.E, self.K, self.F = N, H, E, K, F
         self.dtype, self.training = dtype, bool(training)
-        # training: False/0 forward only; True/1 keep G, U; 2 recompute them in backward
-        self.mode = 0 if not training else (2 if training == 2 else 1)
+        # training: False/0 forward only; True/1 keep G, U; 2 recompute them in backward.
+        # gather_rows (bf16): GEMM1 and dW1/dW3 read rows of x directly, no permuted copy
+        self.mode = (0 if not training else (2 if training == 2 else 1)) | \
+            (_lib.MOE_LAYER_GATHER_ROWS if gather_rows else 0)
         self.aux_alpha = float(aux_alpha)
         self.capacity = int(capacity)   # 0 = dropless
         self.device = torch.device(device)

@@ -95,6 +95,19 @@ size_t moe_grouped_workspace_size(void);
 size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F,
                           moe_dtype dt, int32_t training);
 
+/* Flag OR-ed into `training` (the same value for moe_workspace_size,
+ * moe_layer_fwd and moe_layer_bwd), bf16 only: GEMM1 and the dW1/dW3
+ * contraction fetch their rows straight from x with TMA row gathers
+ * (padded row r of expert e = token indices[bins[e-1] + r - padded_bins[e-1]]
+ * / K, pad rows zero) instead of a permuted copy, so the permute step and its
+ * P*H-element buffer disappear ("MegaBlocks - architecture", sec. 2.1: the
+ * permute only feeds the grouped GEMM).  Results are bit-identical to the
+ * default path.  The gathers move four 128-byte rows per TMA instruction, and
+ * on B200 their issue rate holds GEMM1 to roughly a third of its default
+ * speed, so this is a memory option, off by default.  With fp32 the
+ * workspace size is 0 and the layer calls return MOE_ERR_INVALID_ARG. */
+#define MOE_LAYER_GATHER_ROWS 4
+
 /* Zero the device status word of `ws` (async on `stream`). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
 

@@ -58,6 +58,19 @@ def test_workspace_sizes(lib):
     assert lib.moe_dispatch_meta_workspace_size(100, 2, 4) >= 256
 
 
+def test_gather_rows_flag_drops_the_permuted_copy(lib):
+    N, H, E, K, F = 4096, 4096, 8, 2, 14336
+    P = lib.moe_padded_rows_max(N, E, K)
+    G = _lib.MOE_LAYER_GATHER_ROWS
+    for mode in (0, 1, 2):
+        plain = lib.moe_workspace_size(N, H, E, K, F, MOE_BF16, mode)
+        gathered = lib.moe_workspace_size(N, H, E, K, F, MOE_BF16, mode | G)
+        assert plain - gathered == P * H * 2, mode
+    assert lib.moe_workspace_size(N, H, E, K, F, MOE_BF16, 3) == 0            # no mode 3
+    assert lib.moe_workspace_size(N, H, E, K, F, MOE_BF16, 8) == 0            # unknown flag
+    assert lib.moe_workspace_size(256, 128, 4, 2, 256, MOE_F32, 1 | G) == 0   # bf16 only
+
+
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
 
 
