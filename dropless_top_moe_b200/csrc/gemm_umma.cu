@@ -948,9 +948,15 @@ using namespace umma;
 
 bool umma_shape_supported(int H, int F) { return H % 128 == 0 && F % 128 == 0 && H >= 128 && F >= 128; }
 
-// Kernel choice per GEMM (measured on B200, training-step and forward
-// workloads): CTA pairs wherever a 256 x 256 tile fits, except the dgrad to x,
-// whose 256-row single-CTA tiles were faster.
+// Kernel choice per GEMM (measured on B200, interleaved in one process on the
+// training-step and forward workloads).  A CTA pair (256 x 256, one 128-row
+// tile per CTA) halves each CTA's B traffic and keeps two accumulator sets in
+// TMEM, so a heavy epilogue (SwiGLU, SwiGLU backward, weight gradients)
+// overlaps the next tile's main loop; but a pair always multiplies 256 rows,
+// and an expert with an odd tile count wastes half of its last unit.  A single
+// CTA with two 128-row halves (256 x 256, one accumulator set) skips the MMA of
+// a missing half; with a light store epilogue that wins: GEMM2 and the dgrad
+// to x run that way (GEMM2 8-20 % faster than in pairs), the rest in pairs.
 
 // [G | U] = x_perm * [W1_e | W3_e] per group; act = silu(G) * U.  act, G and U
 // may each be NULL (the backward's recompute asks for G and U only).
@@ -979,7 +985,6 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
                                const int32_t* pb, int E, int H, int F, int64_t P, void* act, void* out,
                                void* gate_up, int* status, cudaStream_t s, const RowGather* ga) {
   typedef __nv_bfloat16 bf;
-  const bool pair = true;
   // GEMM1 + SwiGLU: [G | U] = x_perm * [W1_e | W3_e], act = silu(G) * U
   moe_status st = gemm1_umma(x_perm, W1, W3, pb, E, H, F, P, act,
                              gate_up ? (bf*)gate_up : nullptr,
@@ -987,7 +992,6 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
   if (st != MOE_OK) return st;
   // GEMM2: out = act * W2_e
   {
-    (void)pair;
     Params p = blank_params(pb, E, P, status);
     const int bn = (H % 256 == 0) ? 256 : 128;
     if (!map2d(&p.ta0, act, F, P, F, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, 64)) return MOE_ERR_CUDA;
@@ -997,7 +1001,6 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.out0 = (bf*)out;
     p.ldo = H;
     const int64_t up = (P / BM) * p.n_tiles;
-    if (bn == 256 && pair) return launch<256, 1, 2, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
     if (bn == 256) return launch<256, 2, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
     return launch<128, 1, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
   }
