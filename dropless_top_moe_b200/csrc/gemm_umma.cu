@@ -381,11 +381,22 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
 
 // B tile of one k block into sb; k is the k offset (ROWS / DENSE) or the
 // group row (WGRAD); tb is the map to read (SPLIT_K picks it per k block).
-// In a pair each CTA fetches its half of B's columns (SPLIT_N: W1 | W3).
+// In a pair each CTA fetches its half of B's columns (SPLIT_N: W1 | W3).  On a
+// lone unit (an M = 128 pair MMA, see the kernel) CTA r's half feeds the TMEM
+// lanes 64r.. of both CTAs, so with SPLIT_N each CTA takes 64 columns of W1
+// and the same 64 of W3, keeping a gate and its up projection in one lane.
 template <int BN, int CG, int SCHED, bool B_MN, int SPLIT>
 __device__ __forceinline__ void load_b(const Params& p, const Tile& tl, uint32_t sb, uint32_t fb,
-                                       uint32_t rank, int k, const CUtensorMap* tb) {
+                                       uint32_t rank, int k, const CUtensorMap* tb, bool lone = false) {
   if constexpr (CG == 2) {
+    if constexpr (SCHED == SCHED_ROWS && B_MN && SPLIT == SPLIT_N) {
+      if (lone) {
+        static_assert(BN == 256, "lone SPLIT_N units take one 64-column box of W1 and of W3 per CTA");
+        tma_load_3d_pair(sb, &p.tb0, fb, tl.n0 + 64 * (int)rank, k, tl.e);
+        tma_load_3d_pair(sb + 8192, &p.tb1, fb, tl.n0 + 64 * (int)rank, k, tl.e);
+        return;
+      }
+    }
     if constexpr (SCHED == SCHED_WGRAD) {
 #pragma unroll
       for (int j = 0; j < BN / 128; ++j) {
@@ -443,6 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   constexpr int ACC_COLS = S::ACC_COLS;
   constexpr int UNIT = S::UNIT;
   constexpr bool PAIR = CG == 2;
+  // A pair's unit whose second 128-row tile does not exist (an expert with an
+  // odd tile count) runs as an M = 128 pair MMA: CTA r multiplies rows
+  // 64r .. 64r + 63 of the tile, and each CTA's TMEM receives its 64 rows
+  // twice, lanes 0-63 holding output columns [0, BN/2) and lanes 64-127
+  // columns [BN/2, BN), both in accumulator columns [0, BN/2).
+  constexpr bool LONE = PAIR && MT == 1 && SCHED == SCHED_ROWS &&
+                        (EPI != EPI_SWIGLU || (SPLIT == SPLIT_N && B_MN && BN == 256));
   static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte swizzle atoms aligned");
   static_assert(STAGES >= 2, "pipeline needs at least two stages");
   static_assert(MT == 1 || SCHED != SCHED_DENSE, "the router uses single 128-row tiles");
@@ -555,7 +573,9 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
             const int hh = PAIR ? 2 * h + (int)rank : h;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              tk[h][i] = h < n_mma_h ? tok_of(tl.row0 + hh * BM + 4 * lane + i) : p.g_N;
+              tk[h][i] = h < n_mma_h ? tok_of(tl.row0 + (LONE && tl.halves == 1 ? 64 * (int)rank : hh * BM) +
+                                              4 * lane + i)
+                                     : p.g_N;
           }
         } else {
 #pragma unroll
@@ -573,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           const int kc = SCHED == SCHED_WGRAD ? (int)(tl.row0 + (int64_t)kb * BK) : kb * BK;
           if (lane == 0) {
             if (!PAIR || rank == 0) mbar_expect_tx(full_bar(stage), tx);
-            load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, kc, &p.tb0);
+            load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, kc, &p.tb0, LONE && tl.halves == 1);
           }
           if constexpr (SCHED == SCHED_WGRAD) {
             int cur[4];
@@ -640,9 +660,11 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
               const CUtensorMap* ta = &p.ta0;
               const CUtensorMap* tb = &p.tb0;
               if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
+              const bool lone = LONE && tl.halves == 1;
               for (int h = 0; h < n_mma_h; ++h)
-                tma_load_2d_pair(sa + h * (BM * BK * 2), ta, fb, k, (int)tl.row0 + BM * (2 * h + (int)rank));
-              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, k, tb);
+                tma_load_2d_pair(sa + h * (BM * BK * 2), ta, fb, k,
+                                 (int)tl.row0 + (lone ? 64 * (int)rank : BM * (2 * h + (int)rank)));
+              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, k, tb, lone);
             }
           } else {
             const uint32_t fb = full_bar(stage);
@@ -676,7 +698,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && rank == 0) {
       const int n_mma = (SCHED == SCHED_DENSE) ? p.n_mma : BN;
-      const uint32_t idesc = idesc_bf16(PAIR ? 2 * BM : BM, n_mma, A_MN, B_MN);
+      const uint32_t idesc_full = idesc_bf16(PAIR ? 2 * BM : BM, n_mma, A_MN, B_MN);
+      const uint32_t idesc_lone = idesc_bf16(BM, n_mma, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -688,6 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
         if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+        const uint32_t idesc = (LONE && tl.halves == 1) ? idesc_lone : idesc_full;
         for (int kb = 0; kb < tl.nkb; ++kb) {
           if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
           tc_fence_after();
@@ -768,11 +792,26 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
+      bool lone_done = false;
+      if constexpr (LONE) {
+        if (tl.halves == 1) {
+          // M = 128 result: rows 64 * rank + (q & 1) * 32 + lane, lanes 64g..
+          // holding output columns [g * BN/2, (g + 1) * BN/2) of the MMA (with
+          // SPLIT_N SwiGLU: 64 gate and 64 up columns of act columns 64g..)
+          const int g = q >> 1;
+          const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+          Tile th = tl;
+          th.row0 = tl.row0 + 64 * (int)rank;
+          th.n0 = tl.n0 + g * (EPI == EPI_SWIGLU ? BN / 4 : BN / 2);
+          epilogue_half<BN / 2, SCHED, EPI>(p, th, tacc, (q & 1) * 32 + lane, part);
+          lone_done = true;
+        }
+      }
       if constexpr (PAIR) {
         // this CTA's tiles 2h + rank of the unit; tiles past the expert's end
         // (a short last unit) are computed on garbage rows and not stored
 #pragma unroll 1
-        for (int h = 0; h < MT; ++h) {
+        for (int h = 0; h < MT && !lone_done; ++h) {
           const int j = 2 * h + (int)rank;
           if (j >= tl.halves) continue;
           const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
