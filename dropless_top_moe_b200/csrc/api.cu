@@ -322,9 +322,10 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
                          int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
   MOE_TRY(check_ffn(H, F, dt));
-  const void* ptrs[] = {x, W_r, W1, W3, W2, y, top_experts, weights, indices, bins, padded_bins};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  // token-sized arrays may be NULL for an empty batch (N = 0)
+  const void* ptrs[] = {W_r, W1, W3, W2, bins, padded_bins, x, y, top_experts, weights, indices};
+  for (int i = 0; i < 11; ++i)
+    if ((!ptrs[i] && (i < 6 || N > 0)) || !aligned16(ptrs[i])) return MOE_ERR_INVALID_ARG;
   if (!layer_flags_ok(training, dt)) return MOE_ERR_INVALID_ARG;
   const size_t need = moe_workspace_size(N, H, E, K, F, dt, training);
   if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
@@ -358,14 +359,27 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                          moe_stream_t stream) {
   MOE_TRY(check_shape(N, H, E, K, dt));
   MOE_TRY(check_ffn(H, F, dt));
-  const void* ptrs[] = {dy, x, W_r, W1, W3, W2, top_experts, weights, indices, bins, padded_bins,
-                        dx, dW_r, dW1, dW3, dW2};
-  for (const void* q : ptrs)
-    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  // token-sized arrays may be NULL for an empty batch (N = 0)
+  const void* ptrs[] = {W_r, W1, W3, W2, bins, padded_bins, dW_r, dW1, dW3, dW2,
+                        dy, x, top_experts, weights, indices, dx};
+  for (int i = 0; i < 16; ++i)
+    if ((!ptrs[i] && (i < 10 || N > 0)) || !aligned16(ptrs[i])) return MOE_ERR_INVALID_ARG;
   if (!layer_flags_ok(training, dt) || ((training & 3) != 1 && (training & 3) != 2)) return MOE_ERR_INVALID_ARG;
   const size_t need = moe_workspace_size(N, H, E, K, F, dt, training);
   if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
+  if (N == 0) {
+    // no tokens: every weight gradient is an empty sum
+    const size_t eb = elem_bytes(dt);
+    if (cudaMemsetAsync(dW_r, 0, (size_t)H * E * eb, s) != cudaSuccess ||
+        cudaMemsetAsync(dW1, 0, (size_t)E * H * F * eb, s) != cudaSuccess ||
+        cudaMemsetAsync(dW3, 0, (size_t)E * H * F * eb, s) != cudaSuccess ||
+        cudaMemsetAsync(dW2, 0, (size_t)E * F * H * eb, s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+  }
   LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
   const RowGather ga = {x, indices, bins, N, K};

@@ -389,9 +389,8 @@ template <int BN, int CG, int SCHED, bool B_MN, int SPLIT>
 __device__ __forceinline__ void load_b(const Params& p, const Tile& tl, uint32_t sb, uint32_t fb,
                                        uint32_t rank, int k, const CUtensorMap* tb, bool lone = false) {
   if constexpr (CG == 2) {
-    if constexpr (SCHED == SCHED_ROWS && B_MN && SPLIT == SPLIT_N) {
-      if (lone) {
-        static_assert(BN == 256, "lone SPLIT_N units take one 64-column box of W1 and of W3 per CTA");
+    if constexpr (SCHED == SCHED_ROWS && B_MN && SPLIT == SPLIT_N && BN == 256) {
+      if (lone) {   // one 64-column box of W1 and the same of W3 per CTA
         tma_load_3d_pair(sb, &p.tb0, fb, tl.n0 + 64 * (int)rank, k, tl.e);
         tma_load_3d_pair(sb + 8192, &p.tb1, fb, tl.n0 + 64 * (int)rank, k, tl.e);
         return;

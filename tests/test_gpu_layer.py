@@ -240,3 +240,27 @@ def test_memory_optimised_backward_is_bit_identical(shape):
     assert torch.equal(outs[1][0], outs[2][0])
     for k in outs[1][1]:
         assert torch.equal(outs[1][1][k], outs[2][1][k]), k
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_empty_batch(dtype):
+    """N = 0: the forward writes all-zero bins and nothing else; the backward
+    gives zero weight gradients (sums over no tokens).  Token-sized buffers
+    are empty tensors (NULL pointers)."""
+    H, F = (256, 256) if dtype == "bf16" else (64, 96)
+    shape = small_shape("empty", N=0, H=H, E=8, K=2, F=F, dtype=dtype, training=True)
+    c = make_case(shape, seed=3, with_dy=True)
+    layer = moe.MoELayer(0, H, shape.E, shape.K, F, dtype=shape.torch_dtype, training=True)
+    layer.bins.fill_(-1)
+    layer.padded_bins.fill_(-1)
+    y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    g = layer.grad_buffers()
+    for v in g.values():
+        v.fill_(1.0)
+    layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert tuple(y.shape) == (0, H)
+    assert int(layer.bins.abs().sum()) == 0 and int(layer.padded_bins.abs().sum()) == 0
+    for k in ("dW_r", "dW1", "dW3", "dW2"):
+        assert int(torch.count_nonzero(g[k])) == 0, k
