@@ -300,7 +300,7 @@ moe_status moe_unpermute_router_bwd(const void* dx_perm, const float* dlogit, co
   if (aux)
     return dense_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, bins, probs, N, H, E, K, dt, aux_alpha,
                             aux_grad, dx, dW_r, scratch + al256(unpermute_router_bwd_scratch(H, E, P)),
-                            (cudaStream_t)stream);
+                            (int*)ws, (cudaStream_t)stream);
   return unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins, N,
                               H, E, K, P, dt, dx, dW_r, scratch, (cudaStream_t)stream);
 }
@@ -407,7 +407,7 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
   // and dropped assignments need every (token, expert) logit: dense path
   if ((aux_alpha != 0.0f || capacity > 0) && N > 0)
     MOE_TRY(dense_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, bins, w.probs, N, H, E, K, dt,
-                             aux_alpha, aux_grad, dx, dW_r, w.dense_scratch, s));
+                             aux_alpha, aux_grad, dx, dW_r, w.dense_scratch, w.status, s));
   else
     MOE_TRY(unpermute_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, indices, bins,
                                  padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, s));

@@ -12,7 +12,11 @@
 //   a_t,e = g * alpha*E/N * p_t,e * (f_e - sum_i f_i p_t,i)      (g = dL/dL_aux)
 // D[t,e] = a_t,e + the renormalisation gradient of token t's kept experts.
 // Then dx[t] = sum_k dX_perm[pos(t,k)] + sum_e D[t,e] W_r[:,e] and
-// dW_r = x^T D, both as tiled fp32 reductions in a fixed order.
+// dW_r = x^T D.  bf16 layers with E % 64 == 0 and H % 256 == 0 run both as
+// tcgen05 GEMMs on D rounded once to bf16 (gemm_umma.cu); otherwise tiled
+// fp32 CUDA-core reductions here.  Every sum runs in a fixed order.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -57,11 +61,20 @@ aux_finalize_kernel(const float* __restrict__ part, int n_chunks, const int32_t*
   if (e == 0) *loss = alpha * (float)E * s_v[0];
 }
 
-// D[t, e] for one token per warp.
+// D[t, e] for one token per warp, into D (fp32) or Dh (bf16, for the
+// tensor-core kernels, which also get the token-chunk ends chunk_end[c] =
+// min((c + 1) * chunk, N rounded up to 64)).
 __global__ void __launch_bounds__(256)
 router_dense_dlogits_kernel(const float* __restrict__ probs, const float* __restrict__ dlogit,
                             const int32_t* __restrict__ top, const int32_t* __restrict__ bins, int N, int E,
-                            int K, float coef, float* __restrict__ D) {
+                            int K, float coef, float* __restrict__ D, __nv_bfloat16* __restrict__ Dh,
+                            int32_t* __restrict__ chunk_end, int chunk) {
+  if (chunk_end && blockIdx.x == 0) {
+    const int n_chunks = (N + chunk - 1) / chunk;
+    const int last = (int)round_up(N, 64);
+    for (int c = threadIdx.x; c < n_chunks; c += blockDim.x)
+      chunk_end[c] = (c + 1) * chunk < last ? (c + 1) * chunk : last;
+  }
   __shared__ float s_f[256];
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     s_f[e] = (float)(bins[e] - (e ? bins[e - 1] : 0)) / ((float)N * (float)K);
@@ -77,7 +90,8 @@ router_dense_dlogits_kernel(const float* __restrict__ probs, const float* __rest
       float d = coef * p[e] * (s_f[e] - s);
       for (int k = 0; k < K; ++k)
         if (top[(size_t)t * K + k] == e) d += dlogit[(size_t)t * K + k];
-      D[(size_t)t * E + e] = d;
+      if (Dh) Dh[(size_t)t * E + e] = __float2bfloat16(d);
+      else D[(size_t)t * E + e] = d;
     }
   }
 }
@@ -204,7 +218,10 @@ constexpr int kWgradChunk = 1024;
 size_t aux_loss_scratch(int N, int E) { return (size_t)cdiv(N > 0 ? N : 1, kAuxChunk) * E * sizeof(float); }
 
 size_t dense_router_bwd_scratch(int N, int H, int E) {
-  return (size_t)N * E * sizeof(float) + (size_t)cdiv(N > 0 ? N : 1, kWgradChunk) * H * E * sizeof(float);
+  // fp32 D (or bf16 D) | partials [chunks, H, E] fp32 | chunk ends
+  const int64_t chunks = cdiv(N > 0 ? N : 1, kWgradChunk);
+  return (size_t)round_up((int64_t)N * E * sizeof(float), 256) + (size_t)chunks * H * E * sizeof(float) +
+         (size_t)round_up(chunks * 4, 256);
 }
 
 moe_status aux_loss_fwd(const float* probs, const int32_t* bins, int N, int K, int E, float alpha, float* loss,
@@ -223,15 +240,35 @@ template <typename T>
 static moe_status dense_router_bwd_t(const void* dx_perm, const float* dlogit, const void* x, const void* W_r,
                                      const int32_t* top, const int32_t* pos, const int32_t* bins,
                                      const float* probs, int N, int H, int E, int K, float coef, void* dx,
-                                     void* dWr, void* scratch, cudaStream_t s) {
+                                     void* dWr, void* scratch, int* status, cudaStream_t s) {
   float* D = (float*)scratch;
-  float* part = D + (size_t)N * E;
+  float* part = (float*)((char*)scratch + round_up((int64_t)N * E * sizeof(float), 256));
   const int warps = 8;
   int blocks = (int)cdiv(N, warps);
   if (blocks > 148 * 8) blocks = 148 * 8;
   if (blocks < 1) blocks = 1;
+  if (std::is_same<T, __nv_bfloat16>::value && router_bwd_umma_supported(H, E)) {
+    // tensor cores: D in bf16 (rounded once from the fp32 value), then
+    // dx = D * W_r^T + unpermute sum and dW_r = x^T * D as tcgen05 GEMMs
+    // scratch: Dh [N, E] bf16 (in D's place) | fp32 partials | chunk ends
+    const int n_chunks = (int)cdiv(N, kWgradChunk);
+    __nv_bfloat16* Dh = (__nv_bfloat16*)scratch;
+    int32_t* chunk_end = (int32_t*)(part + (size_t)n_chunks * H * E);
+    MOE_TRACED("router_dense_dlogits", s, (router_dense_dlogits_kernel<<<blocks, 256, 0, s>>>(
+                                              probs, dlogit, top, bins, N, E, K, coef, nullptr, Dh, chunk_end,
+                                              kWgradChunk)));
+    MOE_LAUNCH_CHECK();
+    moe_status st = router_dx_umma(Dh, W_r, N, H, E, dx, status, s);
+    if (st == MOE_OK) st = unpermute_add_rows(dx_perm, pos, N, H, K, MOE_BF16, dx, s);
+    if (st == MOE_OK) st = router_wgrad_umma(x, Dh, chunk_end, n_chunks, N, H, E, part, status, s);
+    if (st != MOE_OK) return st;
+    MOE_TRACED("dense_router_wgrad_reduce", s, (dense_router_wgrad_reduce_kernel<T><<<(unsigned)cdiv((int64_t)H * E, 256),
+                                                   256, 0, s>>>(part, n_chunks, H, E, (T*)dWr)));
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+  }
   MOE_TRACED("router_dense_dlogits", s, (router_dense_dlogits_kernel<<<blocks, 256, 0, s>>>(
-                                            probs, dlogit, top, bins, N, E, K, coef, D)));
+                                            probs, dlogit, top, bins, N, E, K, coef, D, nullptr, nullptr, 1)));
   MOE_LAUNCH_CHECK();
   dim3 g1((unsigned)cdiv(H, kDT), (unsigned)cdiv(N, kDT));
   MOE_TRACED("dense_router_dx", s, (dense_router_dx_kernel<T><<<g1, 256, 0, s>>>(
@@ -251,14 +288,14 @@ static moe_status dense_router_bwd_t(const void* dx_perm, const float* dlogit, c
 moe_status dense_router_bwd(const void* dx_perm, const float* dlogit, const void* x, const void* W_r,
                             const int32_t* top, const int32_t* pos, const int32_t* bins, const float* probs,
                             int N, int H, int E, int K, moe_dtype dt, float aux_alpha, float aux_grad,
-                            void* dx, void* dWr, void* scratch, cudaStream_t s) {
+                            void* dx, void* dWr, void* scratch, int* status, cudaStream_t s) {
   if (N == 0) return MOE_OK;
   const float coef = aux_grad * aux_alpha * (float)E / (float)N;
   return dt == MOE_F32
              ? dense_router_bwd_t<float>(dx_perm, dlogit, x, W_r, top, pos, bins, probs, N, H, E, K, coef, dx,
-                                         dWr, scratch, s)
+                                         dWr, scratch, status, s)
              : dense_router_bwd_t<__nv_bfloat16>(dx_perm, dlogit, x, W_r, top, pos, bins, probs, N, H, E, K,
-                                                 coef, dx, dWr, scratch, s);
+                                                 coef, dx, dWr, scratch, status, s);
 }
 
 }  // namespace moe

@@ -46,7 +46,7 @@ constexpr int kGroupM = 8;          // M tiles per raster group (L2 reuse of B p
 
 enum Sched { SCHED_ROWS = 0, SCHED_WGRAD = 1, SCHED_DENSE = 2 };
 enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3, EPI_WGRAD_PAIR = 4,
-           EPI_ROUTER = 5 };
+           EPI_ROUTER = 5, EPI_ROUTER_DX = 6, EPI_WGRAD_F32 = 7 };
 enum Split { SPLIT_NONE = 0, SPLIT_K = 1, SPLIT_N = 2 };
 
 struct Params {
@@ -133,7 +133,7 @@ __device__ __forceinline__ int64_t total_tiles(const Params& p, const int32_t* s
   } else if constexpr (SCHED == SCHED_WGRAD) {
     return (int64_t)p.E * p.m_tiles_w * p.n_tiles;
   } else {
-    return cdiv(p.P, BM);
+    return cdiv(p.P, BM) * (p.n_tiles > 1 ? p.n_tiles : 1);
   }
 }
 
@@ -184,10 +184,12 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32
     tl.nkb = hi > lo ? (int)((hi - lo) / BK) : 0;
     tl.halves = UNIT;
   } else {
+    // plain row tiles x n_tiles column tiles (the router: one column tile)
+    const int64_t nt = p.n_tiles > 1 ? p.n_tiles : 1;
     tl.e = 0;
-    tl.row0 = t * BM;
+    tl.row0 = (t / nt) * BM;
     tl.m0 = 0;
-    tl.n0 = 0;
+    tl.n0 = (int)((t % nt) * BN);
     tl.nkb = p.kdim / BK;
     tl.halves = 1;
   }
@@ -357,7 +359,7 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       store_row_bf16x32(p.out0 + off + c, dg);
       store_row_bf16x32(p.out1 + off + c, du);
     }
-  } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) {
+  } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR || EPI == EPI_WGRAD_F32) {
     const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
 #pragma unroll 1
     for (int c = c_begin; c < c_end; c += 32) {
@@ -367,10 +369,32 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       float v[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-      if (EPI == EPI_WGRAD_PAIR && c >= BN / 2)
+      if constexpr (EPI == EPI_WGRAD_F32) {
+        // fp32 partial sums (one slice per group, reduced in order afterwards)
+        float4* d = reinterpret_cast<float4*>(p.logits + off + c);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else if (EPI == EPI_WGRAD_PAIR && c >= BN / 2) {
         store_row_bf16x32(p.out1 + off + (c - BN / 2), v);
-      else
+      } else {
         store_row_bf16x32(p.out0 + off + c, v);
+      }
+    }
+  } else if constexpr (EPI == EPI_ROUTER_DX) {
+    // router backward, dense: out0[t, n0 + c] = (D * W_r^T)[t, n0 + c] for the
+    // tile's rows below P (= N); the unpermute pass then adds the K rows
+    const bool valid = grow < p.P;
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      tmem_ld_wait();
+      if (valid) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        store_row_bf16x32(p.out0 + grow * p.ldo + tl.n0 + c, v);
+      }
     }
   } else {  // EPI_ROUTER: softmax, top-K, renormalise on this row's E logits
     if (part != 0) return;
@@ -427,7 +451,7 @@ __device__ __forceinline__ void load_b(const Params& p, const Tile& tl, uint32_t
     } else if constexpr (SCHED == SCHED_DENSE && B_MN) {
       for (int j = 0; j < p.n_mma / 64; ++j) tma_load_2d(sb + j * 8192, tb, fb, 64 * j, k);
     } else if constexpr (SCHED == SCHED_DENSE) {
-      tma_load_2d(sb, tb, fb, k, 0);
+      tma_load_2d(sb, tb, fb, k, tl.n0);
     } else if constexpr (B_MN) {
 #pragma unroll
       for (int j = 0; j < BN / 64; ++j) {
@@ -777,6 +801,13 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
               for (int c = part * (BN / 4); c < (part + 1) * (BN / 4); c += 32) {
                 store_row_bf16x32(p.out0 + off + c, z);
                 store_row_bf16x32(p.out1 + off + c, z);
+              }
+            } else if constexpr (EPI == EPI_WGRAD_F32) {
+#pragma unroll 1
+              for (int c = part * (BN / 2); c < (part + 1) * (BN / 2); c += 32) {
+                float4* d = reinterpret_cast<float4*>(p.logits + off + c);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) d[q] = make_float4(0.f, 0.f, 0.f, 0.f);
               }
             } else {
 #pragma unroll 1
@@ -1178,6 +1209,45 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   p.weights = w;
   if (mn) return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER, false, true, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
   return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
+}
+
+// ---- dense router backward on tensor cores ----------------------------------
+
+bool router_bwd_umma_supported(int H, int E) { return E % 64 == 0 && E <= 256 && H % 256 == 0; }
+
+// dx = D * W_r^T (the unpermute pass adds the K expert rows afterwards, in
+// place): D [N, E] bf16 is K-major A, W_r [H, E] K-major B (its rows are the
+// output columns); 128-token x 256-column tiles, K = E.
+moe_status router_dx_umma(const void* D, const void* W_r, int N, int H, int E, void* dx, int* status,
+                          cudaStream_t s) {
+  typedef __nv_bfloat16 bf;
+  Params p = blank_params(nullptr, 1, N, status);
+  if (!map2d(&p.ta0, D, E, N, E, 64, 128) || !map2d(&p.tb0, W_r, E, H, E, 64, 256)) return MOE_ERR_CUDA;
+  p.kdim = E;
+  p.n_mma = 256;
+  p.n_tiles = H / 256;
+  p.out0 = (bf*)dx;
+  p.ldo = H;
+  return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER_DX, false, false, SPLIT_NONE>(
+      "dense_router_dx", p, cdiv(N, BM) * p.n_tiles, s);
+}
+
+// dW_r partials: part[c] = x[chunk c]^T * D[chunk c] for token chunks whose
+// ends (multiples of 64, the last = N rounded up to 64) are chunk_end[c], one
+// weight-gradient group per chunk; x [N, H] and D [N, E] both MN-major, the
+// tokens past N read as zeros.  part: [n_chunks, H, E] fp32.
+moe_status router_wgrad_umma(const void* x, const void* D, const int32_t* chunk_end, int n_chunks, int N,
+                             int H, int E, float* part, int* status, cudaStream_t s) {
+  Params p = blank_params(chunk_end, n_chunks, round_up(N, BK), status);
+  if (!map2d(&p.ta0, x, H, N, H, 64, 64) || !map2d(&p.tb0, D, E, N, E, 64, 64)) return MOE_ERR_CUDA;
+  p.n_mma = 64;
+  p.m_tiles_w = H / BM;
+  p.n_tiles = E / 64;
+  p.logits = part;
+  p.ldo = E;
+  p.out_estride = (int64_t)H * E;
+  return launch<64, 1, 1, SCHED_WGRAD, EPI_WGRAD_F32, true, true, SPLIT_NONE>(
+      "dense_router_wgrad", p, (int64_t)n_chunks * p.m_tiles_w * p.n_tiles, s);
 }
 
 }  // namespace moe

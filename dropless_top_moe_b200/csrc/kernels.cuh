@@ -26,6 +26,9 @@ moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices
 // permute.cu
 moe_status permute_rows(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* pb,
                         int N, int H, int E, int K, moe_dtype dt, void* x_perm, cudaStream_t s);
+// dx[t] = (sum_k dx_perm[pos[t, k]], in increasing k) + dx[t], in place
+moe_status unpermute_add_rows(const void* dx_perm, const int32_t* pos, int N, int H, int K, moe_dtype dt,
+                              void* dx, cudaStream_t s);
 moe_status combine_rows(const void* out, const float* w, const int32_t* pos, int N, int K, int H,
                         moe_dtype dt, void* y, cudaStream_t s);
 moe_status combine_bwd_rows(const void* dy, const void* out, const float* w, const int32_t* pos,
@@ -48,7 +51,7 @@ moe_status aux_loss_fwd(const float* probs, const int32_t* bins, int N, int K, i
 moe_status dense_router_bwd(const void* dx_perm, const float* dlogit, const void* x, const void* W_r,
                             const int32_t* top, const int32_t* pos, const int32_t* bins, const float* probs,
                             int N, int H, int E, int K, moe_dtype dt, float aux_alpha, float aux_grad,
-                            void* dx, void* dWr, void* scratch, cudaStream_t s);
+                            void* dx, void* dWr, void* scratch, int* status, cudaStream_t s);
 
 // gemm_simt.cu - fp32 grouped GEMMs
 moe_status grouped_swiglu_simt(const void* x_perm, const void* W1, const void* W3, const void* W2,
@@ -84,6 +87,14 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
                                const int32_t* pb, int E, int H, int F, int64_t P, void* act,
                                void* out, void* gate_up, int* status, cudaStream_t s,
                                const RowGather* ga = nullptr);
+// Dense router backward (bf16, E % 64 == 0, H % 256 == 0): dx = D * W_r^T
+// (then unpermute_add_rows), and per-token-chunk fp32 partials of x^T * D
+// (then an in-order reduction over the chunks); D [N, E] bf16.
+bool router_bwd_umma_supported(int H, int E);
+moe_status router_dx_umma(const void* D, const void* W_r, int N, int H, int E, void* dx, int* status,
+                          cudaStream_t s);
+moe_status router_wgrad_umma(const void* x, const void* D, const int32_t* chunk_end, int n_chunks, int N,
+                             int H, int E, float* part, int* status, cudaStream_t s);
 moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const void* act,
                                    const void* gate_up, const void* W1, const void* W3,
                                    const void* W2, const int32_t* pb, int E, int H, int F, int64_t P,

@@ -188,7 +188,10 @@ __global__ void transpose_kernel(const T* __restrict__ in, int R, int C, int C_p
   }
 }
 
-// dx[t] = sum_k dx_perm[pos[t,k]] + sum_k dlogit[t,k] * W_rT[top[t,k]]
+// dx[t] = sum_k dx_perm[pos[t,k]] + sum_k dlogit[t,k] * W_rT[top[t,k]];
+// with WrT == NULL the second term is dx[t]'s own value (read, then
+// overwritten by the same thread): the dense router backward stores its
+// D * W_r^T there first.
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads)
 unpermute_dx_kernel(const T* __restrict__ dx_perm, const float* __restrict__ dlogit,
@@ -199,8 +202,8 @@ unpermute_dx_kernel(const T* __restrict__ dx_perm, const float* __restrict__ dlo
   const int nvec = H / V;
   for (int t = grid_warp(); t < N; t += grid_warps()) {
     const int my_pos = lane < K ? pos[(size_t)t * K + lane] : -1;
-    const float my_dl = lane < K ? dlogit[(size_t)t * K + lane] : 0.f;
-    const int my_e = lane < K ? top[(size_t)t * K + lane] : 0;
+    const float my_dl = (WrT && lane < K) ? dlogit[(size_t)t * K + lane] : 0.f;
+    const int my_e = (WrT && lane < K) ? top[(size_t)t * K + lane] : 0;
     for (int v0 = 0; v0 < nvec; v0 += 32 * kSeg) {
       float acc[kSeg][V];
 #pragma unroll
@@ -222,7 +225,20 @@ unpermute_dx_kernel(const T* __restrict__ dx_perm, const float* __restrict__ dlo
           }
         }
       }
-      for (int k = 0; k < K; ++k) {
+      if (!WrT) {
+        const T* add = dx + (size_t)t * H;
+#pragma unroll
+        for (int s = 0; s < kSeg; ++s) {
+          const int v = v0 + s * 32 + lane;
+          if (v < nvec) {
+            float f[V];
+            Vec<T>::to_float(*reinterpret_cast<const uint4*>(add + (size_t)v * V), f);
+#pragma unroll
+            for (int j = 0; j < V; ++j) acc[s][j] += f[j];
+          }
+        }
+      }
+      for (int k = 0; k < K && WrT; ++k) {
         const int p = __shfl_sync(0xffffffffu, my_pos, k);
         const float dl = __shfl_sync(0xffffffffu, my_dl, k);
         const int e = __shfl_sync(0xffffffffu, my_e, k);
@@ -417,6 +433,21 @@ static moe_status unpermute_router_bwd_t(const void* dx_perm, const float* dlogi
   MOE_LAUNCH_CHECK();
   dim3 g2((unsigned)cdiv(H, 256), (unsigned)E);
   MOE_TRACED("router_wgrad_reduce", s, (router_wgrad_reduce_kernel<T><<<g2, 256, 0, s>>>(part, padded_bins, E, H, (T*)dWr)));
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+moe_status unpermute_add_rows(const void* dx_perm, const int32_t* pos, int N, int H, int K, moe_dtype dt,
+                              void* dx, cudaStream_t s) {
+  if (N == 0) return MOE_OK;
+  if (dt == MOE_F32) {
+    MOE_TRACED("unpermute_dx", s, (unpermute_dx_kernel<float><<<row_grid(N), kRowThreads, 0, s>>>(
+                                      (const float*)dx_perm, nullptr, nullptr, nullptr, pos, N, H, K, (float*)dx)));
+  } else {
+    MOE_TRACED("unpermute_dx", s, (unpermute_dx_kernel<__nv_bfloat16><<<row_grid(N), kRowThreads, 0, s>>>(
+                                      (const __nv_bfloat16*)dx_perm, nullptr, nullptr, nullptr, pos, N, H, K,
+                                      (__nv_bfloat16*)dx)));
+  }
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

@@ -137,9 +137,14 @@ def test_layer_is_bitwise_deterministic():
         assert torch.equal(a, b)
 
 
+# bf16 with E % 64 == 0 and H % 256 == 0 runs the dense router backward on
+# tensor cores (D rounded to bf16); the other shapes on CUDA cores in fp32
 AUX = [small_shape("aux_f32", N=256, H=64, E=8, K=2, F=96, dtype="f32", training=True),
        small_shape("aux_bf16", N=700, H=256, E=64, K=4, F=256, training=True),
-       small_shape("aux_bf16_e8", N=333, H=128, E=8, K=2, F=128, training=True)]
+       small_shape("aux_bf16_e128", N=1500, H=512, E=128, K=6, F=256, skew="zipf", skew_param=1.0,
+                   training=True),
+       small_shape("aux_bf16_e8", N=333, H=128, E=8, K=2, F=128, training=True),
+       small_shape("aux_bf16_n3", N=3, H=256, E=64, K=2, F=256, training=True)]
 
 
 @pytest.mark.parametrize("shape", AUX, ids=lambda s: s.name)
@@ -176,6 +181,8 @@ def test_aux_loss_stage_matches_oracle():
 
 CAP = [small_shape("cap_f32", N=256, H=64, E=8, K=2, F=96, dtype="f32", training=True),
        small_shape("cap_bf16_zipf", N=900, H=256, E=16, K=4, F=256, skew="zipf", skew_param=1.0,
+                   training=True),
+       small_shape("cap_bf16_e64", N=1000, H=256, E=64, K=4, F=256, skew="zipf", skew_param=1.0,
                    training=True)]
 
 
