@@ -48,6 +48,7 @@ SIGNATURES = {
                             FL, FL, P, P, P, P, P, P, SZ, P]),
     "moe_dispatch_meta_noalloc": (I32, [P, I32, I32, I32, P, P, P, P, P, P, P]),
     "moe_sum_rank_ordered": (I32, [P, I32, I64, I32, FL, P, P]),
+    "moe_selftest_wait_timeout": (I32, [P, I64, P]),
     "moe_trace_attach": (I32, [P, I32, P, P]),
     "moe_trace_detach": (I32, []),
 }

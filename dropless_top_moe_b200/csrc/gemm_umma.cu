@@ -517,6 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    // grouped rows beyond the buffers' P rows are not computed: report it
+    if (SCHED != SCHED_DENSE && blockIdx.x == 0 && p.status && p.padded_bins[p.E - 1] > p.P)
+      atomicOr(p.status, MOE_DEVERR_ROWS);
     fence_barrier_init();
     fence_proxy_async();
   }
@@ -945,9 +948,17 @@ static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upp
   Params p = p_in;
   if (p.group_m <= 0) p.group_m = S::UNIT >= 4 ? (kGroupM * 2) / S::UNIT : kGroupM;
   auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return MOE_ERR_CUDA;
+  // once per device: later calls (a CUDA graph capture among them) only launch
+  static bool smem_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!smem_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    smem_set[dev] = true;
   }
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
@@ -967,9 +978,6 @@ static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upp
   int64_t units = sm_count();
   if (CG == 2) {
     static int cached[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
     if (!cached[dev]) {
       int n = 0;
       cfg.gridDim = dim3((unsigned)sm_count(), 1, 1);

@@ -152,8 +152,9 @@ moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices
                                      padded_start)));
   MOE_LAUNCH_CHECK();
   if (NK > 0) {
+    // (32 + 2) * E counters: at most 34 KB for E <= 256, within the default
+    // 48 KB of dynamic shared memory, so no attribute call is needed
     const size_t smem = (size_t)(kMetaPlaceThreads / 32 + 2) * E * sizeof(int);
-    cudaFuncSetAttribute(meta_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     MOE_TRACED("meta_place", s, (meta_place_kernel<<<n_chunks, kMetaPlaceThreads, smem, s>>>(top, NK, E, capacity, chunk_counts,
                                                                 sorted_start, padded_start, indices,
                                                                 bin_ids, pos)));

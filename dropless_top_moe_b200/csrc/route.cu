@@ -114,8 +114,15 @@ static moe_status launch_route_simt(const T* x, const T* W_r, int N, int H, int 
   if (blocks < 1) blocks = 1;
 #define MOE_ROUTE_CASE(EM)                                                                     \
   if (E <= EM) {                                                                               \
-    cudaFuncSetAttribute(route_simt_kernel<T, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                         (int)smem);                                                           \
+    static bool smem_set[64] = {false};                  /* once per device: the 200 KB cap */ \
+    int dev = 0;                                                                               \
+    cudaGetDevice(&dev);                                                                       \
+    if (dev < 0 || dev >= 64) dev = 0;                                                         \
+    if (!smem_set[dev]) {                                                                      \
+      cudaFuncSetAttribute(route_simt_kernel<T, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           200 * 1024);                                                        \
+      smem_set[dev] = true;                                                                    \
+    }                                                                                          \
     MOE_TRACED("route_simt", s,                                                                 \
                (route_simt_kernel<T, EM><<<blocks, threads, smem, s>>>(x, W_r, N, H, E, K, logits,  \
                                                                        probs, top, w)));       \

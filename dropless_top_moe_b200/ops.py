@@ -191,6 +191,13 @@ def moe_aux_loss(probs, bins, K: int, alpha: float, ws=None):
     return loss, P
 
 
+def selftest_wait_timeout(status, timeout_ns: int):
+    """Run the bounded pipeline wait on a barrier nothing arrives at; after
+    timeout_ns it sets MOE_DEVERR_TIMEOUT in status (a device int32 tensor)."""
+    call("moe_selftest_wait_timeout", _p(status), int(timeout_ns), _stream())
+    return status
+
+
 class MoELayer:
     """Whole-layer forward / backward through moe_layer_fwd / moe_layer_bwd.
 

@@ -308,6 +308,16 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
 moe_status moe_sum_rank_ordered(const void* shards, int32_t n_ranks, int64_t numel, moe_dtype dt,
                                 float scale, void* out, moe_stream_t stream);
 
+/* Diagnostics (no counterpart on the pages): one block waits, with the same
+ * bounded mbarrier wait every tcgen05 GEMM pipeline stage uses, on a barrier
+ * that nothing arrives at; after timeout_ns (1 us .. 1 s) it gives up and
+ * sets MOE_DEVERR_TIMEOUT in *status (a device int32, OR-ed in; zero it
+ * first).  The kernel then returns normally and the CUDA context stays
+ * usable: this is how a stalled pipeline surfaces, as a status bit rather
+ * than a hung GPU.  Asynchronous on `stream`; MOE_ERR_INVALID_ARG for a NULL
+ * status or a limit out of range. */
+moe_status moe_selftest_wait_timeout(int32_t* status, int64_t timeout_ns, moe_stream_t stream);
+
 /* Per-launch timing.  While attached, every kernel launch made by any entry
  * point records events[2*i] on its stream just before launch i and
  * events[2*i+1] just after it, stores a static kernel name in labels[i]

@@ -116,3 +116,9 @@ def test_meta_and_grouped_reject_bad_arguments(lib):
     # P must be a multiple of 128
     assert lib.moe_grouped_swiglu(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 128, 256, 100, MOE_BF16, FAKE, FAKE,
                                   None, FAKE, 4096, None) == MOE_ERR_INVALID_ARG
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    assert lib.moe_selftest_wait_timeout(None, 1000000, None) == MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_wait_timeout(FAKE, 10, None) == MOE_ERR_INVALID_ARG            # < 1 us
+    assert lib.moe_selftest_wait_timeout(FAKE, 5 * 10 ** 9, None) == MOE_ERR_INVALID_ARG   # > 1 s

@@ -1,0 +1,48 @@
+"""Failure detection on the GPU without a fault (GPU only).
+
+A stalled pipeline must end its kernel with a status bit the host can read,
+not hang the GPU: every mbarrier wait of the tcgen05 pipelines is bounded.
+The self-test entry point runs that same wait on a barrier nothing arrives
+at.  Grouped rows beyond a caller's buffer are reported the same way.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dropless_top_moe_b200 as moe
+from dropless_top_moe_b200._lib import MOE_DEVERR_ROWS, MOE_DEVERR_TIMEOUT
+from oracle import moe_oracle as om
+from tests._cases import assert_scaled, make_case, small_shape
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_gives_up_into_the_status_word():
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.selftest_wait_timeout(st, 20_000_000)       # 20 ms
+    torch.cuda.synchronize()
+    assert int(st.item()) & MOE_DEVERR_TIMEOUT
+    # the context is still usable: a layer runs and matches the oracle
+    shape = small_shape("after_timeout", N=300, H=256, E=8, K=2, F=256)
+    c = make_case(shape, seed=41)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F)
+    y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ref = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K)
+    assert_scaled(y, ref["y"], "bf16", "y")
+
+
+def test_padded_rows_beyond_the_buffer_are_reported():
+    H, F, E = 256, 256, 2
+    pb = torch.tensor([256, 640], dtype=torch.int32, device="cuda")   # 640 rows needed
+    P = 512                                                            # buffer holds 512
+    g = torch.Generator(device="cuda").manual_seed(5)
+    x_perm = torch.randn(P, H, generator=g, device="cuda").to(torch.bfloat16)
+    W1 = (torch.randn(E, H, F, generator=g, device="cuda") / 16).to(torch.bfloat16)
+    W3 = (torch.randn(E, H, F, generator=g, device="cuda") / 16).to(torch.bfloat16)
+    W2 = (torch.randn(E, F, H, generator=g, device="cuda") / 16).to(torch.bfloat16)
+    ws = moe.workspace(moe.load().moe_grouped_workspace_size(), "cuda")
+    moe.moe_grouped_swiglu(x_perm, W1, W3, W2, pb, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.device_status(ws) & MOE_DEVERR_ROWS
