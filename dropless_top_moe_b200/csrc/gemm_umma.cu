@@ -297,11 +297,16 @@ __device__ __forceinline__ void router_row(const Params& p, uint32_t tacc, int64
   }
 }
 
+// Shared-memory scratch per epilogue warp for the plain store epilogue: 32
+// rows x 64 bytes (one 32-column chunk of bf16).
+constexpr int kStoreScratch = 32 * 64;
+
 // Epilogue of one 128-row half: TMEM columns [tacc, tacc + BN) of this
-// thread's row -> fused math -> global memory.
+// thread's row -> fused math -> global memory.  scratch: this warp's
+// kStoreScratch bytes of shared memory (EPI_STORE), else 0.
 template <int BN, int SCHED, int EPI>
 __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, uint32_t tacc, int row,
-                                              int part) {
+                                              int part, uint32_t scratch = 0) {
   const int64_t grow = tl.row0 + row;                 // ROWS/DENSE global row
   // the two warps of a lane quarter split the columns: part 0 / part 1
   constexpr int NC = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
@@ -328,16 +333,48 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       }
     }
   } else if constexpr (EPI == EPI_STORE) {
-    __nv_bfloat16* dst = p.out0 + grow * p.ldo + tl.n0;
+    // Each lane holds one row, so storing straight from registers sends 32
+    // rows (32 write requests) per warp store.  Instead the warp's 32 x 32
+    // chunk goes through its shared-memory scratch and leaves as 64-byte row
+    // segments, 4 lanes per row and 8 rows per store.  The scratch keeps a
+    // row's four 16-byte pieces at positions q ^ ((row >> 1) & 3), so both the
+    // writes (a row per lane) and the reads (4 lanes per row) are free of bank
+    // conflicts.
+    const int lane = row & 31;
+    const int64_t row_base = tl.row0 + (row - lane);     // the warp's first row
 #pragma unroll 1
     for (int c = c_begin; c < c_end; c += 32) {
       uint32_t r[32];
       tmem_ld_32(tacc + c, r);
       tmem_ld_wait();
-      float v[32];
+      if (!scratch) {                                     // no scratch: row per lane
+        float v[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-      store_row_bf16x32(dst + c, v);
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        store_row_bf16x32(p.out0 + grow * p.ldo + tl.n0 + c, v);
+        continue;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t a = scratch + (uint32_t)(lane * 64) + ((uint32_t)(q ^ ((lane >> 1) & 3)) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a),
+                     "r"(pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]))),
+                     "r"(pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]))),
+                     "r"(pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]))),
+                     "r"(pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])))
+                     : "memory");
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rr = 8 * i + (lane >> 2), q = lane & 3;
+        const uint32_t a = scratch + (uint32_t)(rr * 64) + ((uint32_t)(q ^ ((rr >> 1) & 3)) << 4);
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+        st_v4(p.out0 + (row_base + rr) * p.ldo + tl.n0 + c + 8 * q, v);
+      }
+      __syncwarp();
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
     const int64_t off = grow * p.ldo + tl.n0;
@@ -504,6 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * S::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int32_t* s_unit_start = reinterpret_cast<int32_t*>(tmem_holder + 4);   // [E + 1]
+  // EPI_STORE: kStoreScratch bytes per epilogue warp, 128-byte aligned
+  const uint32_t store_scratch = (smem_u32(s_unit_start + 260) + 127u) & ~127u;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;          // 0 = leader
@@ -836,7 +875,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           Tile th = tl;
           th.row0 = tl.row0 + 64 * (int)rank;
           th.n0 = tl.n0 + g * (EPI == EPI_SWIGLU ? BN / 4 : BN / 2);
-          epilogue_half<BN / 2, SCHED, EPI>(p, th, tacc, (q & 1) * 32 + lane, part);
+          epilogue_half<BN / 2, SCHED, EPI>(p, th, tacc, (q & 1) * 32 + lane, part,
+                                            EPI == EPI_STORE ? store_scratch + (warp - 2) * kStoreScratch : 0u);
           lone_done = true;
         }
       }
@@ -850,7 +890,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
           Tile th = tl;
           if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + j * BM; else th.row0 = tl.row0 + j * BM;
-          epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part);
+          epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part,
+                                        EPI == EPI_STORE ? store_scratch + (warp - 2) * kStoreScratch : 0u);
         }
       } else {
 #pragma unroll 1
@@ -858,7 +899,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
           Tile th = tl;
           if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + h * BM; else th.row0 = tl.row0 + h * BM;
-          epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part);
+          epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part,
+                                        EPI == EPI_STORE ? store_scratch + (warp - 2) * kStoreScratch : 0u);
         }
       }
       tc_fence_before();
@@ -948,13 +990,14 @@ static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upp
   Params p = p_in;
   if (p.group_m <= 0) p.group_m = S::UNIT >= 4 ? (kGroupM * 2) / S::UNIT : kGroupM;
   auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA>;
+  const size_t smem = S::SMEM + (EPI == EPI_STORE ? (size_t)kEpiWarps * kStoreScratch + 128 : 0);
   // once per device: later calls (a CUDA graph capture among them) only launch
   static bool smem_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (!smem_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM) != cudaSuccess) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
       (void)cudaGetLastError();
       return MOE_ERR_CUDA;
     }
@@ -963,7 +1006,7 @@ static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upp
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = S::SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
