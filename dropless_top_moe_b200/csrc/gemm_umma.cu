@@ -331,6 +331,29 @@ __device__ __forceinline__ void store_chunk_coalesced(uint32_t scratch, int lane
   __syncwarp();
 }
 
+// The reverse for loads: w[i] holds the 16-byte piece (lane & 3) of row
+// 8i + lane / 4 of a 32 x 32 bf16 chunk, read as 64-byte row segments; after
+// the exchange through the warp's scratch, lane i holds row i's 32 values.
+__device__ __forceinline__ void rows_from_coalesced(uint32_t scratch, int lane, const uint4 (&w)[4], float* v) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = 8 * i + (lane >> 2), q = lane & 3;
+    const uint32_t a = scratch + (uint32_t)(rr * 64) + ((uint32_t)(q ^ ((rr >> 1) & 3)) << 4);
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(w[i].x), "r"(w[i].y), "r"(w[i].z),
+                 "r"(w[i].w)
+                 : "memory");
+  }
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t a = scratch + (uint32_t)(lane * 64) + ((uint32_t)(q ^ ((lane >> 1) & 3)) << 4);
+    uint4 u;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(a) : "memory");
+    Vec<__nv_bfloat16>::to_float(u, v + 8 * q);
+  }
+  __syncwarp();
+}
+
 // Epilogue of one 128-row half: TMEM columns [tacc, tacc + BN) of this
 // thread's row -> fused math -> global memory.  scratch: this warp's
 // kStoreScratch bytes of shared memory (EPI_STORE), else 0.
@@ -383,9 +406,24 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       uint32_t r[32];
       tmem_ld_32(tacc + c, r);
       float gf[32], uf[32], dg[32], du[32];
-      load_row_bf16x32(p.aux0 + off + c, gf);
-      load_row_bf16x32(p.aux1 + off + c, uf);
-      tmem_ld_wait();
+      if (scratch) {
+        // G and U as 64-byte row segments, 4 lanes per row (each element is
+        // read here before this warp writes it, so dG, dU may alias G, U)
+        uint4 wg[4], wu[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t o = (row_base + 8 * i + (lane >> 2)) * p.ldo + tl.n0 + c + 8 * (lane & 3);
+          wg[i] = *reinterpret_cast<const uint4*>(p.aux0 + o);
+          wu[i] = *reinterpret_cast<const uint4*>(p.aux1 + o);
+        }
+        tmem_ld_wait();
+        rows_from_coalesced(scratch, lane, wg, gf);
+        rows_from_coalesced(scratch, lane, wu, uf);
+      } else {
+        load_row_bf16x32(p.aux0 + off + c, gf);
+        load_row_bf16x32(p.aux1 + off + c, uf);
+        tmem_ld_wait();
+      }
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float da = __uint_as_float(r[j]);
@@ -551,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   // 2-8 % faster on B200); the SwiGLU epilogues, whose two or three outputs
   // would make as many round trips and which CTA pairs overlap with the
   // main loop anyway, measured up to 4 % slower with it and store directly.
-  constexpr bool kCoalesced = EPI == EPI_STORE || EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR;
+  constexpr bool kCoalesced = EPI == EPI_STORE || EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR || EPI == EPI_SWIGLU_BWD;
   const uint32_t store_scratch = (smem_u32(s_unit_start + 260) + 127u) & ~127u;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1000,7 +1038,7 @@ static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upp
   Params p = p_in;
   if (p.group_m <= 0) p.group_m = S::UNIT >= 4 ? (kGroupM * 2) / S::UNIT : kGroupM;
   auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA>;
-  constexpr bool coalesced = EPI == EPI_STORE || EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR;
+  constexpr bool coalesced = EPI == EPI_STORE || EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR || EPI == EPI_SWIGLU_BWD;
   const size_t smem = S::SMEM + (coalesced ? (size_t)kEpiWarps * kStoreScratch + 128 : 0);
   // once per device: later calls (a CUDA graph capture among them) only launch
   static bool smem_set[64] = {false};
