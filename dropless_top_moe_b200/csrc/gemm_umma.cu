@@ -9,21 +9,28 @@
 // MegaBlocks grouped path copies them to the host; MoonEP sec. 02 argues for
 // static shapes without host sync).
 //
-// One CTA per SM, 6 warps:
-//   warp 0      TMA producer: A and B tiles into a STAGES-deep smem ring
-//   warp 1      TMEM allocator and MMA issuer (one thread): 128 x BN x 16
-//               tcgen05.mma per k-step, fp32 accumulators in TMEM, two
-//               accumulator buffers so the epilogue of tile i overlaps the
-//               main loop of tile i+1
-//   warps 2..5  epilogue: tcgen05.ld rows -> registers -> fused math -> global
+// One CTA (or one CTA pair, cta_group::2) per SM, 10 warps:
+//   warp 0      producer: A and B tiles by TMA into a STAGES-deep smem ring
+//               (optionally A rows gathered from x with tile::gather4)
+//   warp 1      TMEM allocator and MMA issuer (one thread): tcgen05.mma per
+//               16-deep k step, fp32 accumulators in TMEM, double-buffered
+//               where two accumulator sets fit so the epilogue of tile i
+//               overlaps the main loop of tile i+1
+//   warps 2..9  epilogue, two warps per TMEM lane quarter: tcgen05.ld rows ->
+//               registers -> fused math -> global (through a per-warp
+//               shared-memory scratch where that coalesces the accesses)
+// Tile shapes: BN output columns; MT 128-row tiles per CTA; CG = 2 pairs two
+// CTAs on one M = 256 MMA (each CTA holds its 128 rows and half of B's
+// columns); an expert's odd last tile runs as an M = 128 pair MMA.
 // Schedules
 //   ROWS   C[rows of group e, :] = A[rows, :] * B_e   (forward, dgrad)
 //   WGRAD  C_e = A[group e rows, :]^T * B[group e rows, :]   (weight grads;
 //          K = the group's padded rows, zero rows contribute nothing)
-//   DENSE  C = A * B over plain row tiles (router logits)
-// Every accumulation runs in a fixed order (k-steps in sequence, no split-K),
-// so results are bitwise reproducible.  Every wait is bounded (status bit
-// MOE_DEVERR_TIMEOUT); no TMA multicast is used.
+//   DENSE  C = A * B over plain row tiles x column tiles (router logits, the
+//          dense router backward)
+// Every accumulation runs in a fixed order (k-steps in sequence, no split-K
+// across CTAs), so results are bitwise reproducible.  Every wait is bounded
+// (status bit MOE_DEVERR_TIMEOUT); no TMA load uses multicast.
 #include <cuda.h>
 #include <math.h>
 #include <stdlib.h>
