@@ -183,6 +183,19 @@ def recorded_traffic(kernel: str):
     return None
 
 
+def routing_stats(layer, shape):
+    """Load of the last routed batch: per-expert assignment counts (from the
+    layer's inclusive bins), maxvio = max count / mean count - 1, and the
+    padded rows the grouped GEMMs computed."""
+    import numpy as np
+    bins = layer.bins.cpu().numpy().astype(np.int64)
+    counts = np.diff(np.concatenate([[0], bins]))
+    mean = counts.sum() / max(shape.E, 1)
+    return {"min_count": int(counts.min()), "max_count": int(counts.max()),
+            "maxvio": round(float(counts.max() / mean - 1.0), 3) if mean > 0 else None,
+            "assignments": int(counts.sum()), "padded_rows": int(layer.padded_bins[-1].item())}
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -325,6 +338,7 @@ def run_ours(args, rank, world, local_rank):
                                "capacity": capacity or "dropless"},
                    "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
                          (3 * shape.E * shape.H * shape.F * 2 / 1e9)},
+        "routing": routing_stats(layer, shape),
         "tflops": round((layer_flops(work) - (2 * work.N * work.H * work.E) * (3 if shape.training else 1)
                          + (2 * shape.N * shape.H * shape.E) * (3 if shape.training else 1))
                         / (ms_max * 1e-3) / 1e12, 1),
