@@ -161,9 +161,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- traffic
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, only while the
-    kernel's source is unchanged since the capture (else None)."""
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, only while the kernel's source is unchanged since the capture
+    (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -172,9 +173,9 @@ def recorded_traffic(kernel: str):
         if line.startswith("#") or not line.strip():
             continue
         parts = line.split()
-        if len(parts) < 4 or parts[0] != kernel:
+        if len(parts) < 5 or parts[0] != kernel or parts[1] != workload:
             continue
-        bytes_, fname, sha = float(parts[1]), parts[2], parts[3]
+        bytes_, fname, sha = float(parts[2]), parts[3], parts[4]
         try:
             cur = hashlib.sha256(open(os.path.join(src, fname), "rb").read()).hexdigest()[:16]
         except OSError:
@@ -323,7 +324,9 @@ def run_ours(args, rank, world, local_rank):
         achieved = by.get(dom, 0) / dom_avg_s / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} copy bandwidth"}
-    tr = recorded_traffic(dom)
+    default_variant = args.aux_alpha == 0 and args.capacity_factor == 0 and args.train_mode == 1
+    # the capture is of the named workload's default variant only
+    tr = recorded_traffic(dom, shape.name) if default_variant else None
     roof["traffic"] = tr
 
     result = {
