@@ -122,3 +122,20 @@ def test_selftest_rejects_bad_arguments(lib):
     assert lib.moe_selftest_wait_timeout(None, 1000000, None) == MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_wait_timeout(FAKE, 10, None) == MOE_ERR_INVALID_ARG            # < 1 us
     assert lib.moe_selftest_wait_timeout(FAKE, 5 * 10 ** 9, None) == MOE_ERR_INVALID_ARG   # > 1 s
+
+
+def test_header_and_c_example_compile_as_c99():
+    """include/moe.h is plain C: the C caller in tests/c_api compiles as C99
+    (syntax and types only; running it needs a GPU)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    if not os.path.exists(os.path.join(cuda, "include", "cuda_runtime.h")):
+        pytest.skip("no CUDA headers")
+    res = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-fsyntax-only",
+                          "-I", os.path.join(ROOT, "include"), "-I", os.path.join(cuda, "include"),
+                          os.path.join(ROOT, "tests", "c_api", "layer_fwd.c")], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
