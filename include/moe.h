@@ -184,7 +184,9 @@ moe_status moe_permute(const void* x, const int32_t* pos, const int32_t* bins,
  * padded_bins[e]) use expert e:
  *   G = X W1_e, U = X W3_e, act = silu(G) * U, out = act W2_e
  * (LLaMA MoE tutorial sec. 2.1; icman sec. 2.3).  fp32 accumulation; act and
- * out are rounded once to dt.  P = rows of x_perm/act/out (multiple of 128).
+ * out are rounded once to dt.  P = rows of x_perm/act/out (multiple of 128);
+ * groups reaching past row P are computed only up to P, and the tensor-core
+ * (bf16) path then sets MOE_DEVERR_ROWS in the workspace's status word. 
  *   x_perm [P,H]; W1, W3 [E,H,F]; W2 [E,F,H]; act [P,F]; out [P,H];
  *   gate_up: NULL, or [2,P,F] receiving G then U (dt) for the backward pass. */
 moe_status moe_grouped_swiglu(const void* x_perm, const void* W1, const void* W3, const void* W2,
