@@ -1,0 +1,58 @@
+"""Layer parity over a seeded sweep of unusual shapes (GPU only).
+
+Shapes the fixed cases do not reach: H or F not multiples of 256 (the
+128-column tile paths), a single token, odd expert counts, K from 1 to E,
+ragged N.  Forward and backward against the float64 oracle, at the stated
+tolerances; integer routing outputs bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dropless_top_moe_b200 as moe
+from oracle import moe_oracle as om
+from tests._cases import assert_scaled, make_case, small_shape
+
+pytestmark = pytest.mark.gpu
+
+
+def _sweep(n_cases=14, seed=2024):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n_cases):
+        dtype = "bf16" if i % 4 else "f32"
+        if dtype == "bf16":
+            H = int(rng.choice([128, 256, 384, 512, 640]))
+            F = int(rng.choice([128, 256, 384, 512]))
+            E = int(rng.choice([1, 2, 3, 5, 8, 16, 33, 64, 100, 256]))
+        else:
+            H = int(rng.choice([32, 64, 96, 128]))
+            F = int(rng.choice([32, 48, 96, 128]))
+            E = int(rng.choice([1, 2, 3, 5, 8, 16]))
+        K = int(rng.integers(1, min(E, 8) + 1))
+        N = int(rng.choice([1, 7, 129, 333, 700]))
+        cases.append(small_shape(f"sweep{i}_{dtype}_N{N}_H{H}_E{E}_K{K}_F{F}", N=N, H=H, E=E, K=K, F=F,
+                                 dtype=dtype, training=True))
+    return cases
+
+
+@pytest.mark.parametrize("shape", _sweep(), ids=lambda s: s.name)
+def test_layer_shape_sweep(shape):
+    c = make_case(shape, seed=71, with_dy=True)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype, training=True)
+    y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"]).clone()
+    g = layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    np.testing.assert_array_equal(layer.top_experts.cpu().numpy(), ref["top_experts"])
+    m = om.dispatch_meta(ref["top_experts"], shape.E)
+    np.testing.assert_array_equal(layer.bins.cpu().numpy(), m["bins"])
+    np.testing.assert_array_equal(layer.padded_bins.cpu().numpy(), m["padded_bins"])
+    np.testing.assert_array_equal(layer.indices.cpu().numpy(), m["indices"])
+    W1, W3, W2 = c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu()
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], W1, W3, W2, shape.K, routing=ref)["y"]
+    assert_scaled(y, yr, shape.dtype, "y")
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], W1, W3, W2, shape.K, c["dy"].cpu(), routing=ref)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(g[k], gr[k], shape.dtype, k)
