@@ -55,4 +55,10 @@ def test_layer_shape_sweep(shape):
     assert_scaled(y, yr, shape.dtype, "y")
     gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], W1, W3, W2, shape.K, c["dy"].cpu(), routing=ref)
     for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        if k == "dW_r" and shape.K == 1:
+            # K = 1: the renormalised weight is exactly 1 whatever the logits,
+            # so the router receives no gradient (the oracle shows rounding noise)
+            assert int(torch.count_nonzero(g[k])) == 0
+            assert np.abs(gr[k]).max() < 1e-10
+            continue
         assert_scaled(g[k], gr[k], shape.dtype, k)
