@@ -12,7 +12,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
 MOE_F32, MOE_BF16 = 0, 1
-MOE_DEVERR_EXPERT_ID, MOE_DEVERR_TIMEOUT, MOE_DEVERR_ROWS = 1, 2, 4
+MOE_DEVERR_EXPERT_ID, MOE_DEVERR_TIMEOUT, MOE_DEVERR_ROWS, MOE_DEVERR_MODE = 1, 2, 4, 8
 MOE_LAYER_GATHER_ROWS = 4   # flag OR-ed into the layer's training mode
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA"}

@@ -65,6 +65,19 @@ bool layer_flags_ok(int32_t training, moe_dtype dt) {
   return !(training & MOE_LAYER_GATHER_ROWS) || dt == MOE_BF16;
 }
 
+// Word 1 of the status region records the layout-deciding flags of the last
+// layer forward on the workspace (mode, row gather, aux loss on, token
+// dropping on) as one non-zero byte repeated four times.  The backward reads
+// buffers the forward wrote at offsets these flags decide, so it compares the
+// record with its own flags first; moe_workspace_init clears the record.
+int layer_stamp_byte(int32_t flags, float aux_alpha, int32_t capacity) {
+  return 1 + (flags & 7) + (aux_alpha != 0.0f ? 8 : 0) + (capacity > 0 ? 16 : 0);
+}
+
+__global__ void layer_stamp_check_kernel(int* status, int expect) {
+  if (threadIdx.x == 0 && status[1] != expect) atomicOr(status, MOE_DEVERR_MODE);
+}
+
 LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int flags) {
   const int training = flags & 3;
   const bool gather = (flags & MOE_LAYER_GATHER_ROWS) != 0;
@@ -332,10 +345,15 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
   cudaStream_t s = (cudaStream_t)stream;
   LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
+  const int32_t flags = training;
   const bool gather = (training & MOE_LAYER_GATHER_ROWS) != 0;
   training &= 3;
   const bool aux = aux_alpha != 0.0f;
   if ((aux && !aux_loss) || capacity < 0) return MOE_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(w.status + 1, layer_stamp_byte(flags, aux_alpha, capacity), 4, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
   MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, aux ? w.probs : nullptr, top_experts, weights,
                     w.route_scratch, w.status, s));
   MOE_TRY(dispatch_meta(top_experts, (int64_t)N * K, E, indices, nullptr, bins, padded_bins, w.pos,
@@ -383,6 +401,9 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
   LayerWs w = carve(ws, N, H, E, K, F, dt, training);
   const int64_t P = p_max(N, E, K);
   const RowGather ga = {x, indices, bins, N, K};
+  const uint32_t stamp = (uint32_t)layer_stamp_byte(training, aux_alpha, capacity) * 0x01010101u;
+  MOE_TRACED("layer_flags_check", s, (layer_stamp_check_kernel<<<1, 32, 0, s>>>(w.status, (int)stamp)));
+  MOE_LAUNCH_CHECK();
   const bool gather = (training & MOE_LAYER_GATHER_ROWS) != 0;
   training &= 3;
   void* gate_up = w.gate_up;

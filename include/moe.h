@@ -64,10 +64,15 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
-/* Bits of the device status word (first 4 bytes of every workspace). */
+/* Bits of the device status word (first 4 bytes of every workspace; the
+ * layer calls keep a record of the forward's flags in the next 4). */
 #define MOE_DEVERR_EXPERT_ID 0x1   /* a top_experts entry was outside [0,E) */
 #define MOE_DEVERR_TIMEOUT 0x2     /* a bounded pipeline wait gave up */
 #define MOE_DEVERR_ROWS 0x4        /* padded rows exceeded the buffer's rows */
+#define MOE_DEVERR_MODE 0x8        /* moe_layer_bwd's training flags, aux loss (on/off) or token
+                                      dropping (on/off) differ from those of the last
+                                      moe_layer_fwd on this workspace: its outputs are
+                                      meaningless */
 
 /* The caller's cudaStream_t. */
 typedef struct CUstream_st* moe_stream_t;
@@ -283,12 +288,15 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
                          int32_t* top_experts, float* weights, int32_t* indices, int32_t* bins,
                          int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Whole layer backward for the forward run last with this workspace
+/* Whole layer backward for the forward run last with this workspace (which
+ * must have run: the backward reads the token positions it wrote)
  * (training 1 or 2, the forward's value; with 2 the gate and up projections
  * G, U are recomputed here by the forward's own GEMM kernel, bit-identical).  dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F],
  * dW2 [E,F,H], all dt, overwritten.  capacity and aux_alpha must equal the
  * forward's (dropped pairs still pass gradient to the router through the
- * renormalised weights);
+ * renormalised weights); a backward whose training flags, aux loss on/off or
+ * token dropping on/off differ from the forward's sets MOE_DEVERR_MODE (one
+ * 32-thread check kernel, first on the stream);
  * when non-zero, aux_grad = dObjective/dL_aux scales the load-balancing
  * loss's gradient, which is added to the router's (dense router backward). */
 moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const void* W1,

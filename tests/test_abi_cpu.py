@@ -22,6 +22,17 @@ def declared_functions():
                                  text, flags=re.M)))
 
 
+def test_binding_constants_match_the_header():
+    text = open(HEADER).read()
+    defines = {m.group(1): int(m.group(2), 0)
+               for m in re.finditer(r"^#define\s+(MOE_\w+)\s+(0x[0-9a-fA-F]+|\d+)", text, flags=re.M)}
+    for name in ("MOE_DEVERR_EXPERT_ID", "MOE_DEVERR_TIMEOUT", "MOE_DEVERR_ROWS", "MOE_DEVERR_MODE",
+                 "MOE_LAYER_GATHER_ROWS"):
+        assert getattr(_lib, name) == defines[name], name
+    bits = [defines[n] for n in defines if n.startswith("MOE_DEVERR_")]
+    assert len(bits) == len(set(bits)) == 4 and all(b & (b - 1) == 0 for b in bits)
+
+
 @pytest.fixture(scope="module")
 def lib():
     from dropless_top_moe_b200.build import build

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import dropless_top_moe_b200 as moe
-from dropless_top_moe_b200._lib import MOE_DEVERR_ROWS, MOE_DEVERR_TIMEOUT
+from dropless_top_moe_b200._lib import MOE_DEVERR_MODE, MOE_DEVERR_ROWS, MOE_DEVERR_TIMEOUT
 from oracle import moe_oracle as om
 from tests._cases import assert_scaled, make_case, small_shape
 
@@ -46,3 +46,23 @@ def test_padded_rows_beyond_the_buffer_are_reported():
     moe.moe_grouped_swiglu(x_perm, W1, W3, W2, pb, ws=ws)
     torch.cuda.synchronize()
     assert moe.device_status(ws) & MOE_DEVERR_ROWS
+
+
+def test_backward_flags_unlike_the_forward_are_reported():
+    # The backward reads buffers the forward wrote at offsets that the
+    # training flags decide.  Both mismatches below keep every access inside
+    # the workspace (the token positions sit at the same offset in every
+    # layout); the check turns what would be silent garbage into a status bit.
+    shape = small_shape("flags_mismatch", N=300, H=256, E=8, K=2, F=256, training=True)
+    c = make_case(shape, seed=43, with_dy=True)
+    args = (c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+    for fwd_mode, bwd_mode in ((1, 2), (1, 1 | moe.MOE_LAYER_GATHER_ROWS)):
+        layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, training=fwd_mode)
+        layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"])
+        layer.backward(*args)
+        torch.cuda.synchronize()
+        assert layer.status() == 0
+        layer.mode = bwd_mode        # workspace sized for fwd_mode: large enough for bwd_mode
+        layer.backward(*args)
+        torch.cuda.synchronize()
+        assert layer.status() & MOE_DEVERR_MODE, (fwd_mode, bwd_mode)
