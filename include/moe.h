@@ -33,8 +33,9 @@
  *   - The return value reports host-detectable errors only (shapes, dtype,
  *     alignment, workspace size).  Errors found on the device (an expert id
  *     outside [0,E), a padded-row count above the buffer, a bounded wait that
- *     gave up) are OR-ed into the 32-bit status word at the start of the
- *     workspace; read it with moe_get_device_status.  Kernels never trap.
+ *     gave up, a layer backward whose flags differ from the forward's) are
+ *     OR-ed into the 32-bit status word at the start of the workspace; read
+ *     it with moe_get_device_status.  Kernels never trap.
  *   - Outputs are overwritten, never accumulated into.
  *   - Results are bitwise identical from run to run for identical inputs:
  *     no floating-point atomics, every reduction has a fixed order.
@@ -273,7 +274,8 @@ moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int3
 /* Whole layer forward: route -> dispatch_meta -> permute -> grouped SwiGLU
  * -> combine, all on `stream`, no host synchronisation.
  *   y [N,H] (dt); top_experts [N,K]; weights [N,K]; indices [N*K];
- *   bins, padded_bins [E] (all outputs required).
+ *   bins, padded_bins [E] (all required; with N = 0 the token-sized ones
+ *   may be NULL).
  *   capacity: 0 = dropless; > 0 = token-dropping variant (see
  *   moe_dispatch_meta): dropped (token, expert) pairs add nothing to y.
  *   aux_alpha != 0 also computes the load-balancing loss into *aux_loss (a
@@ -288,17 +290,23 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
                          int32_t* top_experts, float* weights, int32_t* indices, int32_t* bins,
                          int32_t* padded_bins, void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Whole layer backward for the forward run last with this workspace (which
- * must have run: the backward reads the token positions it wrote)
- * (training 1 or 2, the forward's value; with 2 the gate and up projections
- * G, U are recomputed here by the forward's own GEMM kernel, bit-identical).  dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F],
- * dW2 [E,F,H], all dt, overwritten.  capacity and aux_alpha must equal the
- * forward's (dropped pairs still pass gradient to the router through the
- * renormalised weights); a backward whose training flags, aux loss on/off or
- * token dropping on/off differ from the forward's sets MOE_DEVERR_MODE (one
- * 32-thread check kernel, first on the stream);
- * when non-zero, aux_grad = dObjective/dL_aux scales the load-balancing
- * loss's gradient, which is added to the router's (dense router backward). */
+/* Whole layer backward of the forward run last on this workspace (the
+ * forward must have run: the backward reads the token positions, the expert
+ * outputs and the activations it left there).
+ *   training: 1 or 2, the forward's value (with 2, G and U are recomputed
+ *   here by the forward's own GEMM kernel, bit-identical).
+ *   dy [N,H]; outputs dx [N,H], dW_r [H,E], dW1, dW3 [E,H,F], dW2 [E,F,H],
+ *   all dt, overwritten.  top_experts, weights, indices, bins, padded_bins:
+ *   the forward's outputs, unchanged.
+ *   capacity and aux_alpha must equal the forward's (dropped pairs still pass
+ *   gradient to the router through the renormalised weights).  A backward
+ *   whose training flags, aux loss on/off or token dropping on/off differ
+ *   from the forward's sets MOE_DEVERR_MODE (one 32-thread check kernel,
+ *   first on the stream).
+ *   aux_grad (used when aux_alpha != 0) = dObjective/dL_aux scales the
+ *   load-balancing loss's gradient, which is added to the router's (dense
+ *   router backward).
+ *   N = 0: the token arrays may be NULL and the weight gradients are zeroed. */
 moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const void* W1,
                          const void* W3, const void* W2, const int32_t* top_experts,
                          const float* weights, const int32_t* indices, const int32_t* bins,
