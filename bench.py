@@ -98,6 +98,56 @@ def bytes_by_kernel(s, padded_rows):
             "meta_count": N * K * 4, "meta_place": N * K * 4 * 3}
 
 
+def kernel_rooflines(per, steps, timed_ms, fl, by, peaks):
+    """Per-kernel figures over the timed region and stage totals.
+
+    per: kernel -> (total ms, launches) from the CUDA events; timed_ms: the
+    whole timed region (a kernel's share is of that); fl / by: the
+    algorithmic FLOPs / HBM bytes per launch.  Each kernel with a work model
+    gets its achieved rate and the fraction of the roof it meets first: the
+    sustained bf16 tensor peak or the HBM copy bandwidth (both measured; a
+    kernel with both models, the router, is judged by its arithmetic
+    intensity against the ridge).  Stage totals: the grouped GEMMs against
+    the tensor peak, the bandwidth-bound row kernels against HBM, and the
+    dispatch metadata (latency-bound) in microseconds per step."""
+    tensor_peak, hbm_peak = peaks["bf16_tflops_sustained"], peaks["hbm_gbs"]
+    ridge = tensor_peak * 1e12 / (hbm_peak * 1e9)          # FLOP per byte
+    kernels = {}
+    for name, (tot, n) in per.items():
+        avg_s = tot / n * 1e-3
+        k = {"launches": n, "ms_avg": round(tot / n, 4), "share": round(tot / timed_ms, 4)}
+        if name in fl:
+            k["tflops"] = round(fl[name] / avg_s / 1e12, 1)
+        if name in by:
+            k["gbs"] = round(by[name] / avg_s / 1e9, 1)
+        if name in fl and (name not in by or fl[name] / by[name] >= ridge):
+            k["bound"], k["frac"] = "tensor", round(fl[name] / avg_s / 1e12 / tensor_peak, 4)
+        elif name in by:
+            k["bound"], k["frac"] = "hbm", round(by[name] / avg_s / 1e9 / hbm_peak, 4)
+        kernels[name] = k
+
+    def total(names, work):
+        t = sum(per[n][0] for n in names) * 1e-3
+        w = sum(work[n] * per[n][1] for n in names)
+        return w / t if t > 0 else 0.0
+
+    gemms = [n for n in per if n in fl and n not in by]
+    rows = [n for n in per if n in by and n not in fl and not n.startswith("meta_")]
+    meta = [n for n in per if n.startswith("meta_")]
+    stages = {}
+    if gemms:
+        r = total(gemms, fl) / 1e12
+        stages["grouped_gemms"] = {"kernels": sorted(gemms), "tflops": round(r, 1),
+                                   "frac": round(r / tensor_peak, 4)}
+    if rows:
+        r = total(rows, by) / 1e9
+        stages["bandwidth_kernels"] = {"kernels": sorted(rows), "gbs": round(r, 1),
+                                       "frac": round(r / hbm_peak, 4)}
+    if meta:
+        stages["metadata_us_per_step"] = round(sum(per[n][0] for n in meta) / steps * 1e3, 2)
+    return kernels, stages
+
+
 def step_tokens(s):
     return s.N
 
@@ -301,16 +351,9 @@ def run_ours(args, rank, world, local_rank):
     fl = flops_by_kernel(work)
     fl["route_umma"] = 2 * shape.N * shape.H * shape.E
     by = bytes_by_kernel(shape, padded_rows)
+    by["route_umma"] = by["route_simt"]
     peaks, peak_src = load_peaks()
-    kernels = {}
-    for name, (tot, n) in per.items():
-        avg = tot / n
-        k = {"launches": n, "ms_avg": round(avg, 4), "share": round(tot / (ms * steps), 4)}
-        if name in fl:
-            k["tflops"] = round(fl[name] / (avg * 1e-3) / 1e12, 1)
-        elif name in by:
-            k["gbs"] = round(by[name] / (avg * 1e-3) / 1e9, 1)
-        kernels[name] = k
+    kernels, stages = kernel_rooflines(per, steps, ms * steps, fl, by, peaks)
     dom = max(per, key=lambda n: per[n][0])
     dom_avg_s = per[dom][0] / per[dom][1] * 1e-3
     if dom in fl:
@@ -345,7 +388,7 @@ def run_ours(args, rank, world, local_rank):
         "tflops": round((layer_flops(work) - (2 * work.N * work.H * work.E) * (3 if shape.training else 1)
                          + (2 * shape.N * shape.H * shape.E) * (3 if shape.training else 1))
                         / (ms_max * 1e-3) / 1e12, 1),
-        "roofline": roof, "kernels": kernels, "gpu_launches": count.value,
+        "roofline": roof, "stages": stages, "kernels": kernels, "gpu_launches": count.value,
         "launches_per_step": per_step, "device_status": status, "clocks": clk,
     }
     result["value"] = round(shape.N * world / (ms_max * 1e-3), 1)

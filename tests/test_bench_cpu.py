@@ -33,3 +33,26 @@ def test_reference_arm_other_ranks_print_nothing():
                          capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert res.returncode == 0, res.stderr
     assert res.stdout.strip() == ""
+
+
+def test_kernel_rooflines_fractions_and_stage_totals():
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops_sustained": 1000.0, "hbm_gbs": 5000.0}      # ridge: 200 FLOP per byte
+    fl = {"gemm_a": 2e12, "gemm_b": 1e12, "router": 1e9}
+    by = {"router": 1e8, "rows": 5e9, "meta_x": 1e6}
+    # (total ms, launches) over 2 steps
+    per = {"gemm_a": (8.0, 2), "gemm_b": (2.0, 2), "router": (0.1, 2), "rows": (2.0, 2),
+           "meta_x": (0.02, 2), "other": (0.5, 2)}
+    k, st = bench.kernel_rooflines(per, 2, 20.0, fl, by, peaks)
+    assert k["gemm_a"]["tflops"] == 500.0 and k["gemm_a"]["bound"] == "tensor" and k["gemm_a"]["frac"] == 0.5
+    assert k["gemm_b"]["frac"] == 1.0
+    # router: 10 FLOP per byte, below the ridge, so judged against HBM: 1e8 B in 50 us = 2000 GB/s
+    assert k["router"]["bound"] == "hbm" and k["router"]["gbs"] == 2000.0 and k["router"]["frac"] == 0.4
+    assert k["rows"]["gbs"] == 5000.0 and k["rows"]["frac"] == 1.0
+    assert "frac" not in k["other"] and k["other"]["share"] == 0.025
+    # stage totals weight each kernel by its time: (2*2e12 + 2*1e12) FLOP in 10 ms
+    assert st["grouped_gemms"]["kernels"] == ["gemm_a", "gemm_b"]
+    assert st["grouped_gemms"]["tflops"] == 600.0 and st["grouped_gemms"]["frac"] == 0.6
+    assert st["bandwidth_kernels"] == {"kernels": ["rows"], "gbs": 5000.0, "frac": 1.0}
+    assert st["metadata_us_per_step"] == 10.0
