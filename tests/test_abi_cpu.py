@@ -129,6 +129,76 @@ def test_meta_and_grouped_reject_bad_arguments(lib):
                                   None, FAKE, 4096, None) == MOE_ERR_INVALID_ARG
 
 
+def test_stage_entry_points_reject_bad_arguments(lib):
+    INV, UNS, WS = MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE
+    big = 1 << 40
+    # permute: x pos bins padded_bins N H E K dt x_perm
+    assert lib.moe_permute(FAKE, FAKE, FAKE, FAKE, 16, 128, 4, 5, MOE_BF16, FAKE, None) == INV      # K > E
+    assert lib.moe_permute(FAKE, FAKE, FAKE, FAKE, 16, 128, 4, 2, MOE_BF16, None, None) == INV
+    assert lib.moe_permute(FAKE + 4, FAKE, FAKE, FAKE, 16, 128, 4, 2, MOE_BF16, FAKE, None) == INV
+    assert lib.moe_permute(FAKE, FAKE, FAKE, FAKE, 16, 96, 4, 2, MOE_BF16, FAKE, None) == UNS        # H % 128
+    # combine: out weights pos N K H dt y (an empty batch returns before any device work)
+    assert lib.moe_combine(None, FAKE, FAKE, 16, 2, 128, MOE_BF16, FAKE, None) == INV
+    assert lib.moe_combine(FAKE, FAKE, FAKE, 16, 2, 128, MOE_BF16, FAKE + 8, None) == INV
+    assert lib.moe_combine(None, None, None, 0, 2, 128, MOE_BF16, None, None) == 0
+    # combine_bwd: dy out weights pos bins padded_bins N K H E dt dw dlogit d_out
+    assert lib.moe_combine_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 2, 128, 4, MOE_BF16, None, None,
+                               FAKE, None) == INV                                               # no dlogit
+    assert lib.moe_combine_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, 2, 128, 4, MOE_BF16, None, FAKE,
+                               None, None) == INV                                               # no d_out
+    # grouped SwiGLU backward: 7 inputs, padded_bins, E H F P dt, 5 outputs, ws
+    g = [FAKE] * 7 + [FAKE, 4, 128, 256]
+    out = [FAKE] * 5
+    assert lib.moe_grouped_swiglu_bwd(*g, 100, MOE_BF16, *out, FAKE, big, None) == INV          # P % 128
+    assert lib.moe_grouped_swiglu_bwd(*g, 128, MOE_BF16, *out[:4], None, FAKE, big, None) == INV
+    assert lib.moe_grouped_swiglu_bwd(*g, 128, MOE_BF16, *out, FAKE, 16, None) == WS
+    assert lib.moe_grouped_swiglu_bwd(*g[:9], 200, 256, 128, MOE_BF16, *out, FAKE, big, None) == UNS
+    # unpermute + router backward: 9 pointers, probs, aux_alpha aux_grad, N H E K P dt, dx dW_r, ws
+    u = [FAKE] * 9
+    assert lib.moe_unpermute_router_bwd(*u, None, 0.5, 1.0, 16, 128, 4, 2, 256, MOE_BF16, FAKE, FAKE,
+                                        FAKE, big, None) == INV                                 # aux without probs
+    assert lib.moe_unpermute_router_bwd(*u, None, 0.0, 1.0, 16, 128, 4, 2, 256, MOE_BF16, FAKE, FAKE,
+                                        FAKE, 64, None) == WS
+    assert lib.moe_unpermute_router_bwd(*u, None, 0.0, 1.0, 16, 128, 4, 2, 200, MOE_BF16, FAKE, FAKE,
+                                        FAKE, big, None) == INV                                 # P % 128
+    # aux loss: probs bins N K E alpha loss P ws
+    assert lib.moe_aux_loss(FAKE, FAKE, 16, 5, 4, 0.01, FAKE, None, FAKE, big, None) == INV      # K > E
+    assert lib.moe_aux_loss(FAKE, FAKE, 16, 2, 300, 0.01, FAKE, None, FAKE, big, None) == UNS
+    assert lib.moe_aux_loss(FAKE, FAKE, 16, 2, 4, 0.01, None, None, FAKE, big, None) == INV     # no loss
+    assert lib.moe_aux_loss(FAKE, FAKE, 16, 2, 4, 0.01, FAKE, None, FAKE, 8, None) == WS
+    # rank-ordered sum: shards n_ranks numel dt scale out
+    assert lib.moe_sum_rank_ordered(FAKE, 0, 64, MOE_BF16, 1.0, FAKE, None) == INV
+    assert lib.moe_sum_rank_ordered(FAKE, 2, 64, 7, 1.0, FAKE, None) == INV                     # unknown dtype
+    assert lib.moe_sum_rank_ordered(FAKE + 4, 2, 64, MOE_BF16, 1.0, FAKE, None) == INV
+    assert lib.moe_sum_rank_ordered(FAKE, 2, 12, MOE_BF16, 1.0, FAKE, None) == UNS              # 12 % 8
+    assert lib.moe_sum_rank_ordered(FAKE, 2, 0, MOE_BF16, 1.0, FAKE, None) == 0
+    # dispatch metadata without allocation: the fixed scratch bounds N*K
+    assert lib.moe_dispatch_meta_noalloc(FAKE, 16, 5, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == INV
+    assert lib.moe_dispatch_meta_noalloc(FAKE, 16, 2, 300, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == UNS
+    assert lib.moe_dispatch_meta_noalloc(FAKE, 16, 2, 4, FAKE, FAKE, FAKE, None, FAKE, None, None) == INV
+    assert lib.moe_dispatch_meta_noalloc(FAKE, 1000000, 2, 256, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                         None) == WS
+    # tracing
+    assert lib.moe_trace_attach(None, 4, None, FAKE) == INV
+    assert lib.moe_trace_attach(FAKE, 0, None, FAKE) == INV
+
+
+def test_layer_backward_rejects_bad_flags(lib):
+    G = _lib.MOE_LAYER_GATHER_ROWS
+    # 11 pointers | N H E K F dt training capacity aux_alpha aux_grad | dx dW_r dW1 dW3 dW2
+    def bwd(training, dt=MOE_BF16, ws_bytes=1 << 40):
+        return lib.moe_layer_bwd(*([FAKE] * 11), 64, 128, 4, 2, 256, dt, training, 0, 0.0, 1.0,
+                                 *([FAKE] * 5), FAKE, ws_bytes, None)
+    assert bwd(0) == MOE_ERR_INVALID_ARG                 # a forward-only layer has no backward
+    assert bwd(3) == MOE_ERR_INVALID_ARG
+    assert bwd(1 | 8) == MOE_ERR_INVALID_ARG             # unknown flag bit
+    assert bwd(1 | G, dt=MOE_F32) == MOE_ERR_INVALID_ARG  # row gathers are bf16 only
+    assert bwd(1, ws_bytes=1024) == MOE_ERR_WORKSPACE
+    for bad in (3, 8, 1 | 8):
+        assert lib.moe_workspace_size(64, 128, 4, 2, 256, MOE_BF16, bad) == 0
+    assert lib.moe_workspace_size(64, 128, 4, 2, 256, MOE_F32, 1 | G) == 0
+
+
 def test_selftest_rejects_bad_arguments(lib):
     assert lib.moe_selftest_wait_timeout(None, 1000000, None) == MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_wait_timeout(FAKE, 10, None) == MOE_ERR_INVALID_ARG            # < 1 us
