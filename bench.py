@@ -94,7 +94,9 @@ def bytes_by_kernel(s, padded_rows):
             "combine": N * K * H * b + N * K * 8 + N * H * b,
             "combine_bwd": N * H * b + N * K * H * b + padded_rows * H * b + N * K * 12,
             "unpermute_dx": N * K * H * b + N * H * b + N * K * 12,
-            "router_wgrad_partial": N * K * H * b + N * K * 8,
+            # x is needed once per token; the kernel gathers it once per
+            # assignment (K times, the repeats mostly from L2)
+            "router_wgrad_partial": N * H * b + N * K * 8 + (padded_rows // 128) * H * 4,
             "meta_count": N * K * 4, "meta_place": N * K * 4 * 3}
 
 
@@ -107,7 +109,8 @@ def kernel_rooflines(per, steps, timed_ms, fl, by, peaks):
     gets its achieved rate and the fraction of the roof it meets first: the
     sustained bf16 tensor peak or the HBM copy bandwidth (both measured; a
     kernel with both models, the router, is judged by its arithmetic
-    intensity against the ridge).  Stage totals: the grouped GEMMs against
+    intensity against the ridge; the dispatch metadata, a few hundred KB,
+    is latency-bound and gets no fraction).  Stage totals: the grouped GEMMs against
     the tensor peak, the bandwidth-bound row kernels against HBM, and the
     dispatch metadata (latency-bound) in microseconds per step."""
     tensor_peak, hbm_peak = peaks["bf16_tflops_sustained"], peaks["hbm_gbs"]
@@ -120,7 +123,9 @@ def kernel_rooflines(per, steps, timed_ms, fl, by, peaks):
             k["tflops"] = round(fl[name] / avg_s / 1e12, 1)
         if name in by:
             k["gbs"] = round(by[name] / avg_s / 1e9, 1)
-        if name in fl and (name not in by or fl[name] / by[name] >= ridge):
+        if name.startswith("meta_"):
+            k["bound"] = "latency"                        # a few hundred KB per launch
+        elif name in fl and (name not in by or fl[name] / by[name] >= ridge):
             k["bound"], k["frac"] = "tensor", round(fl[name] / avg_s / 1e12 / tensor_peak, 4)
         elif name in by:
             k["bound"], k["frac"] = "hbm", round(by[name] / avg_s / 1e9 / hbm_peak, 4)

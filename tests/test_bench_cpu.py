@@ -51,6 +51,7 @@ def test_kernel_rooflines_fractions_and_stage_totals():
     assert k["router"]["bound"] == "hbm" and k["router"]["gbs"] == 2000.0 and k["router"]["frac"] == 0.4
     assert k["rows"]["gbs"] == 5000.0 and k["rows"]["frac"] == 1.0
     assert "frac" not in k["other"] and k["other"]["share"] == 0.025
+    assert k["meta_x"]["bound"] == "latency" and "frac" not in k["meta_x"]
     # stage totals weight each kernel by its time: (2*2e12 + 2*1e12) FLOP in 10 ms
     assert st["grouped_gemms"]["kernels"] == ["gemm_a", "gemm_b"]
     assert st["grouped_gemms"]["tflops"] == 600.0 and st["grouped_gemms"]["frac"] == 0.6
