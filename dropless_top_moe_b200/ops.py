@@ -33,6 +33,32 @@ def _p(t: Optional[torch.Tensor]):
     return t.data_ptr()
 
 
+def _check(name: str, t: Optional[torch.Tensor], shape=None, dtype=None, numel=None):
+    """Shape and dtype of an argument against the sizes the call derives from
+    the others.  The library reads and writes through raw pointers with those
+    sizes, so a mismatched tensor would be read or written out of bounds;
+    it is refused here instead."""
+    if t is None:
+        return
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: expected {numel} elements, got {t.numel()}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+
+
+def _experts(W1, W3, W2, H: int, dtype):
+    """E, F of the stacked expert weights W1, W3 [E,H,F] and W2 [E,F,H]."""
+    if W1.dim() != 3:
+        raise ValueError(f"W1: expected [E, H, F], got {tuple(W1.shape)}")
+    E, _, F = W1.shape
+    _check("W1", W1, (E, H, F), dtype)
+    _check("W3", W3, (E, H, F), dtype)
+    _check("W2", W2, (E, F, H), dtype)
+    return E, F
+
+
 def _stream():
     return torch.cuda.current_stream().cuda_stream
 
@@ -62,6 +88,7 @@ def device_status(ws: torch.Tensor) -> int:
 def moe_route(x, W_r, K: int, want_logits: bool = False, want_probs: bool = False, ws=None) -> dict:
     N, H = x.shape
     E = W_r.shape[1]
+    _check("W_r", W_r, (H, E), x.dtype)
     dev = x.device
     dt = _dt(x)
     if ws is None:
@@ -80,6 +107,7 @@ def moe_route(x, W_r, K: int, want_logits: bool = False, want_probs: bool = Fals
 
 def moe_dispatch_meta(top_experts, E: int, ws=None, capacity: int = 0) -> dict:
     N, K = top_experts.shape
+    _check("top_experts", top_experts, dtype=torch.int32)
     dev = top_experts.device
     if ws is None:
         ws = workspace(load().moe_dispatch_meta_workspace_size(N, K, E), dev)
@@ -97,8 +125,12 @@ def moe_dispatch_meta(top_experts, E: int, ws=None, capacity: int = 0) -> dict:
 def moe_permute(x, pos, bins, padded_bins, K: int, P: Optional[int] = None, out=None):
     N, H = x.shape
     E = bins.shape[0]
+    _check("pos", pos, dtype=torch.int32, numel=N * K)
+    _check("bins", bins, (E,), torch.int32)
+    _check("padded_bins", padded_bins, (E,), torch.int32)
     if P is None:
-        P = padded_rows_max(N, E, K)
+        P = padded_rows_max(N, E, K) if out is None else out.shape[0]
+    _check("out", out, (P, H), x.dtype)
     if out is None:
         out = torch.empty(P, H, dtype=x.dtype, device=x.device)
     call("moe_permute", _p(x), _p(pos), _p(bins), _p(padded_bins), N, H, E, K, _dt(x), _p(out),
@@ -108,7 +140,8 @@ def moe_permute(x, pos, bins, padded_bins, K: int, P: Optional[int] = None, out=
 
 def moe_grouped_swiglu(x_perm, W1, W3, W2, padded_bins, save_gate_up: bool = False, ws=None):
     P, H = x_perm.shape
-    E, _, F = W1.shape
+    E, F = _experts(W1, W3, W2, H, x_perm.dtype)
+    _check("padded_bins", padded_bins, (E,), torch.int32)
     dev = x_perm.device
     if ws is None:
         ws = workspace(load().moe_grouped_workspace_size(), dev)
@@ -123,6 +156,9 @@ def moe_grouped_swiglu(x_perm, W1, W3, W2, padded_bins, save_gate_up: bool = Fal
 def moe_combine(out, weights, pos, N: int, y=None):
     _, H = out.shape
     K = weights.shape[1]
+    _check("weights", weights, (N, K), torch.float32)
+    _check("pos", pos, dtype=torch.int32, numel=N * K)
+    _check("y", y, (N, H), out.dtype)
     if y is None:
         y = torch.empty(N, H, dtype=out.dtype, device=out.device)
     call("moe_combine", _p(out), _p(weights), _p(pos), N, K, H, _dt(out), _p(y), _stream())
@@ -134,6 +170,11 @@ def moe_combine_bwd(dy, out, weights, pos, bins, padded_bins):
     K = weights.shape[1]
     E = bins.shape[0]
     P = out.shape[0]
+    _check("out", out, (P, H), dy.dtype)
+    _check("weights", weights, (N, K), torch.float32)
+    _check("pos", pos, dtype=torch.int32, numel=N * K)
+    _check("bins", bins, (E,), torch.int32)
+    _check("padded_bins", padded_bins, (E,), torch.int32)
     dev = dy.device
     dw = torch.empty(N, K, dtype=torch.float32, device=dev)
     dlogit = torch.empty(N, K, dtype=torch.float32, device=dev)
@@ -145,7 +186,11 @@ def moe_combine_bwd(dy, out, weights, pos, bins, padded_bins):
 
 def moe_grouped_swiglu_bwd(d_out, x_perm, act, gate_up, W1, W3, W2, padded_bins, ws=None):
     P, H = x_perm.shape
-    E, _, F = W1.shape
+    E, F = _experts(W1, W3, W2, H, x_perm.dtype)
+    _check("d_out", d_out, (P, H), x_perm.dtype)
+    _check("act", act, (P, F), x_perm.dtype)
+    _check("gate_up", gate_up, (2, P, F), x_perm.dtype)
+    _check("padded_bins", padded_bins, (E,), torch.int32)
     dev = x_perm.device
     if ws is None:
         ws = workspace(load().moe_grouped_workspace_size(), dev)
@@ -167,6 +212,15 @@ def moe_unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices,
     E = W_r.shape[1]
     K = top_experts.shape[1]
     P = dx_perm.shape[0]
+    _check("dx_perm", dx_perm, (P, H), x.dtype)
+    _check("dlogit", dlogit, (N, K), torch.float32)
+    _check("W_r", W_r, (H, E), x.dtype)
+    _check("top_experts", top_experts, (N, K), torch.int32)
+    for name, t in (("pos", pos), ("indices", indices)):
+        _check(name, t, dtype=torch.int32, numel=N * K)
+    _check("bins", bins, (E,), torch.int32)
+    _check("padded_bins", padded_bins, (E,), torch.int32)
+    _check("probs", probs, (N, E), torch.float32)
     dev = x.device
     if ws is None:
         ws = workspace(load().moe_unpermute_router_bwd_workspace_size(N, H, E, P), dev)
@@ -181,6 +235,8 @@ def moe_unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices,
 def moe_aux_loss(probs, bins, K: int, alpha: float, ws=None):
     """Load-balancing loss alpha * E * sum_i f_i * P_i; returns (loss [1], P [E])."""
     N, E = probs.shape
+    _check("probs", probs, dtype=torch.float32)
+    _check("bins", bins, (E,), torch.int32)
     dev = probs.device
     if ws is None:
         ws = workspace(load().moe_aux_loss_workspace_size(N, E), dev)
@@ -232,7 +288,17 @@ class MoELayer:
         self.aux_loss = torch.zeros(1, dtype=torch.float32, device=dev)
         self._grads = None
 
+    def _check_params(self, x, W_r, W1, W3, W2):
+        N, H, E, F, dt = self.N, self.H, self.E, self.F, self.dtype
+        _check("x", x, (N, H), dt)
+        _check("W_r", W_r, (H, E), dt)
+        _check("W1", W1, (E, H, F), dt)
+        _check("W3", W3, (E, H, F), dt)
+        _check("W2", W2, (E, F, H), dt)
+
     def forward(self, x, W_r, W1, W3, W2, y=None):
+        self._check_params(x, W_r, W1, W3, W2)
+        _check("y", y, (self.N, self.H), self.dtype)
         y = self.y if y is None else y
         call("moe_layer_fwd", _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), self.N, self.H, self.E, self.K,
              self.F, self.dt, self.mode, self.capacity, self.aux_alpha, _p(self.aux_loss), _p(y),
@@ -256,7 +322,13 @@ class MoELayer:
         """Gradients of sum(y * dy) (+ aux_grad * aux_loss when aux_alpha != 0)."""
         if not self.training:
             raise RuntimeError("layer was built with training=False")
+        self._check_params(x, W_r, W1, W3, W2)
+        _check("dy", dy, (self.N, self.H), self.dtype)
         g = self.grad_buffers() if grads is None else grads
+        shapes = {"dx": (self.N, self.H), "dW_r": (self.H, self.E), "dW1": (self.E, self.H, self.F),
+                  "dW3": (self.E, self.H, self.F), "dW2": (self.E, self.F, self.H)}
+        for k, shp in shapes.items():
+            _check(k, g[k], shp, self.dtype)
         call("moe_layer_bwd", _p(dy), _p(x), _p(W_r), _p(W1), _p(W3), _p(W2), _p(self.top_experts),
              _p(self.weights), _p(self.indices), _p(self.bins), _p(self.padded_bins), self.N, self.H,
              self.E, self.K, self.F, self.dt, self.mode, self.capacity, self.aux_alpha, float(aux_grad),
