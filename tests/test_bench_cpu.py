@@ -57,3 +57,27 @@ def test_kernel_rooflines_fractions_and_stage_totals():
     assert st["grouped_gemms"]["tflops"] == 600.0 and st["grouped_gemms"]["frac"] == 0.6
     assert st["bandwidth_kernels"] == {"kernels": ["rows"], "gbs": 5000.0, "frac": 1.0}
     assert st["metadata_us_per_step"] == 10.0
+
+
+def test_recorded_traffic_only_for_the_captured_source_and_workload(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    # the committed summary matches the current GEMM source for the training step
+    assert bench.recorded_traffic("gemm1_swiglu", "train_step") == 5.212e9
+    assert bench.recorded_traffic("gemm1_swiglu", "mixtral") is None
+    assert bench.recorded_traffic("permute", "train_step") is None
+    # a summary whose source hash is stale gives no traffic
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    csrc = tmp_path / "dropless_top_moe_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("// kernel\n")
+    import hashlib
+    sha = hashlib.sha256(b"// kernel\n").hexdigest()[:16]
+    (prof / "ncu_traffic.txt").write_text(f"# header\nk_new train_step 1e9 k.cu {sha}\n"
+                                          f"k_old train_step 2e9 k.cu 0123456789abcdef\n"
+                                          f"k_list train_step 3e9 k.cu 0123456789abcdef,{sha}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("k_new", "train_step") == 1e9
+    assert bench.recorded_traffic("k_old", "train_step") is None
+    assert bench.recorded_traffic("k_list", "train_step") == 3e9
