@@ -26,6 +26,7 @@ MUTANTS = [
      "best = p.shape[1] - 1 - np.argmax(p[:, ::-1], axis=1)"),
     ("no_renormalisation", "return v / v.sum(axis=-1, keepdims=True)", "return v"),
     ("logits_transposed_weights", "return f64(x) @ f64(W_r)", "return f64(x) @ f64(W_r)[::-1]"),
+    ("gaps_among_k_only", "m = min(K + 1, l.shape[1])", "m = min(K, l.shape[1])"),
     # dispatch metadata
     ("unstable_sort", "    for i, e in enumerate(te):\n        if not keep[i]:",
      "    for i, e in reversed(list(enumerate(te))):\n        if not keep[i]:"),

@@ -67,6 +67,20 @@ def test_router_logits_match_library_matmul():
     np.testing.assert_allclose(om.router_logits(inp["x"], inp["W_r"]), ref, rtol=1e-13, atol=1e-15)
 
 
+def test_topk_gaps_match_brute_force():
+    """Smallest gap among each row's K+1 largest logits (K when K = E), from
+    torch.topk's sorted values and a plain double loop."""
+    g = torch.Generator().manual_seed(9)
+    for E, K in ((8, 2), (8, 8), (5, 1), (64, 6)):
+        logits = torch.randn(50, E, generator=g, dtype=torch.float64)
+        got = om.topk_gaps(logits.numpy(), K)
+        m = min(K + 1, E)
+        vals = torch.topk(logits, m, dim=-1, sorted=True).values.numpy()
+        for t in range(50):
+            want = min((vals[t, j] - vals[t, j + 1] for j in range(m - 1)), default=math.inf)
+            assert got[t] == want
+
+
 def test_gap_repair_enforces_margin():
     shp, inp = small(N=512, E=8, K=2, H=32)
     gaps = om.topk_gaps(om.router_logits(inp["x"], inp["W_r"]), 2)
