@@ -1,7 +1,10 @@
-"""Data-parallel gradient reduction across replicas: two gloo ranks on CPU.
+"""Data-parallel gradient reduction across replicas: gloo ranks on CPU.
 
 Each rank holds gradients of its own tokens; after allreduce_grads every rank
-must hold the rank-ordered average, bitwise equal across ranks and runs."""
+must hold the rank-ordered average, bitwise equal across ranks and runs.  The
+library's rank-ordered sum kernel needs a GPU, so these CPU ranks exercise
+the exchange (all-to-all of shards, all-gather, chunking and padding) with a
+rank-ordered sum written here; the kernel itself is checked on the GPU."""
 import os
 import socket
 
@@ -19,6 +22,13 @@ def _free_port():
         return s.getsockname()[1]
 
 
+def _cpu_ordered_sum(recv, world, scale, out):
+    acc = torch.zeros(out.shape, dtype=torch.float32)
+    for r in range(world):
+        acc += recv[r].to(torch.float32)
+    out.copy_((acc * scale).to(out.dtype))
+
+
 def _worker(rank, world, port, q):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -28,15 +38,21 @@ def _worker(rank, world, port, q):
         for dt in (torch.float32, torch.bfloat16):
             g = torch.Generator().manual_seed(100 + rank)
             ts = [torch.randn(3, 70, 33, generator=g).to(dt), torch.randn(1001, generator=g).to(dt)]
-            allreduce_grads(ts, average=True, chunk_elems=512)
+            allreduce_grads(ts, average=True, chunk_elems=512, local_sum=_cpu_ordered_sum)
             out.append([t.clone() for t in ts])
         q.put((rank, out))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2])
-def test_allreduce_grads_two_gloo_ranks(world):
+def test_default_sum_refuses_cpu_tensors():
+    from dropless_top_moe_b200.parallel import ordered_sum
+    with pytest.raises(RuntimeError, match="CUDA"):
+        ordered_sum(torch.zeros(2, 8), 2, 0.5, torch.zeros(8))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_allreduce_grads_gloo_ranks(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
