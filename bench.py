@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--workload", default="train_step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload forward timings of the other configurations")
     ap.add_argument("--train-mode", type=int, default=1, choices=[1, 2],
                     help="1: keep the SwiGLU gates for the backward; 2: recompute them (less memory)")
     ap.add_argument("--aux-alpha", type=float, default=0.0, help="load-balancing loss weight (0 = off)")
@@ -127,6 +129,8 @@ def kernel_rooflines(per, steps, timed_ms, fl, by, peaks):
             k["bound"] = "latency"                        # a few hundred KB per launch
         elif name in fl and (name not in by or fl[name] / by[name] >= ridge):
             k["bound"], k["frac"] = "tensor", round(fl[name] / avg_s / 1e12 / tensor_peak, 4)
+            if "bf16_tflops" in peaks:
+                k["frac_burst"] = round(fl[name] / avg_s / 1e12 / peaks["bf16_tflops"], 4)
         elif name in by:
             k["bound"], k["frac"] = "hbm", round(by[name] / avg_s / 1e9 / hbm_peak, 4)
         kernels[name] = k
@@ -144,6 +148,8 @@ def kernel_rooflines(per, steps, timed_ms, fl, by, peaks):
         r = total(gemms, fl) / 1e12
         stages["grouped_gemms"] = {"kernels": sorted(gemms), "tflops": round(r, 1),
                                    "frac": round(r / tensor_peak, 4)}
+        if "bf16_tflops" in peaks:
+            stages["grouped_gemms"]["frac_burst"] = round(r / peaks["bf16_tflops"], 4)
     if rows:
         r = total(rows, by) / 1e9
         stages["bandwidth_kernels"] = {"kernels": sorted(rows), "gbs": round(r, 1),
@@ -254,15 +260,196 @@ def routing_stats(layer, shape):
 
 # ---------------------------------------------------------------- our arm
 
+class Tracer:
+    """CUDA events the library records just before and after each of its
+    kernel launches (moe_trace_attach), with the launch names."""
+
+    def __init__(self, cap: int):
+        self.cap = 0
+        self.evs = []
+        self.count = ctypes.c_int32(0)
+        self.grow(cap)
+
+    def grow(self, cap: int):
+        import torch
+        if cap <= self.cap:
+            return
+        new = [torch.cuda.Event(enable_timing=True) for _ in range(2 * (cap - self.cap))]
+        for e in new:           # torch creates the underlying cudaEvent on first record
+            e.record()
+        torch.cuda.synchronize()
+        self.evs += new
+        self.cap = cap
+        self.arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in self.evs])
+        self.labels = (ctypes.c_char_p * cap)()
+
+    def attach(self):
+        from dropless_top_moe_b200._lib import call
+        self.count.value = 0
+        call("moe_trace_attach", self.arr, self.cap, self.labels, ctypes.byref(self.count))
+
+    def detach(self):
+        from dropless_top_moe_b200._lib import call
+        call("moe_trace_detach")
+
+    def per_kernel(self):
+        """kernel name -> (total ms, launches) over the launches recorded."""
+        per = {}
+        for i in range(min(self.count.value, self.cap)):
+            name = self.labels[i].decode()
+            d = self.evs[2 * i].elapsed_time(self.evs[2 * i + 1])
+            tot, n = per.get(name, (0.0, 0))
+            per[name] = (tot + d, n + 1)
+        return per
+
+
+def launches_per_step(step, tracer):
+    import torch
+    tracer.attach()
+    step()
+    torch.cuda.synchronize()
+    tracer.detach()
+    return tracer.count.value
+
+
+def timed_steps(step, steps, tracer, gpu, flush=None):
+    """Device time of `steps` calls of step() (CUDA events on the current
+    stream, synchronised on both sides) with the per-launch trace attached
+    and the SM clocks sampled meanwhile.  Without `flush` the steps run back
+    to back between two events; with it, flush() (an L2-sized write) runs
+    before every step, outside that step's own pair of events."""
+    import torch
+    clocks = ClockSampler(gpu)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    tracer.attach()
+    if flush is None:
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(steps):
+            step()
+        s1.record()
+        torch.cuda.synchronize()
+        ms = s0.elapsed_time(s1)
+    else:
+        pairs = []
+        for _ in range(steps):
+            flush()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            step()
+            s1.record()
+            pairs.append((s0, s1))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in pairs)
+    tracer.detach()
+    return ms / steps, clocks.stop()
+
+
+def roofline_of(per, steps, ms, shape, layer, capacity, peaks, peak_src, traffic=None):
+    """Per-kernel rooflines, stage totals and the dominant kernel's roofline
+    object of one timed workload."""
+    padded_rows = int(layer.padded_bins[-1].item()) if shape.N else 0
+    # algorithmic work counts the assignments actually computed (all N*K when
+    # dropless; the kept ones in the token-dropping variant)
+    kept = int(layer.bins[-1].item()) if shape.N else 0
+    work = shape.with_(K=1, N=kept) if capacity else shape
+    fl = flops_by_kernel(work)
+    fl["route_umma"] = 2 * shape.N * shape.H * shape.E
+    by = bytes_by_kernel(shape, padded_rows)
+    by["route_umma"] = by["route_simt"]
+    kernels, stages = kernel_rooflines(per, steps, ms * steps, fl, by, peaks)
+    dom = max(per, key=lambda n: per[n][0])
+    dom_avg_s = per[dom][0] / per[dom][1] * 1e-3
+    if dom in fl:
+        peak, burst = peaks["bf16_tflops_sustained"], peaks["bf16_tflops"]
+        achieved = fl[dom] / dom_avg_s / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} sustained bf16 (kernel timed inside a long step)",
+                "peak_burst": burst, "frac_burst": round(achieved / burst, 4)}
+    else:
+        peak = peaks["hbm_gbs"]
+        achieved = by.get(dom, 0) / dom_avg_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} copy bandwidth"}
+    roof["traffic"] = traffic(dom) if traffic else None
+    tfl = (layer_flops(work) - (2 * work.N * work.H * work.E) * (3 if shape.training else 1)
+           + (2 * shape.N * shape.H * shape.E) * (3 if shape.training else 1))
+    return roof, stages, kernels, round(tfl / (ms * 1e-3) / 1e12, 1)
+
+
+def workload_desc(shape):
+    return (f"{shape.name}: N={shape.N} H={shape.H} E={shape.E} top_k={shape.K} F={shape.F} SwiGLU, "
+            f"{'forward+backward' if shape.training else 'forward'}")
+
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def footprint_bytes(shape):
+    """Bytes a step reads at least once: tokens, router and expert weights."""
+    b = 2 if shape.dtype == "bf16" else 4
+    return (shape.N * shape.H + shape.H * shape.E + 3 * shape.E * shape.H * shape.F) * b
+
+
+def run_config(name, steps, dev, tracer, peaks, peak_src):
+    """One forward workload of the layer, timed alone, for the per-config part
+    of the JSON line."""
+    import torch
+
+    from gen import WORKLOADS, make_inputs
+    import dropless_top_moe_b200 as moe
+    shape = WORKLOADS[name]
+    inp = make_inputs(shape, seed=0, device=dev)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=False, device=dev)
+
+    def step():
+        layer.forward(inp["x"], inp["W_r"], inp["W1"], inp["W3"], inp["W2"])
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n_launch = launches_per_step(step, tracer)
+    # enough steps for the clock samples (100 ms apart) to see the run
+    t0 = time.perf_counter()
+    step()
+    torch.cuda.synchronize()
+    est = max(time.perf_counter() - t0, 1e-5)
+    n_steps = int(min(500, max(steps, 0.5 / est)))
+    tracer.grow(n_launch * n_steps)
+    flush = None
+    l2 = "inputs larger than L2 (%.2f GB read per step)" % (footprint_bytes(shape) / 1e9)
+    if footprint_bytes(shape) < 2 * L2_BYTES:
+        buf = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+        flush = buf.zero_
+        l2 = "L2 flushed before every step (256 MB write outside the step's events)"
+    ms, clk = timed_steps(step, n_steps, tracer, dev.index or 0, flush)
+    per = tracer.per_kernel()
+    status = layer.status()
+    roof, stages, kernels, tflops = roofline_of(per, n_steps, ms, shape, layer, 0, peaks, peak_src)
+    out = {"workload": workload_desc(shape), "dtype": shape.dtype, "steps": n_steps, "warmup": 3,
+           "ms_per_step": round(ms, 4), "value": round(shape.N / (ms * 1e-3), 1), "unit": "tokens/s",
+           "tflops": tflops, "l2": l2, "routing": routing_stats(layer, shape), "roofline": roof,
+           "stages": stages, "kernels": kernels, "gpu_launches": tracer.count.value,
+           "launches_per_step": n_launch, "device_status": status, "clocks": clk}
+    del layer, inp
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
+    import math
+
     import torch
     import torch.distributed as dist
 
-    from gen import WORKLOADS, make_inputs, token_rows
+    from gen import WORKLOAD_ORDER, make_inputs, token_rows
     from gen.moe_inputs import _gen
 
     import dropless_top_moe_b200 as moe
-    from dropless_top_moe_b200._lib import call, load
 
     shape = workload(args)
     dev = torch.device("cuda", local_rank)
@@ -272,7 +459,6 @@ def run_ours(args, rank, world, local_rank):
         inp["x"] = token_rows(shape, shape.N, _gen(1000 + rank, dev), dev)
         if shape.training:
             inp["dy"] = torch.randn(shape.N, shape.H, generator=_gen(2000 + rank, dev), device=dev).to(shape.torch_dtype)
-    import math
     # capacity per expert = ceil(N*K/E * cf): cf = 1 is the balanced load
     capacity = (int(math.ceil(shape.N * shape.K / shape.E * args.capacity_factor))
                 if args.capacity_factor > 0 else 0)
@@ -290,110 +476,42 @@ def run_ours(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
 
-    # launches per step (counted through the trace hook)
-    def make_events(n):
-        # torch creates the underlying cudaEvent on first record
-        es = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        for e in es:
-            e.record()
-        torch.cuda.synchronize()
-        return es
-
-    cap = 4096
-    evs = make_events(2 * cap)
-    ev_arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in evs])
-    labels = (ctypes.c_char_p * cap)()
-    count = ctypes.c_int32(0)
-    call("moe_trace_attach", ev_arr, cap, labels, ctypes.byref(count))
-    step()
-    torch.cuda.synchronize()
-    per_step = count.value
-    call("moe_trace_detach")
+    tracer = Tracer(4096)
+    per_step = launches_per_step(step, tracer)
     steps = args.steps
-    cap_needed = per_step * steps
-    if cap_needed > cap:
-        evs += make_events(2 * (cap_needed - cap))
-        cap = cap_needed
-        ev_arr = (ctypes.c_void_p * (2 * cap))(*[e.cuda_event for e in evs])
-        labels = (ctypes.c_char_p * cap)()
-
-    clocks = ClockSampler(local_rank)
+    tracer.grow(per_step * steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    call("moe_trace_attach", ev_arr, cap, labels, ctypes.byref(count))
-    start.record()
-    for _ in range(steps):
-        step()
-    end.record()
-    torch.cuda.synchronize()
-    call("moe_trace_detach")
-    clk = clocks.stop()
+    ms, clk = timed_steps(step, steps, tracer, local_rank)
     if world > 1:
         dist.barrier()
-    ms = start.elapsed_time(end) / steps
     t = torch.tensor([ms], device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_max = float(t.item())
     status = layer.status()
-
-    # per-kernel device time over the timed region
-    per = {}
-    for i in range(count.value):
-        name = labels[i].decode()
-        d = evs[2 * i].elapsed_time(evs[2 * i + 1])
-        tot, n = per.get(name, (0.0, 0))
-        per[name] = (tot + d, n + 1)
-    padded_rows = int(layer.padded_bins[-1].item())
-    # algorithmic work counts the assignments actually computed (all N*K when
-    # dropless; the kept ones in the token-dropping variant)
-    kept = int(layer.bins[-1].item())
-    work = shape.with_(K=1, N=kept) if capacity else shape
-    fl = flops_by_kernel(work)
-    fl["route_umma"] = 2 * shape.N * shape.H * shape.E
-    by = bytes_by_kernel(shape, padded_rows)
-    by["route_umma"] = by["route_simt"]
+    per = tracer.per_kernel()
     peaks, peak_src = load_peaks()
-    kernels, stages = kernel_rooflines(per, steps, ms * steps, fl, by, peaks)
-    dom = max(per, key=lambda n: per[n][0])
-    dom_avg_s = per[dom][0] / per[dom][1] * 1e-3
-    if dom in fl:
-        peak = peaks["bf16_tflops_sustained"]
-        achieved = fl[dom] / dom_avg_s / 1e12
-        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{peak_src} sustained bf16 (kernel timed inside a long step)"}
-    else:
-        peak = peaks["hbm_gbs"]
-        achieved = by.get(dom, 0) / dom_avg_s / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} copy bandwidth"}
     default_variant = args.aux_alpha == 0 and args.capacity_factor == 0 and args.train_mode == 1
     # the capture is of the named workload's default variant only
-    tr = recorded_traffic(dom, shape.name) if default_variant else None
-    roof["traffic"] = tr
+    traffic = (lambda k: recorded_traffic(k, shape.name)) if default_variant else None
+    roof, stages, kernels, tflops = roofline_of(per, steps, ms, shape, layer, capacity, peaks, peak_src, traffic)
 
     result = {
         "metric": METRIC, "value": None, "unit": "tokens/s", "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32",
         "data": "synthetic (seeded normal inputs and random-init weights of the stated shapes)",
-        "config": {"workload": f"{shape.name}: N={shape.N} H={shape.H} E={shape.E} top_k={shape.K} "
-                               f"F={shape.F} SwiGLU, {'forward+backward' if shape.training else 'forward'}",
+        "config": {"workload": workload_desc(shape),
                    "tokens_per_step_per_gpu": shape.N, "parallelism": f"replicas x{world}",
                    "variant": {"train_mode": train_mode, "aux_alpha": args.aux_alpha,
                                "capacity": capacity or "dropless"},
                    "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
                          (3 * shape.E * shape.H * shape.F * 2 / 1e9)},
         "routing": routing_stats(layer, shape),
-        "tflops": round((layer_flops(work) - (2 * work.N * work.H * work.E) * (3 if shape.training else 1)
-                         + (2 * shape.N * shape.H * shape.E) * (3 if shape.training else 1))
-                        / (ms_max * 1e-3) / 1e12, 1),
-        "roofline": roof, "stages": stages, "kernels": kernels, "gpu_launches": count.value,
+        "tflops": round(tflops * ms / ms_max, 1),
+        "roofline": roof, "stages": stages, "kernels": kernels, "gpu_launches": tracer.count.value,
         "launches_per_step": per_step, "device_status": status, "clocks": clk,
     }
     result["value"] = round(shape.N * world / (ms_max * 1e-3), 1)
@@ -473,8 +591,20 @@ def run_ours(args, rank, world, local_rank):
                          "d2h_bytes_per_step": xh.numel() * eb * (2 if shape.training else 1),
                          "note": "host copies of step i+1 / i overlap compute of step i"}
 
+    # The other workloads of the layer (forward only), each timed alone on
+    # this GPU after the headline workload, on rank 0 of a single-GPU run.
+    if (world == 1 and not args.no_configs and args.workload == "train_step" and not args.tokens
+            and not args.experts and default_variant):
+        del layer, grads, inp
+        torch.cuda.empty_cache()
+        result["configs"] = {}
+        for name in WORKLOAD_ORDER:
+            if name != shape.name:
+                result["configs"][name] = run_config(name, min(steps, 20), dev, tracer, peaks, peak_src)
+        inp = None
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(shape, inp, budget_s=20.0)
+        result["cpu_baseline"] = cpu_baseline(shape, inp, target_s=10.0)
     return result
 
 
@@ -514,49 +644,81 @@ def _cores():
         return os.cpu_count()
 
 
-def cpu_baseline(shape, inp=None, budget_s=20.0, o=None):
-    """The oracle, as it stands, on a bounded token sample of the workload:
-    the sample grows until one oracle pass takes at least half the budget."""
+def _oracle_cost(shape, o, rng):
+    """Fixed per-call and per-token seconds of one oracle pass on this host.
+
+    A pass has a cost that does not depend on its token count (the backward
+    zero-fills dense float64 weight gradients of E*H*F elements each, several
+    GB at the training-step sizes) plus a cost per token; two probes of
+    different sizes separate them, so that a timed pass can be sized to make
+    the fixed part small."""
     import numpy as np
-    o = o if o is not None else _oracle_inputs(shape, inp)
-    rng = np.random.default_rng(0)
-    n = 16
-    while True:
+
+    def timed(n):
         tok = np.sort(rng.choice(shape.N, n, replace=False))
         t0 = time.perf_counter()
         _oracle_step(shape, o, tok)
-        dt = time.perf_counter() - t0
-        if dt >= budget_s / 2 or n >= shape.N:
-            break
-        n = int(min(shape.N, max(2 * n, n * (0.6 * budget_s) / max(dt, 1e-3))))
+        return time.perf_counter() - t0
+    n0, n1 = min(8, shape.N), min(128, shape.N)
+    t0 = timed(n0)
+    t1 = timed(n1) if n1 > n0 else t0
+    per_tok = max((t1 - t0) / max(n1 - n0, 1), t1 / max(n1, 1) * 0.05, 1e-7)
+    fixed = max(t0 - n0 * per_tok, 0.0)
+    return fixed, per_tok
+
+
+def _sample_tokens(shape, fixed, per_tok, target_s):
+    """Tokens of one pass that takes about target_s seconds (at least the
+    probe's size, at most the workload's N)."""
+    n = int((target_s - fixed) / per_tok)
+    return max(min(shape.N, 128), min(shape.N, n))
+
+
+def cpu_baseline(shape, inp=None, target_s=10.0, o=None):
+    """The oracle, as it stands, on one bounded token sample of the workload,
+    sized so that one pass takes about target_s seconds (its fixed per-call
+    cost then weighs little in the tokens/s)."""
+    import numpy as np
+    o = o if o is not None else _oracle_inputs(shape, inp)
+    rng = np.random.default_rng(0)
+    fixed, per_tok = _oracle_cost(shape, o, rng)
+    n = _sample_tokens(shape, fixed, per_tok, target_s)
+    tok = np.sort(rng.choice(shape.N, n, replace=False))
+    t0 = time.perf_counter()
+    _oracle_step(shape, o, tok)
+    dt = time.perf_counter() - t0
     return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
             "sample": f"{n} of {shape.N} tokens of {shape.name} ({'fwd+bwd' if shape.training else 'fwd'}), "
-                      f"float64 numpy oracle, {dt:.1f} s"}
+                      f"float64 numpy oracle, {dt:.1f} s (fixed per-call cost {fixed:.1f} s)"}
 
 
 def run_reference(args, rank, world):
-    """--impl reference: the CPU oracle on this workload's config, host cores."""
-    from gen import WORKLOADS
+    """--impl reference: the CPU oracle on this workload's config, host cores.
+
+    Each timed step is one oracle pass over a seeded token sample sized, like
+    the in-line CPU baseline, to about 10 s (less when many steps would run
+    past about 200 s of timed work), so that the oracle's fixed per-call cost
+    does not dominate its tokens/s.  Warm-up steps use a small sample: they
+    are untimed and only warm the host caches and allocator."""
     import numpy as np
     if rank != 0:
         return None
     shape = workload(args)
     o = _oracle_inputs(shape)
     rng = np.random.default_rng(1)
-    # size each step so the whole run stays within a few minutes
-    t0 = time.perf_counter()
-    _oracle_step(shape, o, np.sort(rng.choice(shape.N, 4, replace=False)))
-    per_tok = (time.perf_counter() - t0) / 4
-    n_steps = args.steps + args.warmup
-    n = int(max(1, min(shape.N, (150.0 / max(n_steps, 1)) / max(per_tok, 1e-6))))
+    fixed, per_tok = _oracle_cost(shape, o, rng)
+    target = min(10.0, 200.0 / max(args.steps, 1))
+    n = _sample_tokens(shape, fixed, per_tok, target)
     for _ in range(args.warmup):
-        _oracle_step(shape, o, np.sort(rng.choice(shape.N, n, replace=False)))
+        _oracle_step(shape, o, np.sort(rng.choice(shape.N, min(16, shape.N), replace=False)))
     t0 = time.perf_counter()
     for _ in range(args.steps):
         _oracle_step(shape, o, np.sort(rng.choice(shape.N, n, replace=False)))
     dt = time.perf_counter() - t0
     v = n * args.steps / dt
     ms = dt / args.steps * 1e3
+    sample = (f"{n} of {shape.N} tokens per step (seeded), float64 numpy oracle; fixed per-call cost "
+              f"{fixed:.1f} s, {per_tok * 1e3:.2f} ms per token")
     return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -565,7 +727,7 @@ def run_reference(args, rank, world):
                                    f"F={shape.F} SwiGLU, {'forward+backward' if shape.training else 'forward'}",
                        "tokens_per_step": n},
             "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
-                             "sample": f"{n} of {shape.N} tokens per step"},
+                             "sample": sample},
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

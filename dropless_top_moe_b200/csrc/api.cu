@@ -39,6 +39,7 @@ struct LayerWs {
   int* status;
   void* route_scratch;
   void* meta_scratch;
+  int32_t* routed_bins;   // inclusive cumsum of routed counts (before any capacity drop)
   int32_t* pos;
   void* x_perm;
   void* act;
@@ -95,6 +96,7 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int f
   w.status = (int*)take(kStatusBytes);
   w.route_scratch = take(route_scratch_bytes(H, E, dt));
   w.meta_scratch = take(meta_workspace_bytes(NK, E));
+  w.routed_bins = (int32_t*)take((size_t)E * 4);
   w.pos = (int32_t*)take(NK * 4);
   w.probs = (float*)take((size_t)N * E * 4);
   w.aux_scratch = take(aux_loss_scratch(N, E));
@@ -357,8 +359,9 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
   MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, aux ? w.probs : nullptr, top_experts, weights,
                     w.route_scratch, w.status, s));
   MOE_TRY(dispatch_meta(top_experts, (int64_t)N * K, E, indices, nullptr, bins, padded_bins, w.pos,
-                        w.meta_scratch, w.status, s, capacity));
-  if (aux) MOE_TRY(aux_loss_fwd(w.probs, bins, N, K, E, aux_alpha, aux_loss, nullptr, w.aux_scratch, s));
+                        w.meta_scratch, w.status, s, capacity, w.routed_bins));
+  // f_i of the loss counts routed assignments, dropped ones included
+  if (aux) MOE_TRY(aux_loss_fwd(w.probs, w.routed_bins, N, K, E, aux_alpha, aux_loss, nullptr, w.aux_scratch, s));
   if (N == 0) return MOE_OK;
   const RowGather ga = {x, indices, bins, N, K};
   if (!gather) MOE_TRY(permute_rows(x, w.pos, bins, padded_bins, N, H, E, K, dt, w.x_perm, s));
@@ -426,9 +429,11 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                          w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s, gather ? &ga : nullptr));
   // the sparse router backward walks the kept assignments only; the aux loss
   // and dropped assignments need every (token, expert) logit: dense path
+  // (the router probabilities exist only when the forward computed the loss)
   if ((aux_alpha != 0.0f || capacity > 0) && N > 0)
-    MOE_TRY(dense_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, bins, w.probs, N, H, E, K, dt,
-                             aux_alpha, aux_grad, dx, dW_r, w.dense_scratch, w.status, s));
+    MOE_TRY(dense_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, w.routed_bins,
+                             aux_alpha != 0.0f ? w.probs : nullptr, N, H, E, K, dt, aux_alpha, aux_grad, dx,
+                             dW_r, w.dense_scratch, w.status, s));
   else
     MOE_TRY(unpermute_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, indices, bins,
                                  padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, s));

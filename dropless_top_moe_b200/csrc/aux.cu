@@ -1,13 +1,18 @@
 // Auxiliary load-balancing loss ("MoE computation principle and execution",
 // sec. 4.2): L_aux = alpha * E * sum_i f_i * P_i, with f_i = (assignments
 // routed to expert i) / (N*K) and P_i = mean over tokens of probs[:, i].
+// f_i counts the router's assignments to expert i before any capacity drop
+// (routed_bins: their inclusive cumsum), so the loss does not depend on the
+// token-dropping variant's capacity.
 //
 // Forward: per-chunk column sums of probs (256 tokens per chunk, increasing
 // token order), then one block sums the chunks in order and forms the loss
 // with a fixed-order tree over experts.
 //
-// Backward (dense router gradient, used only when the loss is on): the counts
-// f_i are piecewise constant, so d L_aux / d p_t,i = alpha*E*f_i/N and, through
+// Backward (dense router gradient, used when the loss is on and by the
+// token-dropping variant, whose dropped assignments still pass gradient to
+// the router through the renormalised weights): the counts f_i are piecewise
+// constant, so d L_aux / d p_t,i = alpha*E*f_i/N and, through
 // the softmax, the logits of every expert receive
 //   a_t,e = g * alpha*E/N * p_t,e * (f_e - sum_i f_i p_t,i)      (g = dL/dL_aux)
 // D[t,e] = a_t,e + the renormalisation gradient of token t's kept experts.
@@ -38,7 +43,7 @@ aux_colsum_kernel(const float* __restrict__ probs, int N, int E, float* __restri
 
 // One block of 256 threads (E <= 256).
 __global__ void __launch_bounds__(256)
-aux_finalize_kernel(const float* __restrict__ part, int n_chunks, const int32_t* __restrict__ bins,
+aux_finalize_kernel(const float* __restrict__ part, int n_chunks, const int32_t* __restrict__ routed_bins,
                     int N, int K, int E, float alpha, float* __restrict__ loss, float* __restrict__ P_out) {
   __shared__ float s_v[256];
   const int e = threadIdx.x;
@@ -47,7 +52,7 @@ aux_finalize_kernel(const float* __restrict__ part, int n_chunks, const int32_t*
     float Pe = 0.f;
     for (int c = 0; c < n_chunks; ++c) Pe += part[(size_t)c * E + e];
     Pe /= (float)N;
-    const float cnt = (float)(bins[e] - (e ? bins[e - 1] : 0));
+    const float cnt = (float)(routed_bins[e] - (e ? routed_bins[e - 1] : 0));
     const float fe = cnt / ((float)N * (float)K);
     v = fe * Pe;
     if (P_out) P_out[e] = Pe;
@@ -63,11 +68,16 @@ aux_finalize_kernel(const float* __restrict__ part, int n_chunks, const int32_t*
 
 // D[t, e] for one token per warp, into D (fp32) or Dh (bf16, for the
 // tensor-core kernels, which also get the token-chunk ends chunk_end[c] =
-// min((c + 1) * chunk, N rounded up to 64)).
+// min((c + 1) * chunk, N rounded up to 64)).  probs and routed_bins are read
+// only with the load-balancing term on (probs != NULL and coef != 0); without
+// it D holds the renormalisation gradient alone (token dropping) and the
+// router probabilities, which the forward then does not write, are not read.
+// f_e = routed_bins[e] - routed_bins[e-1] counts the assignments the router
+// made to expert e, before any capacity drop.
 __global__ void __launch_bounds__(256)
 router_dense_dlogits_kernel(const float* __restrict__ probs, const float* __restrict__ dlogit,
-                            const int32_t* __restrict__ top, const int32_t* __restrict__ bins, int N, int E,
-                            int K, float coef, float* __restrict__ D, __nv_bfloat16* __restrict__ Dh,
+                            const int32_t* __restrict__ top, const int32_t* __restrict__ routed_bins, int N,
+                            int E, int K, float coef, float* __restrict__ D, __nv_bfloat16* __restrict__ Dh,
                             int32_t* __restrict__ chunk_end, int chunk) {
   if (chunk_end && blockIdx.x == 0) {
     const int n_chunks = (N + chunk - 1) / chunk;
@@ -75,19 +85,25 @@ router_dense_dlogits_kernel(const float* __restrict__ probs, const float* __rest
     for (int c = threadIdx.x; c < n_chunks; c += blockDim.x)
       chunk_end[c] = (c + 1) * chunk < last ? (c + 1) * chunk : last;
   }
+  const bool aux = probs != nullptr && coef != 0.f;
   __shared__ float s_f[256];
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    s_f[e] = (float)(bins[e] - (e ? bins[e - 1] : 0)) / ((float)N * (float)K);
+  if (aux) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      s_f[e] = (float)(routed_bins[e] - (e ? routed_bins[e - 1] : 0)) / ((float)N * (float)K);
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < N; t += warps) {
-    const float* p = probs + (size_t)t * E;
-    float part = 0.f;
-    for (int e = lane; e < E; e += 32) part = fmaf(s_f[e], p[e], part);
-    const float s = warp_sum(part);
+    const float* p = aux ? probs + (size_t)t * E : nullptr;
+    float s = 0.f;
+    if (aux) {
+      float part = 0.f;
+      for (int e = lane; e < E; e += 32) part = fmaf(s_f[e], p[e], part);
+      s = warp_sum(part);
+    }
     for (int e = lane; e < E; e += 32) {
-      float d = coef * p[e] * (s_f[e] - s);
+      float d = aux ? coef * p[e] * (s_f[e] - s) : 0.f;
       for (int k = 0; k < K; ++k)
         if (top[(size_t)t * K + k] == e) d += dlogit[(size_t)t * K + k];
       if (Dh) Dh[(size_t)t * E + e] = __float2bfloat16(d);
@@ -224,21 +240,22 @@ size_t dense_router_bwd_scratch(int N, int H, int E) {
          (size_t)round_up(chunks * 4, 256);
 }
 
-moe_status aux_loss_fwd(const float* probs, const int32_t* bins, int N, int K, int E, float alpha, float* loss,
-                        float* P, void* scratch, cudaStream_t s) {
+moe_status aux_loss_fwd(const float* probs, const int32_t* routed_bins, int N, int K, int E, float alpha,
+                        float* loss, float* P, void* scratch, cudaStream_t s) {
   const int n_chunks = (int)cdiv(N > 0 ? N : 1, kAuxChunk);
   float* part = (float*)scratch;
   MOE_TRACED("aux_colsum", s, (aux_colsum_kernel<<<n_chunks, 256, 0, s>>>(probs, N, E, part)));
   MOE_LAUNCH_CHECK();
-  MOE_TRACED("aux_finalize", s, (aux_finalize_kernel<<<1, 256, 0, s>>>(part, N > 0 ? n_chunks : 0, bins,
-                                                                       N > 0 ? N : 1, K, E, alpha, loss, P)));
+  MOE_TRACED("aux_finalize", s, (aux_finalize_kernel<<<1, 256, 0, s>>>(part, N > 0 ? n_chunks : 0,
+                                                                       routed_bins, N > 0 ? N : 1, K, E, alpha,
+                                                                       loss, P)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
 
 template <typename T>
 static moe_status dense_router_bwd_t(const void* dx_perm, const float* dlogit, const void* x, const void* W_r,
-                                     const int32_t* top, const int32_t* pos, const int32_t* bins,
+                                     const int32_t* top, const int32_t* pos, const int32_t* routed_bins,
                                      const float* probs, int N, int H, int E, int K, float coef, void* dx,
                                      void* dWr, void* scratch, int* status, cudaStream_t s) {
   float* D = (float*)scratch;
@@ -255,7 +272,7 @@ static moe_status dense_router_bwd_t(const void* dx_perm, const float* dlogit, c
     __nv_bfloat16* Dh = (__nv_bfloat16*)scratch;
     int32_t* chunk_end = (int32_t*)(part + (size_t)n_chunks * H * E);
     MOE_TRACED("router_dense_dlogits", s, (router_dense_dlogits_kernel<<<blocks, 256, 0, s>>>(
-                                              probs, dlogit, top, bins, N, E, K, coef, nullptr, Dh, chunk_end,
+                                              probs, dlogit, top, routed_bins, N, E, K, coef, nullptr, Dh, chunk_end,
                                               kWgradChunk)));
     MOE_LAUNCH_CHECK();
     moe_status st = router_dx_umma(Dh, W_r, N, H, E, dx, status, s);
@@ -268,7 +285,7 @@ static moe_status dense_router_bwd_t(const void* dx_perm, const float* dlogit, c
     return MOE_OK;
   }
   MOE_TRACED("router_dense_dlogits", s, (router_dense_dlogits_kernel<<<blocks, 256, 0, s>>>(
-                                            probs, dlogit, top, bins, N, E, K, coef, D, nullptr, nullptr, 1)));
+                                            probs, dlogit, top, routed_bins, N, E, K, coef, D, nullptr, nullptr, 1)));
   MOE_LAUNCH_CHECK();
   dim3 g1((unsigned)cdiv(H, kDT), (unsigned)cdiv(N, kDT));
   MOE_TRACED("dense_router_dx", s, (dense_router_dx_kernel<T><<<g1, 256, 0, s>>>(
@@ -286,16 +303,19 @@ static moe_status dense_router_bwd_t(const void* dx_perm, const float* dlogit, c
 }
 
 moe_status dense_router_bwd(const void* dx_perm, const float* dlogit, const void* x, const void* W_r,
-                            const int32_t* top, const int32_t* pos, const int32_t* bins, const float* probs,
-                            int N, int H, int E, int K, moe_dtype dt, float aux_alpha, float aux_grad,
-                            void* dx, void* dWr, void* scratch, int* status, cudaStream_t s) {
+                            const int32_t* top, const int32_t* pos, const int32_t* routed_bins,
+                            const float* probs, int N, int H, int E, int K, moe_dtype dt, float aux_alpha,
+                            float aux_grad, void* dx, void* dWr, void* scratch, int* status, cudaStream_t s) {
   if (N == 0) return MOE_OK;
-  const float coef = aux_grad * aux_alpha * (float)E / (float)N;
+  // without the load-balancing term neither probs nor the counts are read
+  const bool aux = aux_alpha != 0.0f && probs != nullptr;
+  const float coef = aux ? aux_grad * aux_alpha * (float)E / (float)N : 0.0f;
+  if (!aux) probs = nullptr;
   return dt == MOE_F32
-             ? dense_router_bwd_t<float>(dx_perm, dlogit, x, W_r, top, pos, bins, probs, N, H, E, K, coef, dx,
-                                         dWr, scratch, status, s)
-             : dense_router_bwd_t<__nv_bfloat16>(dx_perm, dlogit, x, W_r, top, pos, bins, probs, N, H, E, K,
-                                                 coef, dx, dWr, scratch, status, s);
+             ? dense_router_bwd_t<float>(dx_perm, dlogit, x, W_r, top, pos, routed_bins, probs, N, H, E, K, coef,
+                                         dx, dWr, scratch, status, s)
+             : dense_router_bwd_t<__nv_bfloat16>(dx_perm, dlogit, x, W_r, top, pos, routed_bins, probs, N, H, E,
+                                                 K, coef, dx, dWr, scratch, status, s);
 }
 
 }  // namespace moe

@@ -21,7 +21,7 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
 size_t meta_workspace_bytes(int64_t NK, int E);
 moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices, int32_t* bin_ids,
                          int32_t* bins, int32_t* padded_bins, int32_t* pos, void* scratch,
-                         int* status, cudaStream_t s, int capacity = 0);
+                         int* status, cudaStream_t s, int capacity = 0, int32_t* routed_bins = nullptr);
 
 // permute.cu
 moe_status permute_rows(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* pb,
@@ -46,12 +46,15 @@ moe_status unpermute_router_bwd(const void* dx_perm, const float* dlogit, const 
 // aux.cu - load-balancing loss and the dense router backward it needs
 size_t aux_loss_scratch(int N, int E);
 size_t dense_router_bwd_scratch(int N, int H, int E);
-moe_status aux_loss_fwd(const float* probs, const int32_t* bins, int N, int K, int E, float alpha, float* loss,
-                        float* P, void* scratch, cudaStream_t s);
+// routed_bins: inclusive cumsum of the assignments routed to each expert,
+// before any capacity drop (equal to bins when dropless).
+moe_status aux_loss_fwd(const float* probs, const int32_t* routed_bins, int N, int K, int E, float alpha,
+                        float* loss, float* P, void* scratch, cudaStream_t s);
+// probs and routed_bins are read only when aux_alpha != 0 and probs != NULL.
 moe_status dense_router_bwd(const void* dx_perm, const float* dlogit, const void* x, const void* W_r,
-                            const int32_t* top, const int32_t* pos, const int32_t* bins, const float* probs,
-                            int N, int H, int E, int K, moe_dtype dt, float aux_alpha, float aux_grad,
-                            void* dx, void* dWr, void* scratch, int* status, cudaStream_t s);
+                            const int32_t* top, const int32_t* pos, const int32_t* routed_bins,
+                            const float* probs, int N, int H, int E, int K, moe_dtype dt, float aux_alpha,
+                            float aux_grad, void* dx, void* dWr, void* scratch, int* status, cudaStream_t s);
 
 // gemm_simt.cu - fp32 grouped GEMMs
 moe_status grouped_swiglu_simt(const void* x_perm, const void* W1, const void* W3, const void* W2,

@@ -44,8 +44,9 @@ meta_count_kernel(const int32_t* __restrict__ top, int64_t NK, int E, int32_t* _
 __global__ void __launch_bounds__(256)
 meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E, int capacity,
                  int32_t* __restrict__ bins, int32_t* __restrict__ padded_bins,
-                 int32_t* __restrict__ sorted_start, int32_t* __restrict__ padded_start) {
-  __shared__ int s_a[256], s_b[256];
+                 int32_t* __restrict__ sorted_start, int32_t* __restrict__ padded_start,
+                 int32_t* __restrict__ routed_bins) {
+  __shared__ int s_a[256], s_b[256], s_r[256];
   const int e = threadIdx.x;
   int total = 0;
   if (e < E) {
@@ -55,6 +56,7 @@ meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E, int ca
       total += v;
     }
   }
+  s_r[e] = (e < E) ? total : 0;   // routed, before any capacity drop
   // token-dropping variant: only the first `capacity` assignments are kept
   if (capacity > 0 && total > capacity) total = capacity;
   const int padded = (int)round_up(total, kTile);
@@ -65,12 +67,15 @@ meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E, int ca
   for (int off = 1; off < 256; off <<= 1) {
     const int a = (e >= off) ? s_a[e - off] : 0;
     const int b = (e >= off) ? s_b[e - off] : 0;
+    const int r = (e >= off) ? s_r[e - off] : 0;
     __syncthreads();
     s_a[e] += a;
     s_b[e] += b;
+    s_r[e] += r;
     __syncthreads();
   }
   if (e < E) {
+    if (routed_bins) routed_bins[e] = s_r[e];
     if (bins) bins[e] = s_a[e];
     padded_bins[e] = s_b[e];
     sorted_start[e] = s_a[e] - total;
@@ -141,7 +146,7 @@ size_t meta_workspace_bytes(int64_t NK, int E) {
 
 moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices, int32_t* bin_ids,
                          int32_t* bins, int32_t* padded_bins, int32_t* pos, void* scratch,
-                         int* status, cudaStream_t s, int capacity) {
+                         int* status, cudaStream_t s, int capacity, int32_t* routed_bins) {
   const int n_chunks = (int)cdiv(NK > 0 ? NK : 1, kMetaChunk);
   int32_t* chunk_counts = (int32_t*)scratch;
   int32_t* sorted_start = chunk_counts + (size_t)n_chunks * E;
@@ -149,7 +154,7 @@ moe_status dispatch_meta(const int32_t* top, int64_t NK, int E, int32_t* indices
   MOE_TRACED("meta_count", s, (meta_count_kernel<<<n_chunks, 256, E * sizeof(int), s>>>(top, NK, E, chunk_counts, status)));
   MOE_LAUNCH_CHECK();
   MOE_TRACED("meta_scan", s, (meta_scan_kernel<<<1, 256, 0, s>>>(chunk_counts, n_chunks, E, capacity, bins, padded_bins, sorted_start,
-                                     padded_start)));
+                                     padded_start, routed_bins)));
   MOE_LAUNCH_CHECK();
   if (NK > 0) {
     // (32 + 2) * E counters: at most 34 KB for E <= 256, within the default

@@ -22,9 +22,6 @@ constexpr int kNoAllocScratchInts = kNoAllocChunkExperts + 2 * 256;
 // Shared by every call on a device; keeps the last call's contents.
 __device__ __align__(256) int32_t g_meta_scratch[kNoAllocScratchInts];
 
-// Device address of g_meta_scratch per device, looked up on first use.
-void* g_scratch_addr[64] = {nullptr};
-
 }  // namespace
 
 extern "C" moe_status moe_dispatch_meta_noalloc(const int32_t* top_experts, int32_t N, int32_t K,
@@ -36,21 +33,18 @@ extern "C" moe_status moe_dispatch_meta_noalloc(const int32_t* top_experts, int3
   if (!padded_bins || (N > 0 && (!top_experts || !pos))) return MOE_ERR_INVALID_ARG;
   const int64_t NK = (int64_t)N * K;
   if (moe::meta_workspace_bytes(NK, E) > sizeof(g_meta_scratch)) return MOE_ERR_WORKSPACE;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
-  if (!g_scratch_addr[dev]) {
-    // set-up, once per device, with that device current: the array's name is
-    // a host-side stand-in, so the kernels get its device address instead
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_meta_scratch) != cudaSuccess || p == nullptr) {
-      (void)cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    g_scratch_addr[dev] = p;
+  // The array's name is a host-side stand-in, so the kernels get its device
+  // address, looked up with the caller's device current.  The lookup runs on
+  // every call (it allocates nothing and is cheap once the module is loaded):
+  // an address kept from an earlier call could belong to a context that a
+  // device reset has since destroyed.
+  void* scratch = nullptr;
+  if (cudaGetSymbolAddress(&scratch, g_meta_scratch) != cudaSuccess || scratch == nullptr) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
   }
   // The count kernel writes every chunk count (zeros included) and the scan
   // writes every start, so nothing in the array needs clearing first.
-  return moe::dispatch_meta(top_experts, NK, E, indices, bin_ids, bins, padded_bins, pos,
-                            g_scratch_addr[dev], status, (cudaStream_t)stream, 0);
+  return moe::dispatch_meta(top_experts, NK, E, indices, bin_ids, bins, padded_bins, pos, scratch, status,
+                            (cudaStream_t)stream, 0);
 }

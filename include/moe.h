@@ -168,9 +168,11 @@ moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, i
  *   larger sizes return MOE_ERR_WORKSPACE before any device work.
  *   status: NULL, or a device int32 the caller zeroed; MOE_DEVERR_* bits are
  *   OR-ed into it.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  All calls on a device share the one array,
+ *   Every call looks up the array's device address (cudaGetSymbolAddress)
+ *   on the current device, so a device reset or a new context needs no
+ *   re-initialisation.  The first call on a device may load the library's
+ *   device code there: make that first call before any stream capture.  All
+ *   calls on a device share the one array,
  *   which keeps the last call's contents: calls that overlap on the GPU (on
  *   different streams without ordering) race and give wrong results.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
@@ -240,11 +242,15 @@ moe_status moe_grouped_swiglu_bwd(const void* d_out, const void* x_perm, const v
  *                dlogit_i * x[token(i)]
  * (sums in fixed order, fp32).  indices/bins/padded_bins from
  * moe_dispatch_meta; P = rows of dx_perm.
+ * With aux_alpha == 0 the router terms walk the assignments listed in
+ * indices, so every assignment must have been kept (dropless metadata); the
+ * token-dropping variant's router gradient comes from moe_layer_bwd.
  * With aux_alpha != 0 the router also receives the gradient of
  * aux_grad * L_aux (see moe_aux_loss): every logit gets
  *   a[t,e] = aux_grad*aux_alpha*E/N * probs[t,e] * (f_e - sum_i f_i probs[t,i]),
- * f_e = count_e / (N*K), and the router terms use the dense
- * D = a + (dlogit scattered to the kept experts):
+ * f_e = count_e / (N*K) with count_e = bins[e] - bins[e-1] taken as the
+ * assignments routed to e (see moe_aux_loss), and the router terms use the
+ * dense D = a + (dlogit scattered to the experts of every slot):
  *   dx[t] = sum_k dx_perm[pos[t*K+k]] + sum_e D[t,e] W_r[:,e],  dW_r = x^T D
  * (fixed-order fp32 reductions); probs [N,E] float32 is then required.
  * ws: moe_unpermute_router_bwd_workspace_size bytes.
@@ -261,7 +267,10 @@ moe_status moe_unpermute_router_bwd(const void* dx_perm, const float* dlogit, co
 
 /* Auxiliary load-balancing loss ("MoE computation principle and execution",
  * sec. 4.2): *loss = alpha * E * sum_i f_i * P_i with f_i = count_i / (N*K)
- * (count_i from bins) and P_i = mean over tokens of probs[:, i].  Column sums
+ * and P_i = mean over tokens of probs[:, i].  count_i = bins[i] - bins[i-1]
+ * is the number of assignments the router made to expert i: with token
+ * dropping, pass the bins of a dropless (capacity 0) dispatch, since the loss
+ * counts dropped assignments too (the layer calls do this).  Column sums
  * run over 256-token chunks in increasing order, then over the chunks in
  * order, then a fixed pairwise tree over experts: deterministic.
  *   probs [N,E] float32 (moe_route's probs); bins [E]; loss: device float;
@@ -279,7 +288,8 @@ moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int3
  *   capacity: 0 = dropless; > 0 = token-dropping variant (see
  *   moe_dispatch_meta): dropped (token, expert) pairs add nothing to y.
  *   aux_alpha != 0 also computes the load-balancing loss into *aux_loss (a
- *   device float, see moe_aux_loss) and keeps the router probabilities in the
+ *   device float, see moe_aux_loss; with token dropping its f_i still count
+ *   every routed assignment) and keeps the router probabilities in the
  *   workspace for the backward pass; aux_alpha = 0 skips both.
  * ws: moe_workspace_size(..., training) bytes; with training != 0 it keeps
  * what moe_layer_bwd reads. */

@@ -232,7 +232,7 @@ def test_dispatch_meta_capacity_bit_exact():
 def test_memory_optimised_backward_is_bit_identical(shape):
     """training=2 keeps no gate/up projections and recomputes them in the
     backward with the forward's own kernel: same bits as training=1, less
-    workspace."""
+    workspace, and both within tolerance of the oracle."""
     c = make_case(shape, seed=13, with_dy=True)
     outs = {}
     for mode in (1, 2):
@@ -247,6 +247,13 @@ def test_memory_optimised_backward_is_bit_identical(shape):
     assert torch.equal(outs[1][0], outs[2][0])
     for k in outs[1][1]:
         assert torch.equal(outs[1][1][k], outs[2][1][k]), k
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    W1, W3, W2 = c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu()
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], W1, W3, W2, shape.K, routing=ref)["y"]
+    assert_scaled(outs[2][0], yr, shape.dtype, "y")
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], W1, W3, W2, shape.K, c["dy"].cpu(), routing=ref)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(outs[2][1][k], gr[k], shape.dtype, k)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -271,3 +278,95 @@ def test_empty_batch(dtype):
     assert int(layer.bins.abs().sum()) == 0 and int(layer.padded_bins.abs().sum()) == 0
     for k in ("dW_r", "dW1", "dW3", "dW2"):
         assert int(torch.count_nonzero(g[k])) == 0, k
+
+
+# Load-balancing loss and token dropping together: the loss's f_i count every
+# routed assignment, dropped ones included (icman sec. 4.2 defines f_i as the
+# share of tokens the router assigns to expert i; capacity, sec. 3.4, acts
+# after that assignment).  bf16 E % 64 == 0 takes the tensor-core dense router
+# backward, the others the fp32 CUDA-core one.
+AUX_CAP = [small_shape("auxcap_f32", N=256, H=64, E=8, K=2, F=96, dtype="f32", skew="zipf", skew_param=1.0,
+                       training=True),
+           small_shape("auxcap_bf16_e64", N=1000, H=256, E=64, K=4, F=256, skew="zipf", skew_param=1.0,
+                       training=True),
+           small_shape("auxcap_bf16_e16", N=700, H=128, E=16, K=2, F=128, skew="zipf", skew_param=1.0,
+                       training=True)]
+
+
+@pytest.mark.parametrize("shape", AUX_CAP, ids=lambda s: s.name)
+def test_layer_aux_loss_with_token_dropping(shape):
+    alpha, g = 0.02, 0.9
+    cap = om.capacity_from_factor(shape.N, shape.E, 1.0, shape.K)
+    c = make_case(shape, seed=14, with_dy=True)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=True, aux_alpha=alpha, capacity=cap)
+    y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"]).clone()
+    grads = layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"], aux_grad=g)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    np.testing.assert_array_equal(layer.top_experts.cpu().numpy(), ref["top_experts"])
+    m = om.dispatch_meta(ref["top_experts"], shape.E, capacity=cap)
+    assert m["hist"].sum() < shape.N * shape.K          # something was dropped
+    np.testing.assert_array_equal(layer.bins.cpu().numpy(), m["bins"])
+    la = om.aux_loss(ref["probs"], ref["top_experts"], alpha)
+    assert abs(layer.aux_loss.item() - la) <= 1e-4 * abs(la)
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                        routing=ref, capacity=cap)["y"]
+    assert_scaled(y, yr, shape.dtype, "y")
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                         c["dy"].cpu(), routing=ref, aux_alpha=alpha, aux_grad=g, capacity=cap)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(grads[k], gr[k], shape.dtype, k)
+
+
+# Every layer variant on a workspace whose bytes past the status region hold
+# 0xFF (a NaN bit pattern for fp32 and bf16), with NaN-filled outputs: a read
+# of anything the forward did not write, or an output left unwritten, shows
+# up as NaN against the oracle.
+POISON = [("dropless", dict()), ("capacity", dict(capacity_factor=1.0)), ("aux", dict(aux_alpha=0.01)),
+          ("aux_capacity", dict(aux_alpha=0.01, capacity_factor=1.0)), ("memopt", dict(mode=2)),
+          ("gather", dict(gather_rows=True)), ("gather_memopt_capacity", dict(gather_rows=True, mode=2,
+                                                                              capacity_factor=1.0))]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("name,opts", POISON, ids=[p[0] for p in POISON])
+def test_layer_on_poisoned_workspace_matches_oracle(dtype, name, opts):
+    if dtype == "f32" and opts.get("gather_rows"):
+        pytest.skip("row gathers are a bf16 option")
+    if dtype == "bf16":
+        shape = small_shape("poison", N=777, H=256, E=64, K=4, F=256, skew="zipf", skew_param=1.0,
+                            training=True)
+    else:
+        shape = small_shape("poison_f32", N=200, H=64, E=8, K=2, F=96, dtype="f32", skew="zipf",
+                            skew_param=1.0, training=True)
+    cap = (om.capacity_from_factor(shape.N, shape.E, opts["capacity_factor"], shape.K)
+           if "capacity_factor" in opts else 0)
+    alpha, g = opts.get("aux_alpha", 0.0), 1.3
+    c = make_case(shape, seed=15, with_dy=True)
+    layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
+                         training=opts.get("mode", 1), aux_alpha=alpha, capacity=cap,
+                         gather_rows=opts.get("gather_rows", False))
+    layer.ws[256:].fill_(0xFF)
+    grads = layer.grad_buffers()
+    for v in grads.values():
+        v.fill_(float("nan"))
+    layer.y.fill_(float("nan"))
+    y = layer.forward(c["x"], c["W_r"], c["W1"], c["W3"], c["W2"]).clone()
+    layer.backward(c["dy"], c["x"], c["W_r"], c["W1"], c["W3"], c["W2"], aux_grad=g)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    np.testing.assert_array_equal(layer.top_experts.cpu().numpy(), ref["top_experts"])
+    if alpha:
+        la = om.aux_loss(ref["probs"], ref["top_experts"], alpha)
+        assert abs(layer.aux_loss.item() - la) <= 1e-4 * abs(la)
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                        routing=ref, capacity=cap)["y"]
+    assert_scaled(y, yr, shape.dtype, "y")
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                         c["dy"].cpu(), routing=ref, aux_alpha=alpha, aux_grad=g, capacity=cap)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert not torch.isnan(grads[k]).any(), k
+        assert_scaled(grads[k], gr[k], shape.dtype, k)

@@ -9,6 +9,8 @@ dropless row layout of sec. 3).  The gathered tiles hold the same bf16 values
 in the same order as the staged pipeline's x_perm, and every accumulation runs
 in the same order, so the layer must agree with route -> dispatch metadata ->
 permute -> grouped GEMMs -> combine (and the backward stages) bit for bit.
+Every case is also held to the CPU oracle at the layer's tolerances, so an
+error shared by both CUDA paths cannot pass.
 """
 import numpy as np
 import pytest
@@ -16,7 +18,7 @@ import torch
 
 import dropless_top_moe_b200 as moe
 from oracle import moe_oracle as om
-from tests._cases import make_case, small_shape
+from tests._cases import assert_scaled, make_case, small_shape
 
 pytestmark = pytest.mark.gpu
 
@@ -50,6 +52,21 @@ def _staged(c, shape, capacity=0):
     return res
 
 
+def _check_oracle(c, shape, y, g, capacity=0):
+    """y and every gradient against the float64 oracle (routing taken from
+    the oracle's own logits; the inputs keep a 1e-3 logit gap)."""
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    W1, W3, W2 = c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu()
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], W1, W3, W2, shape.K, routing=ref, capacity=capacity)["y"]
+    assert_scaled(y, yr, shape.dtype, "y vs oracle")
+    if g is None:
+        return
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], W1, W3, W2, shape.K, c["dy"].cpu(), routing=ref,
+                         capacity=capacity)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(g[k], gr[k], shape.dtype, f"{k} vs oracle")
+
+
 def _layer(c, shape, mode=1, capacity=0):
     layer = moe.MoELayer(shape.N, shape.H, shape.E, shape.K, shape.F, dtype=shape.torch_dtype,
                          training=mode, capacity=capacity, gather_rows=True)
@@ -71,6 +88,7 @@ def test_layer_gather_matches_staged_pipeline_bitwise(shape):
         assert torch.equal(y, ref["y"]), "y"
         for k in ("dW1", "dW3", "dW2", "dx", "dW_r"):
             assert torch.equal(g[k], ref[k]), f"{k} mode={mode}"
+        _check_oracle(c, shape, y, g)
 
 
 def test_layer_gather_token_dropping_bitwise():
@@ -83,6 +101,7 @@ def test_layer_gather_token_dropping_bitwise():
     assert torch.equal(y, ref["y"])
     for k in ("dW1", "dW3", "dW2"):
         assert torch.equal(g[k], ref[k]), k
+    _check_oracle(c, shape, y, g, capacity=cap)
 
 
 
@@ -99,3 +118,4 @@ def test_gather_forward_only_layer():
     torch.cuda.synchronize()
     assert layer.status() == 0
     assert torch.equal(y, y_ref)
+    _check_oracle(c, shape, y, None)

@@ -189,3 +189,48 @@ def test_sum_rank_ordered_matches_ordered_fp32_sum(dt, n, numel):
     for r in range(n):
         acc += shards[r].float()
     assert torch.equal(out, (acc * (1.0 / n)).to(dt))
+
+
+COMBINE_BWD = [small_shape("cb_f32", N=256, H=128, E=4, K=2, F=256, dtype="f32", training=True),
+               small_shape("cb_bf16", N=700, H=256, E=16, K=4, F=256, training=True),
+               small_shape("cb_bf16_k8", N=333, H=512, E=64, K=8, F=128, skew="zipf", skew_param=1.0,
+                           training=True)]
+
+
+@pytest.mark.parametrize("shape", COMBINE_BWD, ids=lambda s: s.name)
+def test_combine_bwd_dw_and_dlogit_match_oracle(shape):
+    """moe_combine_bwd per stage (MegaBlocks sec. 4: the scatter's backward is
+    a gather; icman sec. 2.2: the router's gradient flows through the kept,
+    renormalised weights).  dw[t,k] against the oracle's dw, and dlogit[t,k]
+    against the oracle's dense softmax-and-renormalisation gradient at the
+    chosen expert, which must vanish at every other expert."""
+    c = make_case(shape, seed=17, with_dy=True)
+    N, E, K = shape.N, shape.E, shape.K
+    r = moe.moe_route(c["x"], c["W_r"], K)
+    m = moe.moe_dispatch_meta(r["top_experts"], E)
+    xp = moe.moe_permute(c["x"], m["pos"], m["bins"], m["padded_bins"], K)
+    _, out, _ = moe.moe_grouped_swiglu(xp, c["W1"], c["W3"], c["W2"], m["padded_bins"])
+    dw, dlogit, d_out = moe.moe_combine_bwd(c["dy"], out, r["weights"], m["pos"], m["bins"], m["padded_bins"])
+    torch.cuda.synchronize()
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], K)
+    np.testing.assert_array_equal(r["top_experts"].cpu().numpy(), ref["top_experts"])
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), K,
+                         c["dy"].cpu(), routing=ref)
+    assert_scaled(dw, gr["dw"], shape.dtype, "dw")
+    te = ref["top_experts"].astype(np.int64)
+    chosen = np.take_along_axis(gr["dlogits"], te, axis=1)
+    assert_scaled(dlogit, chosen, shape.dtype, "dlogit")
+    off = gr["dlogits"].copy()
+    np.put_along_axis(off, te, 0.0, axis=1)
+    assert np.max(np.abs(off)) <= 1e-12 * max(1.0, np.max(np.abs(gr["dlogits"])))
+    # d_out rows: the routing weight times dy, pad rows zero
+    ref_m = om.dispatch_meta(ref["top_experts"], E)
+    dO = d_out.cpu().double().numpy()
+    w = r["weights"].cpu().double().numpy()
+    dy = om.f64(c["dy"].cpu())
+    pos = ref_m["pos"].reshape(N, K)
+    want = np.zeros_like(dO[: int(ref_m["padded_bins"][-1])])
+    for t in range(N):
+        for k in range(K):
+            want[pos[t, k]] = w[t, k] * dy[t]
+    assert_scaled(dO[: want.shape[0]], want, shape.dtype, "d_out")
