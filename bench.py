@@ -96,9 +96,12 @@ def bytes_by_kernel(s, padded_rows):
             "combine": N * K * H * b + N * K * 8 + N * H * b,
             "combine_bwd": N * H * b + N * K * H * b + padded_rows * H * b + N * K * 12,
             "unpermute_dx": N * K * H * b + N * H * b + N * K * 12,
-            # x is needed once per token; the kernel gathers it once per
-            # assignment (K times, the repeats mostly from L2)
+            # x is needed once per token; the CUDA-core kernel (fp32 layers)
+            # gathers it once per assignment (K times, the repeats mostly from L2)
             "router_wgrad_partial": N * H * b + N * K * 8 + (padded_rows // 128) * H * 4,
+            # tensor-core x^T D: x once, the token's K dlogits and expert ids,
+            # dW_r written
+            "router_wgrad": N * H * b + N * K * 8 + H * E * b,
             "meta_count": N * K * 4, "meta_place": N * K * 4 * 3}
 
 

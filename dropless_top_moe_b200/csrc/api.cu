@@ -95,7 +95,7 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int f
   };
   w.status = (int*)take(kStatusBytes);
   w.route_scratch = take(route_scratch_bytes(H, E, dt));
-  w.meta_scratch = take(meta_workspace_bytes(NK, E));
+  w.meta_scratch = take(meta_workspace_bytes(N, E));
   w.routed_bins = (int32_t*)take((size_t)E * 4);
   w.pos = (int32_t*)take(NK * 4);
   w.probs = (float*)take((size_t)N * E * 4);
@@ -110,19 +110,25 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int f
     w.d_gate_up = take(2 * P * F * eb);
     w.dx_perm = take(P * H * eb);
     w.dlogit = (float*)take(NK * 4);
-    w.ur_scratch = take(unpermute_router_bwd_scratch(H, E, P));
+    w.ur_scratch = take(unpermute_router_bwd_scratch(N, H, E, P));
     w.dense_scratch = take(dense_router_bwd_scratch(N, H, E));
   }
   w.total = off;
   return w;
 }
 
+bool routes_on_tensor_cores(int N, int H, int E, int K, moe_dtype dt) {
+  return dt == MOE_BF16 && route_umma_supported(N, H, E, K);
+}
+
+// chunk_counts: with the tensor-core router, also the per-128-token expert
+// counts the dispatch metadata starts from (NULL: not wanted).
 moe_status route_any(const void* x, const void* W_r, int N, int H, int E, int K, moe_dtype dt,
                      float* logits, float* probs, int32_t* top, float* w, void* scratch, int* status,
-                     cudaStream_t s) {
+                     cudaStream_t s, int32_t* chunk_counts = nullptr) {
   if (N == 0) return MOE_OK;
-  if (dt == MOE_BF16 && route_umma_supported(N, H, E, K))
-    return route_umma(x, W_r, N, H, E, K, logits, probs, top, w, scratch, status, s);
+  if (routes_on_tensor_cores(N, H, E, K, dt))
+    return route_umma(x, W_r, N, H, E, K, logits, probs, top, w, scratch, status, s, chunk_counts);
   if (route_simt_supported(H, E, K, (int)elem_bytes(dt)))
     return route_simt(x, W_r, N, H, E, K, dt, logits, probs, top, w, s);
   return MOE_ERR_UNSUPPORTED;
@@ -171,13 +177,14 @@ size_t moe_route_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, moe_
 }
 
 size_t moe_dispatch_meta_workspace_size(int32_t N, int32_t K, int32_t E) {
-  return al256(kStatusBytes) + al256(meta_workspace_bytes((int64_t)N * K, E));
+  (void)K;
+  return al256(kStatusBytes) + al256(meta_workspace_bytes(N, E));
 }
 
 size_t moe_grouped_workspace_size(void) { return al256(kStatusBytes); }
 
 size_t moe_unpermute_router_bwd_workspace_size(int32_t N, int32_t H, int32_t E, int64_t P) {
-  return al256(kStatusBytes) + al256(unpermute_router_bwd_scratch(H, E, P)) +
+  return al256(kStatusBytes) + al256(unpermute_router_bwd_scratch(N, H, E, P)) +
          al256(dense_router_bwd_scratch(N, H, E));
 }
 
@@ -187,7 +194,8 @@ size_t moe_aux_loss_workspace_size(int32_t N, int32_t E) {
 
 size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F, moe_dtype dt,
                           int32_t training) {
-  if (check_shape(N, H, E, K, dt) != MOE_OK || F <= 0 || !layer_flags_ok(training, dt)) return 0;
+  if (check_shape(N, H, E, K, dt) != MOE_OK || check_ffn(H, F, dt) != MOE_OK || !layer_flags_ok(training, dt))
+    return 0;
   return carve(nullptr, N, H, E, K, F, dt, training).total;
 }
 
@@ -228,8 +236,8 @@ moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, i
   if (!padded_bins || (N > 0 && (!top_experts || !pos))) return MOE_ERR_INVALID_ARG;
   if (!ws || ws_bytes < moe_dispatch_meta_workspace_size(N, K, E)) return MOE_ERR_WORKSPACE;
   char* base = (char*)ws;
-  return dispatch_meta(top_experts, (int64_t)N * K, E, indices, bin_ids, bins, padded_bins, pos,
-                       base + al256(kStatusBytes), (int*)ws, (cudaStream_t)stream, capacity);
+  return dispatch_meta(top_experts, N, K, E, indices, bin_ids, bins, padded_bins, pos, base + al256(kStatusBytes),
+                       (int*)ws, (cudaStream_t)stream, capacity);
 }
 
 moe_status moe_permute(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* padded_bins,
@@ -314,10 +322,10 @@ moe_status moe_unpermute_router_bwd(const void* dx_perm, const float* dlogit, co
   char* scratch = (char*)ws + al256(kStatusBytes);
   if (aux)
     return dense_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, bins, probs, N, H, E, K, dt, aux_alpha,
-                            aux_grad, dx, dW_r, scratch + al256(unpermute_router_bwd_scratch(H, E, P)),
+                            aux_grad, dx, dW_r, scratch + al256(unpermute_router_bwd_scratch(N, H, E, P)),
                             (int*)ws, (cudaStream_t)stream);
   return unpermute_router_bwd(dx_perm, dlogit, x, W_r, top_experts, pos, indices, bins, padded_bins, N,
-                              H, E, K, P, dt, dx, dW_r, scratch, (cudaStream_t)stream);
+                              H, E, K, P, dt, dx, dW_r, scratch, (int*)ws, (cudaStream_t)stream);
 }
 
 moe_status moe_aux_loss(const float* probs, const int32_t* bins, int32_t N, int32_t K, int32_t E,
@@ -356,10 +364,13 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
   }
+  // the tensor-core router also counts each 128-token chunk's expert ids
+  // into the metadata scratch, which saves the metadata its counting pass
+  const bool counted = N > 0 && routes_on_tensor_cores(N, H, E, K, dt);
   MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, aux ? w.probs : nullptr, top_experts, weights,
-                    w.route_scratch, w.status, s));
-  MOE_TRY(dispatch_meta(top_experts, (int64_t)N * K, E, indices, nullptr, bins, padded_bins, w.pos,
-                        w.meta_scratch, w.status, s, capacity, w.routed_bins));
+                    w.route_scratch, w.status, s, counted ? (int32_t*)w.meta_scratch : nullptr));
+  MOE_TRY(dispatch_meta(top_experts, N, K, E, indices, nullptr, bins, padded_bins, w.pos, w.meta_scratch,
+                        w.status, s, capacity, w.routed_bins, counted));
   // f_i of the loss counts routed assignments, dropped ones included
   if (aux) MOE_TRY(aux_loss_fwd(w.probs, w.routed_bins, N, K, E, aux_alpha, aux_loss, nullptr, w.aux_scratch, s));
   if (N == 0) return MOE_OK;
@@ -423,20 +434,27 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
       MOE_TRY(gemm1_umma(w.x_perm, W1, W3, padded_bins, E, H, F, P, nullptr, G, U, w.status, s,
                          "gate_up_recompute", gather ? &ga : nullptr));
   }
+  // the sparse router backward of a bf16 layer takes x^T D on the tensor
+  // cores; the combine backward writes D (bf16) beside the dlogits
+  const bool dense_router = (aux_alpha != 0.0f || capacity > 0) && N > 0;
+  void* Dh = (!dense_router && dt == MOE_BF16 && router_wgrad_tc_supported(H, E))
+                 ? unpermute_router_bwd_dh(w.ur_scratch, N, H, E, P)
+                 : nullptr;
   MOE_TRY(combine_bwd_rows(dy, w.out, weights, w.pos, bins, padded_bins, N, K, H, E, dt, nullptr,
-                           w.dlogit, w.d_out, s));
+                           w.dlogit, w.d_out, s, top_experts, Dh));
   MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
                          w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s, gather ? &ga : nullptr));
   // the sparse router backward walks the kept assignments only; the aux loss
   // and dropped assignments need every (token, expert) logit: dense path
   // (the router probabilities exist only when the forward computed the loss)
-  if ((aux_alpha != 0.0f || capacity > 0) && N > 0)
+  if (dense_router)
     MOE_TRY(dense_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, w.routed_bins,
                              aux_alpha != 0.0f ? w.probs : nullptr, N, H, E, K, dt, aux_alpha, aux_grad, dx,
                              dW_r, w.dense_scratch, w.status, s));
   else
     MOE_TRY(unpermute_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, indices, bins,
-                                 padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, s));
+                                 padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, w.status, s,
+                                 Dh != nullptr));
   return MOE_OK;
 }
 

@@ -234,10 +234,23 @@ constexpr int kWgradChunk = 1024;
 size_t aux_loss_scratch(int N, int E) { return (size_t)cdiv(N > 0 ? N : 1, kAuxChunk) * E * sizeof(float); }
 
 size_t dense_router_bwd_scratch(int N, int H, int E) {
-  // fp32 D (or bf16 D) | partials [chunks, H, E] fp32 | chunk ends
+  // fp32 D (or bf16 D) | partials: [chunks, H, E] fp32 of the CUDA-core
+  // weight gradient, or those of the tensor-core one
   const int64_t chunks = cdiv(N > 0 ? N : 1, kWgradChunk);
-  return (size_t)round_up((int64_t)N * E * sizeof(float), 256) + (size_t)chunks * H * E * sizeof(float) +
-         (size_t)round_up(chunks * 4, 256);
+  const size_t simt = (size_t)chunks * H * E * sizeof(float);
+  const size_t tc = router_wgrad_tc_supported(H, E) ? router_wgrad_tc_scratch(N, H, E) : 0;
+  return (size_t)round_up((int64_t)N * E * sizeof(float), 256) + (simt > tc ? simt : tc);
+}
+
+moe_status scatter_dlogits(const float* dlogit, const int32_t* top, int N, int E, int K, void* Dh, cudaStream_t s) {
+  if (N == 0) return MOE_OK;
+  int blocks = (int)cdiv(N, 8);
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  MOE_TRACED("router_dlogits", s, (router_dense_dlogits_kernel<<<blocks, 256, 0, s>>>(
+                                      nullptr, dlogit, top, nullptr, N, E, K, 0.f, nullptr, (__nv_bfloat16*)Dh,
+                                      nullptr, 1)));
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
 }
 
 moe_status aux_loss_fwd(const float* probs, const int32_t* routed_bins, int N, int K, int E, float alpha,
@@ -267,22 +280,16 @@ static moe_status dense_router_bwd_t(const void* dx_perm, const float* dlogit, c
   if (std::is_same<T, __nv_bfloat16>::value && router_bwd_umma_supported(H, E)) {
     // tensor cores: D in bf16 (rounded once from the fp32 value), then
     // dx = D * W_r^T + unpermute sum and dW_r = x^T * D as tcgen05 GEMMs
-    // scratch: Dh [N, E] bf16 (in D's place) | fp32 partials | chunk ends
-    const int n_chunks = (int)cdiv(N, kWgradChunk);
+    // scratch: Dh [N, E] bf16 (in D's place) | partials of x^T * D
     __nv_bfloat16* Dh = (__nv_bfloat16*)scratch;
-    int32_t* chunk_end = (int32_t*)(part + (size_t)n_chunks * H * E);
     MOE_TRACED("router_dense_dlogits", s, (router_dense_dlogits_kernel<<<blocks, 256, 0, s>>>(
-                                              probs, dlogit, top, routed_bins, N, E, K, coef, nullptr, Dh, chunk_end,
-                                              kWgradChunk)));
+                                              probs, dlogit, top, routed_bins, N, E, K, coef, nullptr, Dh, nullptr,
+                                              1)));
     MOE_LAUNCH_CHECK();
     moe_status st = router_dx_umma(Dh, W_r, N, H, E, dx, status, s);
     if (st == MOE_OK) st = unpermute_add_rows(dx_perm, pos, N, H, K, MOE_BF16, dx, s);
-    if (st == MOE_OK) st = router_wgrad_umma(x, Dh, chunk_end, n_chunks, N, H, E, part, status, s);
-    if (st != MOE_OK) return st;
-    MOE_TRACED("dense_router_wgrad_reduce", s, (dense_router_wgrad_reduce_kernel<T><<<(unsigned)cdiv((int64_t)H * E, 256),
-                                                   256, 0, s>>>(part, n_chunks, H, E, (T*)dWr)));
-    MOE_LAUNCH_CHECK();
-    return MOE_OK;
+    if (st == MOE_OK) st = router_wgrad_tc(x, Dh, N, H, E, dWr, part, status, s);
+    return st;
   }
   MOE_TRACED("router_dense_dlogits", s, (router_dense_dlogits_kernel<<<blocks, 256, 0, s>>>(
                                             probs, dlogit, top, routed_bins, N, E, K, coef, D, nullptr, nullptr, 1)));

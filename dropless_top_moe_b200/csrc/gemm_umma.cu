@@ -26,8 +26,8 @@
 //   ROWS   C[rows of group e, :] = A[rows, :] * B_e   (forward, dgrad)
 //   WGRAD  C_e = A[group e rows, :]^T * B[group e rows, :]   (weight grads;
 //          K = the group's padded rows, zero rows contribute nothing)
-//   DENSE  C = A * B over plain row tiles x column tiles (router logits, the
-//          dense router backward)
+//   DENSE  C = A * B over plain row tiles x column tiles (the dense router
+//          backward's D * W_r^T)
 // Every accumulation runs in a fixed order (k-steps in sequence, no split-K
 // across CTAs), so results are bitwise reproducible.  Every wait is bounded
 // (status bit MOE_DEVERR_TIMEOUT); no TMA load uses multicast.
@@ -47,7 +47,6 @@ constexpr int BM = 128;
 constexpr int BK = 64;              // one 128-byte swizzle row of bf16
 constexpr int kEpiWarps = 8;              // two warps per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kA_BYTES = BM * BK * 2;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 // M units per raster group (L2 reuse of the weight panels): 4 units of 256
 // rows, about one expert's rows at the training step's 1024 tokens per
@@ -56,7 +55,7 @@ constexpr int kGroupM = 4;
 
 enum Sched { SCHED_ROWS = 0, SCHED_WGRAD = 1, SCHED_DENSE = 2 };
 enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3, EPI_WGRAD_PAIR = 4,
-           EPI_ROUTER = 5, EPI_ROUTER_DX = 6, EPI_WGRAD_F32 = 7 };
+           EPI_ROUTER_DX = 6 };
 enum Split { SPLIT_NONE = 0, SPLIT_K = 1, SPLIT_N = 2 };
 
 struct Params {
@@ -84,11 +83,6 @@ struct Params {
   const __nv_bfloat16* aux1;
   int64_t ldo;        // row stride (elements) of out* / aux*
   int64_t out_estride;// WGRAD: elements between consecutive experts' outputs
-  float* logits;      // DENSE router outputs
-  float* probs;
-  int32_t* top;
-  float* weights;
-  int K;
   int* status;
 };
 
@@ -222,88 +216,6 @@ __device__ __forceinline__ void load_row_bf16x32(const __nv_bfloat16* src, float
     v[8 * q + 2] = bf16_lo(w.y); v[8 * q + 3] = bf16_hi(w.y);
     v[8 * q + 4] = bf16_lo(w.z); v[8 * q + 5] = bf16_hi(w.z);
     v[8 * q + 6] = bf16_lo(w.w); v[8 * q + 7] = bf16_hi(w.w);
-  }
-}
-
-template <int KMAX>
-__device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals)[KMAX], int (&ids)[KMAX]) {
-  // Descending list; strict '>' keeps an earlier (lower-id) equal value above.
-#pragma unroll
-  for (int j = KMAX - 1; j >= 0; --j) {
-    if (j < K && v > vals[j]) {
-      if (j > 0 && v > vals[j - 1]) {
-        vals[j] = vals[j - 1];
-        ids[j] = ids[j - 1];
-      } else {
-        vals[j] = v;
-        ids[j] = id;
-      }
-    }
-  }
-}
-
-// Router epilogue for one token row: E fp32 logits in TMEM columns
-// [tacc, tacc + E) -> optional logits / probs, top-K ids (descending, ties to
-// the lower id) and renormalised weights exp(l_k - l_max) / sum_kept.
-template <int KMAX>
-__device__ __forceinline__ void router_row(const Params& p, uint32_t tacc, int64_t grow) {
-  const int E = p.E, K = p.K;     // MMA columns beyond E (padding to 16) are ignored
-  const bool live = grow < p.P;
-  float vals[KMAX];
-  int ids[KMAX];
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
-  float m = -INFINITY;
-#pragma unroll 1
-  for (int c = 0; c < E; c += 32) {
-    uint32_t r[32];
-    tmem_ld_32(tacc + c, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (c + j < E) {
-        const float v = __uint_as_float(r[j]);
-        m = fmaxf(m, v);
-        topk_insert<KMAX>(v, c + j, K, vals, ids);
-        if (live && p.logits) p.logits[grow * E + c + j] = v;
-      }
-    }
-  }
-  if (p.probs) {
-    float Z = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < E; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32(tacc + c, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (c + j < E) Z += expf(__uint_as_float(r[j]) - m);
-    }
-#pragma unroll 1
-    for (int c = 0; c < E; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32(tacc + c, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (live && c + j < E) p.probs[grow * E + c + j] = expf(__uint_as_float(r[j]) - m) / Z;
-    }
-  }
-  if (live) {
-    float S = 0.f, ev[KMAX];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      ev[j] = (j < K) ? expf(vals[j] - vals[0]) : 0.f;
-      S += ev[j];
-    }
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j < K) {
-        p.top[grow * K + j] = ids[j];
-        p.weights[grow * K + j] = ev[j] / S;
-      }
-    }
   }
 }
 
@@ -444,7 +356,7 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       store_row_bf16x32(p.out0 + off + c, dg);
       store_row_bf16x32(p.out1 + off + c, du);
     }
-  } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR || EPI == EPI_WGRAD_F32) {
+  } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) {
     const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
 #pragma unroll 1
     for (int c = c_begin; c < c_end; c += 32) {
@@ -454,12 +366,7 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       float v[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-      if constexpr (EPI == EPI_WGRAD_F32) {
-        // fp32 partial sums (one slice per group, reduced in order afterwards)
-        float4* d = reinterpret_cast<float4*>(p.logits + off + c);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      } else if (scratch) {
+      if (scratch) {
         // rows are output rows m0 + row (lane i: m0 + row - lane + i)
         const int64_t o = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row - lane) * p.ldo + tl.n0;
         if (EPI == EPI_WGRAD_PAIR && c >= BN / 2) store_chunk_coalesced(scratch, lane, p.out1 + o + (c - BN / 2), p.ldo, v);
@@ -486,10 +393,6 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
         store_row_bf16x32(p.out0 + grow * p.ldo + tl.n0 + c, v);
       }
     }
-  } else {  // EPI_ROUTER: softmax, top-K, renormalise on this row's E logits
-    if (part != 0) return;
-    if (p.K <= 8) router_row<8>(p, tacc, grow);
-    else router_row<16>(p, tacc, grow);
   }
 }
 
@@ -902,13 +805,6 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
                 store_row_bf16x32(p.out0 + off + c, z);
                 store_row_bf16x32(p.out1 + off + c, z);
               }
-            } else if constexpr (EPI == EPI_WGRAD_F32) {
-#pragma unroll 1
-              for (int c = part * (BN / 2); c < (part + 1) * (BN / 2); c += 32) {
-                float4* d = reinterpret_cast<float4*>(p.logits + off + c);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) d[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-              }
             } else {
 #pragma unroll 1
               for (int c = part * (BN / 2); c < (part + 1) * (BN / 2); c += 32) store_row_bf16x32(p.out0 + off + c, z);
@@ -1284,43 +1180,6 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
   return MOE_OK;
 }
 
-// ---- router on tensor cores -----------------------------------------------
-
-bool route_umma_supported(int N, int H, int E, int K) {
-  (void)N;
-  return E >= 1 && E <= 256 && K <= 16 && H % 64 == 0;
-}
-
-size_t route_umma_scratch(int H, int E) { return (size_t)round_up(E < 16 ? 16 : E, 16) * H * 2; }
-
-moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K, float* logits,
-                      float* probs, int32_t* top, float* w, void* scratch, int* status, cudaStream_t s) {
-  Params p = blank_params(nullptr, E, N, status);
-  if (!map2d(&p.ta0, x, H, N, H, 64, 128)) return MOE_ERR_CUDA;
-  const bool mn = E % 64 == 0;
-  // MMA N: E rounded up to 16 (the smallest M = 128 MMA width); the extra
-  // columns read zeros (out-of-bounds rows of the K-major map) and are ignored
-  const int n_mma = E < 16 ? 16 : (int)round_up(E, 16);
-  if (mn) {
-    // B operand MN-major straight from W_r [H, E]: 64-expert boxes
-    if (!map2d(&p.tb0, W_r, E, H, E, 64, 64)) return MOE_ERR_CUDA;
-  } else {
-    // B operand K-major: W_r^T [E, H] kept in the workspace
-    moe_status st = transpose_matrix(W_r, H, E, MOE_BF16, scratch, s, n_mma);   // rows E.. are 0
-    if (st != MOE_OK) return st;
-    if (!map2d(&p.tb0, scratch, H, n_mma, H, 64, (uint32_t)n_mma)) return MOE_ERR_CUDA;
-  }
-  p.kdim = H;
-  p.n_mma = n_mma;
-  p.K = K;
-  p.logits = logits;
-  p.probs = probs;
-  p.top = top;
-  p.weights = w;
-  if (mn) return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER, false, true, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
-  return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER, false, false, SPLIT_NONE>("route_umma", p, cdiv(N, BM), s);
-}
-
 // ---- dense router backward on tensor cores ----------------------------------
 
 bool router_bwd_umma_supported(int H, int E) { return E % 64 == 0 && E <= 256 && H % 256 == 0; }
@@ -1340,24 +1199,6 @@ moe_status router_dx_umma(const void* D, const void* W_r, int N, int H, int E, v
   p.ldo = H;
   return launch<256, 1, 1, SCHED_DENSE, EPI_ROUTER_DX, false, false, SPLIT_NONE>(
       "dense_router_dx", p, cdiv(N, BM) * p.n_tiles, s);
-}
-
-// dW_r partials: part[c] = x[chunk c]^T * D[chunk c] for token chunks whose
-// ends (multiples of 64, the last = N rounded up to 64) are chunk_end[c], one
-// weight-gradient group per chunk; x [N, H] and D [N, E] both MN-major, the
-// tokens past N read as zeros.  part: [n_chunks, H, E] fp32.
-moe_status router_wgrad_umma(const void* x, const void* D, const int32_t* chunk_end, int n_chunks, int N,
-                             int H, int E, float* part, int* status, cudaStream_t s) {
-  Params p = blank_params(chunk_end, n_chunks, round_up(N, BK), status);
-  if (!map2d(&p.ta0, x, H, N, H, 64, 64) || !map2d(&p.tb0, D, E, N, E, 64, 64)) return MOE_ERR_CUDA;
-  p.n_mma = 64;
-  p.m_tiles_w = H / BM;
-  p.n_tiles = E / 64;
-  p.logits = part;
-  p.ldo = E;
-  p.out_estride = (int64_t)H * E;
-  return launch<64, 1, 1, SCHED_WGRAD, EPI_WGRAD_F32, true, true, SPLIT_NONE>(
-      "dense_router_wgrad", p, (int64_t)n_chunks * p.m_tiles_w * p.n_tiles, s);
 }
 
 }  // namespace moe

