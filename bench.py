@@ -647,14 +647,17 @@ def _cores():
         return os.cpu_count()
 
 
-def _oracle_cost(shape, o, rng):
-    """Fixed per-call and per-token seconds of one oracle pass on this host.
+def _size_sample(shape, o, rng, target_s):
+    """Token count of an oracle pass that takes about target_s seconds on
+    this host, found by timing passes of growing seeded samples.
 
-    A pass has a cost that does not depend on its token count (the backward
-    zero-fills dense float64 weight gradients of E*H*F elements each, several
-    GB at the training-step sizes) plus a cost per token; two probes of
-    different sizes separate them, so that a timed pass can be sized to make
-    the fixed part small."""
+    A pass does not cost in proportion to its tokens while the sample is
+    small: the backward zero-fills dense float64 weight gradients (E*H*F
+    elements each, several GB at the training-step sizes) and every expert
+    a sample touches streams its float64 weights.  So the sample grows from
+    256 tokens, each next size extrapolated from the last two passes, until
+    a pass takes at least half the target (or the sample is the whole
+    batch).  Returns (tokens, seconds) of that last pass."""
     import numpy as np
 
     def timed(n):
@@ -662,37 +665,29 @@ def _oracle_cost(shape, o, rng):
         t0 = time.perf_counter()
         _oracle_step(shape, o, tok)
         return time.perf_counter() - t0
-    n0, n1 = min(8, shape.N), min(128, shape.N)
-    t0 = timed(n0)
-    t1 = timed(n1) if n1 > n0 else t0
-    per_tok = max((t1 - t0) / max(n1 - n0, 1), t1 / max(n1, 1) * 0.05, 1e-7)
-    fixed = max(t0 - n0 * per_tok, 0.0)
-    return fixed, per_tok
 
-
-def _sample_tokens(shape, fixed, per_tok, target_s):
-    """Tokens of one pass that takes about target_s seconds (at least the
-    probe's size, at most the workload's N)."""
-    n = int((target_s - fixed) / per_tok)
-    return max(min(shape.N, 128), min(shape.N, n))
+    n, prev = min(256, shape.N), None
+    while True:
+        dt = timed(n)
+        if dt >= 0.5 * target_s or n >= shape.N:
+            return n, dt
+        guess = 4 * n
+        if prev is not None and dt > prev[1] and n > prev[0]:
+            guess = n + (target_s - dt) * (n - prev[0]) / (dt - prev[1])
+        prev = (n, dt)
+        n = int(min(shape.N, max(1.5 * n, min(guess, 8 * n))))
 
 
 def cpu_baseline(shape, inp=None, target_s=10.0, o=None):
     """The oracle, as it stands, on one bounded token sample of the workload,
-    sized so that one pass takes about target_s seconds (its fixed per-call
-    cost then weighs little in the tokens/s)."""
+    grown until one pass takes about target_s seconds (its fixed per-call
+    costs then weigh little in the tokens/s); the last pass is the number."""
     import numpy as np
     o = o if o is not None else _oracle_inputs(shape, inp)
-    rng = np.random.default_rng(0)
-    fixed, per_tok = _oracle_cost(shape, o, rng)
-    n = _sample_tokens(shape, fixed, per_tok, target_s)
-    tok = np.sort(rng.choice(shape.N, n, replace=False))
-    t0 = time.perf_counter()
-    _oracle_step(shape, o, tok)
-    dt = time.perf_counter() - t0
+    n, dt = _size_sample(shape, o, np.random.default_rng(0), target_s)
     return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
             "sample": f"{n} of {shape.N} tokens of {shape.name} ({'fwd+bwd' if shape.training else 'fwd'}), "
-                      f"float64 numpy oracle, {dt:.1f} s (fixed per-call cost {fixed:.1f} s)"}
+                      f"float64 numpy oracle, {dt:.1f} s"}
 
 
 def run_reference(args, rank, world):
@@ -700,18 +695,17 @@ def run_reference(args, rank, world):
 
     Each timed step is one oracle pass over a seeded token sample sized, like
     the in-line CPU baseline, to about 10 s (less when many steps would run
-    past about 200 s of timed work), so that the oracle's fixed per-call cost
-    does not dominate its tokens/s.  Warm-up steps use a small sample: they
-    are untimed and only warm the host caches and allocator."""
+    past about 200 s of timed work), so that the oracle's fixed per-call
+    costs do not dominate its tokens/s.  Warm-up steps use a small sample:
+    they are untimed and only warm the host caches and allocator."""
     import numpy as np
     if rank != 0:
         return None
     shape = workload(args)
     o = _oracle_inputs(shape)
     rng = np.random.default_rng(1)
-    fixed, per_tok = _oracle_cost(shape, o, rng)
     target = min(10.0, 200.0 / max(args.steps, 1))
-    n = _sample_tokens(shape, fixed, per_tok, target)
+    n, _ = _size_sample(shape, o, rng, target)
     for _ in range(args.warmup):
         _oracle_step(shape, o, np.sort(rng.choice(shape.N, min(16, shape.N), replace=False)))
     t0 = time.perf_counter()
@@ -720,8 +714,7 @@ def run_reference(args, rank, world):
     dt = time.perf_counter() - t0
     v = n * args.steps / dt
     ms = dt / args.steps * 1e3
-    sample = (f"{n} of {shape.N} tokens per step (seeded), float64 numpy oracle; fixed per-call cost "
-              f"{fixed:.1f} s, {per_tok * 1e3:.2f} ms per token")
+    sample = f"{n} of {shape.N} tokens per step (seeded), float64 numpy oracle, {dt / args.steps:.1f} s per step"
     return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -56,8 +56,18 @@ struct LayerWs {
   size_t total;
 };
 
-size_t route_scratch_bytes(int H, int E, moe_dtype dt) {
-  return dt == MOE_BF16 ? route_umma_scratch(H, E) : 0;
+bool routes_on_tensor_cores(int N, int H, int E, int K, moe_dtype dt) {
+  return dt == MOE_BF16 && route_umma_supported(N, H, E, K);
+}
+
+size_t route_scratch_bytes(int N, int H, int E, int K, moe_dtype dt) {
+  return routes_on_tensor_cores(N, H, E, K, dt) ? route_umma_scratch(N, H, E, K) : 0;
+}
+
+// Tokens per dispatch-metadata chunk in the layer: the tensor-core router
+// counts each of its chunks' expert ids; otherwise the metadata counts 128.
+int layer_meta_chunk(int N, int H, int E, int K, moe_dtype dt) {
+  return routes_on_tensor_cores(N, H, E, K, dt) ? route_chunk_tokens(N, H, E, K) : 128;
 }
 
 // training: mode 0 / 1 / 2 in the low bits, MOE_LAYER_GATHER_ROWS (bf16 only) on top
@@ -94,8 +104,8 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int f
     return r;
   };
   w.status = (int*)take(kStatusBytes);
-  w.route_scratch = take(route_scratch_bytes(H, E, dt));
-  w.meta_scratch = take(meta_workspace_bytes(N, E));
+  w.route_scratch = take(route_scratch_bytes(N, H, E, K, dt));
+  w.meta_scratch = take(meta_workspace_bytes(N, E, layer_meta_chunk(N, H, E, K, dt)));
   w.routed_bins = (int32_t*)take((size_t)E * 4);
   w.pos = (int32_t*)take(NK * 4);
   w.probs = (float*)take((size_t)N * E * 4);
@@ -115,10 +125,6 @@ LayerWs carve(void* base, int N, int H, int E, int K, int F, moe_dtype dt, int f
   }
   w.total = off;
   return w;
-}
-
-bool routes_on_tensor_cores(int N, int H, int E, int K, moe_dtype dt) {
-  return dt == MOE_BF16 && route_umma_supported(N, H, E, K);
 }
 
 // chunk_counts: with the tensor-core router, also the per-128-token expert
@@ -172,8 +178,8 @@ int64_t moe_padded_rows_max(int32_t N, int32_t E, int32_t K) {
 }
 
 size_t moe_route_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, moe_dtype dt) {
-  (void)N; (void)K;
-  return al256(kStatusBytes) + al256(route_scratch_bytes(H, E, dt));
+  if (check_shape(N, H, E, K, dt) != MOE_OK) return 0;
+  return al256(kStatusBytes) + al256(route_scratch_bytes(N, H, E, K, dt));
 }
 
 size_t moe_dispatch_meta_workspace_size(int32_t N, int32_t K, int32_t E) {
@@ -370,7 +376,7 @@ moe_status moe_layer_fwd(const void* x, const void* W_r, const void* W1, const v
   MOE_TRY(route_any(x, W_r, N, H, E, K, dt, nullptr, aux ? w.probs : nullptr, top_experts, weights,
                     w.route_scratch, w.status, s, counted ? (int32_t*)w.meta_scratch : nullptr));
   MOE_TRY(dispatch_meta(top_experts, N, K, E, indices, nullptr, bins, padded_bins, w.pos, w.meta_scratch,
-                        w.status, s, capacity, w.routed_bins, counted));
+                        w.status, s, capacity, w.routed_bins, counted, layer_meta_chunk(N, H, E, K, dt)));
   // f_i of the loss counts routed assignments, dropped ones included
   if (aux) MOE_TRY(aux_loss_fwd(w.probs, w.routed_bins, N, K, E, aux_alpha, aux_loss, nullptr, w.aux_scratch, s));
   if (N == 0) return MOE_OK;

@@ -18,23 +18,25 @@ moe_status router_wgrad_tc(const void* x, const void* Dh, int N, int H, int E, v
                            int* status, cudaStream_t s);
 
 // router.cu - tensor-core router (bf16, E <= 256, H % 64 == 0).  With
-// chunk_counts it also writes the per-128-token expert counts of the dispatch
-// metadata ([ceil(N/128)][E], see dispatch_meta).
+// chunk_counts it also writes the per-chunk expert counts of the dispatch
+// metadata ([ceil(N / T)][E], T = route_chunk_tokens tokens per chunk, see
+// dispatch_meta).
 bool route_umma_supported(int N, int H, int E, int K);
-size_t route_umma_scratch(int H, int E);
+int route_chunk_tokens(int N, int H, int E, int K);
+size_t route_umma_scratch(int N, int H, int E, int K);
 moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K, float* logits,
                       float* probs, int32_t* top, float* w, void* scratch, int* status,
                       cudaStream_t s, int32_t* chunk_counts = nullptr);
 
-// meta.cu - metadata over chunks of 128 tokens.  Scratch: per-chunk expert
-// counts [meta_chunks(N)][E] (which the bf16 router can fill, counts_ready),
-// then 2*E ints.
-int64_t meta_chunks(int64_t N);
-size_t meta_workspace_bytes(int64_t N, int E);
+// meta.cu - metadata over chunks of T tokens (T a power of two <= 128).
+// Scratch: per-chunk expert counts [meta_chunks(N, T)][E] (which the bf16
+// router can fill with its own chunking: counts_ready), then 2*E ints.
+int64_t meta_chunks(int64_t N, int T = 128);
+size_t meta_workspace_bytes(int64_t N, int E, int T = 128);
 moe_status dispatch_meta(const int32_t* top, int64_t N, int K, int E, int32_t* indices, int32_t* bin_ids,
                          int32_t* bins, int32_t* padded_bins, int32_t* pos, void* scratch, int* status,
                          cudaStream_t s, int capacity = 0, int32_t* routed_bins = nullptr,
-                         bool counts_ready = false);
+                         bool counts_ready = false, int T = 128);
 
 // permute.cu
 moe_status permute_rows(const void* x, const int32_t* pos, const int32_t* bins, const int32_t* pb,

@@ -4,8 +4,8 @@
 // expert id only, a few bits).
 //
 // A counting sort is the whole sort when keys are at most 8 bits wide.  The
-// assignments are cut into chunks of 128 tokens (128*K flat ids, the router's
-// row tile):
+// assignments are cut into chunks of T tokens (T*K flat ids; T = 128, or the
+// router's chunk when it supplies the counts):
 //   count  - per chunk, a shared-memory histogram of its expert ids (integer
 //            atomics: a count does not depend on their order).  The bf16
 //            layer skips this launch: its router epilogue writes the same
@@ -30,7 +30,6 @@
 
 namespace moe {
 
-constexpr int kMetaTok = 128;            // tokens per chunk (the router's row tile)
 constexpr int kMetaThreads = 1024;       // place / scan blocks
 constexpr int64_t kInlineScanReads = int64_t(1) << 22;   // counts read over the grid by step (a)
 
@@ -40,15 +39,15 @@ __host__ __device__ inline int pow2_at_least(int v) {
   return p;
 }
 
-int64_t meta_chunks(int64_t N) { return cdiv(N > 0 ? N : 1, kMetaTok); }
+int64_t meta_chunks(int64_t N, int T) { return cdiv(N > 0 ? N : 1, T); }
 
 __global__ void __launch_bounds__(256)
-meta_count_kernel(const int32_t* __restrict__ top, int64_t NK, int K, int E, int32_t* __restrict__ chunk_counts,
-                  int* status) {
+meta_count_kernel(const int32_t* __restrict__ top, int64_t NK, int K, int E, int T,
+                  int32_t* __restrict__ chunk_counts, int* status) {
   extern __shared__ int s_hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
-  const int64_t per = (int64_t)kMetaTok * K;
+  const int64_t per = (int64_t)T * K;
   const int64_t base = (int64_t)blockIdx.x * per;
   const int64_t end = base + per < NK ? base + per : NK;
   for (int64_t i0 = base + threadIdx.x; i0 < end; i0 += 4 * (int64_t)blockDim.x) {
@@ -153,7 +152,7 @@ meta_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks, int E, int ca
 // exclusive offsets and starts the expert starts (meta_scan_kernel).
 template <bool INLINE>
 __global__ void __launch_bounds__(kMetaThreads)
-meta_place_kernel(const int32_t* __restrict__ top, int64_t NK, int K, int E, int n_chunks, int capacity,
+meta_place_kernel(const int32_t* __restrict__ top, int64_t NK, int K, int E, int T, int n_chunks, int capacity,
                   const int32_t* __restrict__ chunk_counts, const int32_t* __restrict__ starts,
                   int32_t* __restrict__ bins, int32_t* __restrict__ padded_bins, int32_t* __restrict__ routed_bins,
                   int32_t* __restrict__ indices, int32_t* __restrict__ bin_ids, int32_t* __restrict__ pos) {
@@ -203,8 +202,8 @@ meta_place_kernel(const int32_t* __restrict__ top, int64_t NK, int K, int E, int
   }
   __syncthreads();
   // (b) placement, in increasing flat id
-  const int64_t base = (int64_t)c * kMetaTok * K;
-  int64_t end = base + (int64_t)kMetaTok * K;
+  const int64_t base = (int64_t)c * T * K;
+  int64_t end = base + (int64_t)T * K;
   if (end > NK) end = NK;
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int64_t r0 = base; r0 < end; r0 += kMetaThreads) {
@@ -248,15 +247,15 @@ meta_place_kernel(const int32_t* __restrict__ top, int64_t NK, int K, int E, int
   }
 }
 
-size_t meta_workspace_bytes(int64_t N, int E) {
-  return (size_t)(meta_chunks(N) * E + 2 * E) * sizeof(int32_t);
+size_t meta_workspace_bytes(int64_t N, int E, int T) {
+  return (size_t)(meta_chunks(N, T) * E + 2 * E) * sizeof(int32_t);
 }
 
 moe_status dispatch_meta(const int32_t* top, int64_t N, int K, int E, int32_t* indices, int32_t* bin_ids,
                          int32_t* bins, int32_t* padded_bins, int32_t* pos, void* scratch, int* status,
-                         cudaStream_t s, int capacity, int32_t* routed_bins, bool counts_ready) {
+                         cudaStream_t s, int capacity, int32_t* routed_bins, bool counts_ready, int T) {
   const int64_t NK = N * K;
-  const int n_chunks = (int)meta_chunks(N);
+  const int n_chunks = (int)meta_chunks(N, T);
   int32_t* chunk_counts = (int32_t*)scratch;
   int32_t* starts = chunk_counts + (size_t)n_chunks * E;
   if (N == 0) {
@@ -267,20 +266,20 @@ moe_status dispatch_meta(const int32_t* top, int64_t N, int K, int E, int32_t* i
     return MOE_OK;
   }
   if (!counts_ready) {
-    MOE_TRACED("meta_count", s, (meta_count_kernel<<<n_chunks, 256, E * sizeof(int), s>>>(top, NK, K, E,
+    MOE_TRACED("meta_count", s, (meta_count_kernel<<<n_chunks, 256, E * sizeof(int), s>>>(top, NK, K, E, T,
                                                                                            chunk_counts, status)));
     MOE_LAUNCH_CHECK();
   }
   if ((int64_t)n_chunks * n_chunks * E <= kInlineScanReads) {
     MOE_TRACED("meta_place", s, (meta_place_kernel<true><<<n_chunks, kMetaThreads, 0, s>>>(
-                                    top, NK, K, E, n_chunks, capacity, chunk_counts, nullptr, bins, padded_bins,
+                                    top, NK, K, E, T, n_chunks, capacity, chunk_counts, nullptr, bins, padded_bins,
                                     routed_bins, indices, bin_ids, pos)));
   } else {
     MOE_TRACED("meta_scan", s, (meta_scan_kernel<<<1, kMetaThreads, 0, s>>>(chunk_counts, n_chunks, E, capacity,
                                                                            bins, padded_bins, routed_bins, starts)));
     MOE_LAUNCH_CHECK();
     MOE_TRACED("meta_place", s, (meta_place_kernel<false><<<n_chunks, kMetaThreads, 0, s>>>(
-                                    top, NK, K, E, n_chunks, capacity, chunk_counts, starts, nullptr, nullptr,
+                                    top, NK, K, E, T, n_chunks, capacity, chunk_counts, starts, nullptr, nullptr,
                                     nullptr, indices, bin_ids, pos)));
   }
   MOE_LAUNCH_CHECK();

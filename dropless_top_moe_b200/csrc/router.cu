@@ -1,24 +1,27 @@
 // Tensor-core router for bf16 layers: logits = x W_r, softmax, top-K (equal
 // values to the lower expert id), renormalised weights ("MoE computation
-// principle and execution", sec. 2.1-2.2), plus the per-128-token expert
+// principle and execution", sec. 2.1-2.2), plus the per-chunk expert
 // histogram the dispatch metadata starts from ("MegaBlocks - architecture",
 // sec. 2.3: histogram of the sorted expert ids).
 //
 // The router reads x once and does little arithmetic per byte (E FLOP per
-// byte of x), so it is bound by HBM unless too few CTAs stream x.  One
-// 128-token row tile is split along H over a cluster of S CTAs (S = 1..8,
-// chosen so that the grid fills the SMs): CTA r multiplies its contiguous
-// share of the 64-wide k blocks on the tensor cores (TMA -> shared memory ->
-// tcgen05.mma, fp32 accumulators in TMEM), writes its 128 x E partial logits
-// into its own shared memory, and after a cluster barrier every CTA sums the
-// S partials of a slice of the rows, in the fixed order r = 0..S-1, through
-// distributed shared memory.  No global scratch, no atomics on floats, so the
-// logits are the same bits on every run.
+// byte of x), so it is bound by HBM as long as enough CTAs stream x.  A CTA
+// multiplies one 128-token row tile (TMA -> shared memory -> tcgen05.mma,
+// fp32 accumulators in TMEM), one CTA per SM.  When the row tiles are too
+// few to fill the GPU (small N), a tile's H is split over a cluster of S CTAs
+// (S = 2..8):
+// each writes its 128 x E partial logits to a global scratch (it stays in
+// L2), a cluster barrier publishes them, and CTA r then finishes rows
+// [r*128/S, (r+1)*128/S) of the tile, summing the S partials in the fixed
+// order s = 0..S-1.  S depends only on N, H, E and K, never on the device, so
+// the logits are the same bits on every run.
 //
 // Warps: 0 TMA producer, 1 TMEM owner and MMA issuer, 2-5 TMEM -> shared
-// memory; then one thread per row finishes the rows of this CTA's share:
-// the sum of the partials, max, a sorted top-K list (ties to the lower id),
-// softmax when asked, renormalisation.  Every mbarrier wait is bounded
+// memory (S = 1) or global scratch; then one thread per row finishes a row:
+// the sum of the partials, the max, a sorted top-K list (ties to the lower
+// id), the softmax when asked, the renormalisation, and its experts into this
+// CTA's histogram (integer shared-memory atomics), which is written as the
+// count row of the CTA's 128/S-token chunk.  Every mbarrier wait is bounded
 // (MOE_DEVERR_TIMEOUT); no TMA load uses multicast.
 //
 // B operand: W_r [H, E] is read MN-major straight from the caller's matrix
@@ -42,6 +45,7 @@ constexpr int kRBK = 64;                   // k block (one 128-byte swizzle row 
 constexpr int kRouteThreads = 192;
 constexpr int kA = kRows * kRBK * 2;       // A bytes per stage
 constexpr uint64_t kRouteTimeoutNs = 2000000000ull;
+constexpr int kRouteSlots = 148;           // SMs the split aims to fill (fixed: results must not depend on the GPU)
 
 struct RouteParams {
   CUtensorMap tx;          // x [N, H]: 64 x 128 boxes
@@ -49,20 +53,22 @@ struct RouteParams {
   int N, H, E, K;
   int n_mma;               // MMA N: E rounded up to 16
   int nkb;                 // k blocks over H
+  float* part;             // S > 1: partial logits [S][N][n_mma]
   float* logits;
   float* probs;
   int32_t* top;
   float* weights;
-  int32_t* chunk_counts;   // [tiles][E] or NULL
+  int32_t* chunk_counts;   // [tiles * S][E] or NULL
   int* status;
 };
 
 template <int EPT>
 struct RouteShape {
-  static constexpr int NB = EPT == 8 ? 4 : (EPT == 4 ? 2 : 1);    // 64-column B boxes
-  static constexpr int B_BYTES = NB * 8192;
-  static constexpr int STAGE = kA + B_BYTES;
-  static constexpr int STAGES = NB == 2 ? 3 : 4;
+  static constexpr int NB = EPT == 8 ? 4 : (EPT == 4 ? 2 : 1);    // 64-column B boxes per k block
+  static constexpr int KB = 1;                                     // k blocks per stage
+  static constexpr int B_BYTES = NB * 8192;                        // per k block
+  static constexpr int STAGE = KB * (kA + B_BYTES);
+  static constexpr int STAGES = (192 * 1024) / STAGE;              // one CTA per SM
   static constexpr int STRIDE = EPT * 32 + 1;   // partial-logit row stride (floats), odd: no bank conflicts
   static constexpr int PART_BYTES = kRows * STRIDE * 4;
   static_assert(PART_BYTES <= STAGES * STAGE, "partial logits reuse the pipeline buffers");
@@ -75,15 +81,8 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
 }
-// Generic address of the same shared-memory location in CTA `rank` of this
-// cluster: ordinary loads through it read the peer's shared memory, and the
-// compiler may batch them (they are ordered after the cluster barrier like
-// any other memory access).
-template <typename T>
-__device__ __forceinline__ const T* peer_ptr(const T* p, uint32_t rank) {
-  uint64_t r;
-  asm("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"((uint64_t)p), "r"(rank));
-  return reinterpret_cast<const T*>(r);
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 // Insert (v, id) into a descending list of the K largest; a strict '>' keeps
@@ -104,15 +103,9 @@ __device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals
     }
   }
 }
-__device__ __forceinline__ void red_cluster_add(uint32_t addr, uint32_t v) {
-  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
 
 template <int EPT, bool B_MN, int KMAX>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_constant__ RouteParams p) {
+__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_constant__ RouteParams p) {
   using S_ = RouteShape<EPT>;
   constexpr int STAGES = S_::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -125,16 +118,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_const
   const uint32_t tfull = bar_base + 8u * (2 * STAGES);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * S_::STAGE + 8 * (2 * STAGES + 1));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  uint32_t* s_hist = tmem_holder + 4;                 // [256] this tile's expert counts (rank 0's)
-  const uint32_t part = base;                          // partial logits, after the main loop
+  int* s_hist = reinterpret_cast<int*>(tmem_holder + 4);    // [256] expert counts of this CTA's rows
+  const uint32_t part = base;                                 // S = 1: partial logits, after the main loop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t S = cluster_nctarank();
   const uint32_t rank = cluster_ctarank();
   const int tile = (int)cluster_id_x();
   const int row0 = tile * kRows;
-  // this CTA's contiguous share of the k blocks
-  const int q = p.nkb / (int)S, rem = p.nkb % (int)S;
+  // this CTA's contiguous share of the stages of KB k blocks
+  const int q = (p.nkb / S_::KB) / (int)S, rem = (p.nkb / S_::KB) % (int)S;
   const int kb0 = (int)rank * q + ((int)rank < rem ? (int)rank : rem);
   const int nk = q + ((int)rank < rem ? 1 : 0);
 
@@ -161,20 +154,26 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_const
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      const uint32_t tx_bytes = kA + (B_MN ? S_::B_BYTES : (uint32_t)p.n_mma * kRBK * 2);
+      const uint32_t tx_bytes = S_::KB * (kA + (B_MN ? S_::B_BYTES : (uint32_t)p.n_mma * kRBK * 2));
       int stage = 0;
       uint32_t phase = 0;
       for (int i = 0; i < nk; ++i) {
         if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kRouteTimeoutNs)) break;
-        const uint32_t sa = base + stage * S_::STAGE, sb = sa + kA;
-        const int k = (kb0 + i) * kRBK;
+        const uint32_t sa0 = base + stage * S_::STAGE;
         mbar_expect_tx(full_bar(stage), tx_bytes);
-        tma_load_2d(sa, &p.tx, full_bar(stage), k, row0);
-        if constexpr (B_MN) {
 #pragma unroll
-          for (int j = 0; j < S_::NB; ++j) tma_load_2d(sb + j * 8192, &p.tw, full_bar(stage), 64 * j, k);
-        } else {
-          tma_load_2d(sb, &p.tw, full_bar(stage), k, 0);
+        for (int b = 0; b < S_::KB; ++b)     // x first: the row pieces of one stage back to back
+          tma_load_2d(sa0 + b * kA, &p.tx, full_bar(stage), ((kb0 + i) * S_::KB + b) * kRBK, row0);
+#pragma unroll
+        for (int b = 0; b < S_::KB; ++b) {
+          const uint32_t sb = sa0 + S_::KB * kA + b * S_::B_BYTES;
+          const int k = ((kb0 + i) * S_::KB + b) * kRBK;
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int j = 0; j < S_::NB; ++j) tma_load_2d(sb + j * 8192, &p.tw, full_bar(stage), 64 * j, k);
+          } else {
+            tma_load_2d(sb, &p.tw, full_bar(stage), k, 0);
+          }
         }
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
@@ -189,12 +188,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_const
       for (int i = 0; i < nk; ++i) {
         if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status, kRouteTimeoutNs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sa = base + stage * S_::STAGE, sb = sa + kA;
+        const uint32_t sa0 = base + stage * S_::STAGE;
 #pragma unroll
-        for (int kk = 0; kk < kRBK / 16; ++kk) {
-          const uint64_t ad = desc_k_sw128(sa + kk * 32);
-          const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
-          mma_bf16(tmem_base, ad, bd, idesc, (i | kk) != 0 ? 1u : 0u);
+        for (int b = 0; b < S_::KB; ++b) {
+          const uint32_t sa = sa0 + b * kA, sb = sa0 + S_::KB * kA + b * S_::B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kRBK / 16; ++kk) {
+            const uint64_t ad = desc_k_sw128(sa + kk * 32);
+            const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
+            mma_bf16(tmem_base, ad, bd, idesc, (i | b | kk) != 0 ? 1u : 0u);
+          }
         }
         mma_commit(empty_bar(stage));
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -203,16 +206,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_const
       else *abort_flag = 1;
     }
   } else {
-    // ------------------------------------------------ TMEM -> partial logits
+    // --------------------------------- TMEM -> partial logits (smem or global)
     int ok = 0;
     if (lane == 0) ok = mbar_wait_bounded(tfull, 0, abort_flag, p.status, kRouteTimeoutNs) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     tc_fence_after();
     const int qd = warp & 3;                       // TMEM lane quarter of this warp
     const int row = qd * 32 + lane;
+    const int64_t t = (int64_t)row0 + row;
     const uint32_t dst = part + (uint32_t)(row * S_::STRIDE) * 4u;
 #pragma unroll
     for (int c = 0; c < EPT; ++c) {
+      if (c * 32 >= p.n_mma) break;
       uint32_t r[32];
       if (ok) {
         tmem_ld_32(tmem_base + ((uint32_t)(qd * 32) << 16) + (uint32_t)(c * 32), r);
@@ -221,23 +226,33 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_const
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = 0u;
       }
+      if (S == 1) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) st_shared_f32(dst + (uint32_t)(c * 32 + j) * 4u, __uint_as_float(r[j]));
+        for (int j = 0; j < 32; ++j) st_shared_f32(dst + (uint32_t)(c * 32 + j) * 4u, __uint_as_float(r[j]));
+      } else if (t < p.N) {
+        // n_mma is a multiple of 16: whole 16-column halves of the chunk
+        float4* g = reinterpret_cast<float4*>(p.part + ((size_t)rank * p.N + t) * p.n_mma + c * 32);
+        const int nv = (p.n_mma - c * 32) >= 32 ? 8 : 4;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < nv)
+            g[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                               __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+      }
     }
   }
   tc_fence_before();
-  cluster_sync();     // every CTA's partial logits and zeroed histogram visible to the cluster
+  if (S > 1) cluster_sync();     // every CTA's partial logits published (release / acquire, cluster scope)
+  else __syncthreads();
   tc_fence_after();
 
-  // ------------------------------------------------ rows: S partials -> routing
+  // ------------------------------------------------ rows: partials -> routing
   // One thread per row: CTA r finishes rows [r*R, (r+1)*R), R = 128 / S.
-  // Pass 1 sums the row's S partial logits (in the fixed order s = 0..S-1,
-  // through distributed shared memory), keeps the running max and a sorted
-  // top-K list, and writes the sums back into this CTA's own row (no other
-  // CTA reads this CTA's rows of its own range); the probabilities, when
-  // wanted, take two more passes over that local row.
+  // Pass 1 sums the row's partial logits (over s = 0..S-1 in order), keeps the
+  // running max and the sorted top-K list; the probabilities, when wanted,
+  // take two more passes over the summed row, kept in this CTA's own shared
+  // memory row (S = 1: in place; S > 1 the pipeline buffers are free).
   const int rows_per = kRows / (int)S;
-  const uint32_t hist0 = map_to_rank(smem_u32(s_hist), 0);
   if ((int)threadIdx.x < rows_per) {
     const int row = (int)rank * rows_per + (int)threadIdx.x;
     const int64_t t = (int64_t)row0 + row;
@@ -247,28 +262,33 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_const
       int ids[KMAX];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
-      float m = -INFINITY;
+
 #pragma unroll 1
       for (int c = 0; c < p.E; c += 32) {
         float v[32];
+        if (S == 1) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-        for (uint32_t s = 0; s < S; ++s) {
-          const float* src = peer_ptr(mine + c, s);
+          for (int j = 0; j < 32; ++j) v[j] = mine[c + j];
+        } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c + j < p.E) v[j] += src[j];
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          for (uint32_t s = 0; s < S; ++s) {
+            const float* src = p.part + ((size_t)s * p.N + t) * p.n_mma + c;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < p.n_mma) v[j] += src[j];
+          }
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           if (c + j < p.E) {
-            if (p.probs) mine[c + j] = v[j];
-            m = fmaxf(m, v[j]);
+            if (S > 1 && p.probs) mine[c + j] = v[j];
             topk_insert<KMAX>(v[j], c + j, p.K, vals, ids);
             if (p.logits) p.logits[t * p.E + c + j] = v[j];
           }
         }
       }
+      const float m = vals[0];   // the row's largest logit
       if (p.probs) {
         float Z = 0.f;
         for (int e = 0; e < p.E; ++e) Z += expf(mine[e] - m);
@@ -286,15 +306,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const __grid_const
         if (j < p.K) {
           p.top[t * p.K + j] = ids[j];
           p.weights[t * p.K + j] = ev[j] / Ssum;
-          if (p.chunk_counts) red_cluster_add(hist0 + (uint32_t)ids[j] * 4u, 1u);
+          if (p.chunk_counts) atomicAdd(&s_hist[ids[j]], 1);
         }
       }
     }
   }
-  cluster_sync();     // peers are done reading this CTA's partials; the histogram is complete
-  if (rank == 0 && p.chunk_counts) {
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x)
-      p.chunk_counts[(size_t)tile * p.E + e] = (int32_t)s_hist[e];
+  __syncthreads();
+  if (p.chunk_counts) {
+    // this CTA's rows are chunk tile * S + rank of 128 / S tokens; a chunk
+    // that starts at or past N does not exist (the last tile's trailing CTAs)
+    const int64_t chunk = (int64_t)tile * S + rank;
+    if (chunk * rows_per < p.N)
+      for (int e = threadIdx.x; e < p.E; e += blockDim.x) p.chunk_counts[chunk * p.E + e] = s_hist[e];
   }
   if (warp == 1) {
     __syncwarp();
@@ -333,17 +356,9 @@ bool map2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int device_sms() {
-  static int cache[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!cache[dev]) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
-  }
-  return cache[dev];
+int route_ept(int E) {
+  const int n_mma = (int)round_up(E, 16);
+  return n_mma <= 32 ? 1 : n_mma <= 64 ? 2 : n_mma <= 128 ? 4 : 8;
 }
 
 template <int EPT, bool B_MN, int KMAX>
@@ -388,10 +403,30 @@ moe_status launch_route(const RouteParams& p, int S, int tiles, cudaStream_t s) 
 
 bool route_umma_supported(int N, int H, int E, int K) {
   (void)N;
-  return E >= 1 && E <= 256 && K >= 1 && K <= 32 && K <= E && H % 64 == 0;
+  return E >= 1 && E <= 256 && K >= 1 && K <= 32 && K <= E && H % kRBK == 0;
 }
 
-size_t route_umma_scratch(int H, int E) { return E % 8 == 0 ? 0 : (size_t)round_up(E, 16) * H * 2; }
+// H slices per row tile: the largest power of two (up to 8) that keeps
+// tiles * S CTAs within one per SM, with at least four k blocks per slice.
+// (More CTAs than SMs would not shorten the busiest SM's share of x.)
+int route_split(int N, int H, int E, int K) {
+  (void)E;
+  (void)K;
+  const int tiles = (int)cdiv(N > 0 ? N : 1, kRows);
+  const int stages = H / kRBK;
+  int S = 1;
+  while (S < 8 && tiles * S * 2 <= kRouteSlots && stages / (S * 2) >= 4) S *= 2;
+  return S;
+}
+
+int route_chunk_tokens(int N, int H, int E, int K) { return kRows / route_split(N, H, E, K); }
+
+size_t route_umma_scratch(int N, int H, int E, int K) {
+  const size_t n_mma = (size_t)round_up(E, 16);
+  const size_t wt = E % 8 == 0 ? 0 : (size_t)round_up(n_mma * H * 2, 256);
+  const int S = route_split(N, H, E, K);
+  return wt + (S > 1 ? (size_t)S * N * n_mma * sizeof(float) : 0);
+}
 
 moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K, float* logits, float* probs,
                       int32_t* top, float* w, void* scratch, int* status, cudaStream_t s, int32_t* chunk_counts) {
@@ -399,8 +434,9 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   RouteParams p;
   memset(&p, 0, sizeof(p));
   const int n_mma = (int)round_up(E, 16);
-  const int ept = n_mma <= 32 ? 1 : n_mma <= 64 ? 2 : n_mma <= 128 ? 4 : 8;
+  const int ept = route_ept(E);
   const bool mn = E % 8 == 0;
+  const size_t wt_bytes = mn ? 0 : (size_t)round_up((int64_t)n_mma * H * 2, 256);
   if (!map2d(&p.tx, x, H, N, 64, kRows)) return MOE_ERR_CUDA;
   if (mn) {
     // MN-major B straight from W_r [H, E]: 64-expert boxes, experts past E read as zeros
@@ -417,19 +453,15 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   p.K = K;
   p.n_mma = n_mma;
   p.nkb = H / kRBK;
+  p.part = (float*)((char*)scratch + wt_bytes);
   p.logits = logits;
   p.probs = probs;
   p.top = top;
   p.weights = w;
   p.chunk_counts = chunk_counts;
   p.status = status;
-  // H slices per row tile: fill the SMs (two CTAs per SM up to 128 experts
-  // and K <= 8, one otherwise: shared memory or registers), keeping at least
-  // four k blocks per slice
   const int tiles = (int)cdiv(N, kRows);
-  const int slots = device_sms() * (ept == 8 || K > 8 ? 1 : 2);
-  int S = 1;
-  while (S < 8 && tiles * S * 2 <= slots && p.nkb / (S * 2) >= 4) S *= 2;
+  const int S = route_split(N, H, E, K);
 #define MOE_ROUTE_K(EPT_, MN_)                                                 \
   return K <= 8 ? launch_route<EPT_, MN_, 8>(p, S, tiles, s)                  \
                 : (K <= 16 ? launch_route<EPT_, MN_, 16>(p, S, tiles, s)      \
@@ -446,7 +478,6 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   }
 #undef MOE_ROUTE_K
 }
-
 
 // ---------------------------------------------------------------------------
 // Router weight gradient on tensor cores: dW_r = x^T D, D [N, E] bf16 holding

@@ -89,7 +89,9 @@ int64_t moe_padded_rows_max(int32_t N, int32_t E, int32_t K);
 
 /* Workspace bytes for each entry point.  A workspace is caller-owned device
  * memory; its first 256 bytes hold the device status word and must be
- * zeroed once (moe_workspace_init) before first use. */
+ * zeroed once (moe_workspace_init) before first use.  The router's and the
+ * layer's sizes depend on the whole shape and are 0 for a shape the call
+ * would reject. */
 size_t moe_route_workspace_size(int32_t N, int32_t H, int32_t E, int32_t K, moe_dtype dt);
 size_t moe_dispatch_meta_workspace_size(int32_t N, int32_t K, int32_t E);
 size_t moe_grouped_workspace_size(void);

@@ -236,7 +236,8 @@ def test_workspace_sizes_over_many_shapes_do_not_crash():
         P = lib.moe_padded_rows_max(N, E, K)
         assert lib.moe_unpermute_router_bwd_workspace_size(N, H, E, P) > 0
         assert lib.moe_dispatch_meta_workspace_size(N, K, E) > 0
-        assert lib.moe_route_workspace_size(N, H, E, K, dt) > 0
+        route = lib.moe_route_workspace_size(N, H, E, K, dt)
+        assert route == 0 if (dt == 1 and H % 128) else route > 0
         if dt == 1 and (H % 128 or F % 128):
             assert sizes == [0, 0, 0]          # bf16 needs H, F multiples of 128
         else:
