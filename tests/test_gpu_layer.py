@@ -114,6 +114,32 @@ def _bwd_case(shape, seed):
     return c, layer, g
 
 
+# The bf16 router's H split (S = 8, 4, 2 for these shapes) gives the dispatch
+# metadata chunks of 16, 32 and 64 tokens, counted in the router's epilogue;
+# N is not a multiple of the chunk, so the last chunk is ragged.
+SPLIT = [small_shape("split8", N=1000, H=2048, E=64, K=4, F=256, training=True),
+         small_shape("split4_zipf", N=700, H=1024, E=16, K=2, F=128, skew="zipf", skew_param=1.0,
+                     training=True),
+         small_shape("split2_e256", N=6000, H=1024, E=256, K=8, F=128, skew="normal", skew_param=0.75,
+                     training=True)]
+
+
+@pytest.mark.parametrize("shape", SPLIT, ids=lambda s: s.name)
+def test_layer_with_split_router_matches_oracle(shape):
+    c, layer, g = _bwd_case(shape, seed=16)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
+    check_routing_and_meta(layer, shape, ref)
+    yr = om.moe_forward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                        routing=ref)["y"]
+    assert_scaled(layer.y, yr, shape.dtype, "y")
+    gr = om.moe_backward(c["x_cpu"], c["W_r_cpu"], c["W1"].cpu(), c["W3"].cpu(), c["W2"].cpu(), shape.K,
+                         c["dy"].cpu(), routing=ref)
+    for k in ("dx", "dW_r", "dW1", "dW3", "dW2"):
+        assert_scaled(g[k], gr[k], shape.dtype, k)
+
+
 @pytest.mark.parametrize("shape", BWD_SMALL, ids=lambda s: s.name)
 def test_layer_backward_small(shape):
     c, layer, g = _bwd_case(shape, seed=5)

@@ -26,6 +26,12 @@ ROUTE_SHAPES = [
     small_shape("r_bf16_zipf", N=640, H=256, E=64, K=6, skew="zipf", skew_param=1.0),
     small_shape("r_bf16_e4", N=300, H=128, E=4, K=2),
     small_shape("r_bf16_e100", N=333, H=256, E=100, K=5),
+    # few row tiles and a long H: the router splits H over a cluster of S CTAs
+    # (S = 8, 4 and 2 here) and sums the partial logits in slice order
+    small_shape("r_split8_e8", N=300, H=2048, E=8, K=2),
+    small_shape("r_split8_e64", N=1000, H=4096, E=64, K=6),
+    small_shape("r_split4_e256", N=700, H=1024, E=256, K=8, skew="normal", skew_param=1.0),
+    small_shape("r_split2_e40_k12", N=6000, H=1024, E=40, K=12),
 ]
 
 
