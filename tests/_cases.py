@@ -2,12 +2,16 @@
 the tolerance checks the layer's parity is held to.
 
 Tolerances: y and gradients within max|err| <= 2e-2 * max|ref| for bf16 and
-<= 1e-4 * max|ref| for fp32; routing weights and probabilities are fp32
-outputs and take the fp32 bar (their logits accumulate H products in fp32,
-e.g. ~1.3e-5 absolute on the weights at H = 7168); every integer output
-bit-exact.
+<= 1e-4 * max|ref| for fp32; every integer output bit-exact.  Router logits,
+probabilities and routing weights are fp32 outputs whose error comes from the
+fp32 sum of H products (a bf16 x bf16 product is exact in fp32, so only the
+summation rounds): routing_tol bounds it as a multiple of sqrt(H) rounding
+steps of the running sum scaled by the logits' RMS (about 4e-5 on the
+weights at H = 7168, 3e-6 at H = 128).
 """
 from __future__ import annotations
+
+import math
 
 import numpy as np
 import torch
@@ -32,6 +36,38 @@ def assert_scaled(got, ref, dtype: str, what: str = ""):
     e = scaled_err(got, ref)
     assert e <= TOL[dtype], f"{what}: max|err|/max|ref| = {e:.3e} > {TOL[dtype]}"
     return e
+
+
+ROUND32 = 2.0 ** -24   # unit roundoff of fp32
+
+
+def routing_tol(H: int, logit_rms: float) -> float:
+    """Bound on the absolute error of a router logit.  The GPU sums H products
+    in fp32 (exact for bf16 operands) in its own order, tensor-core k steps
+    and H slices included.  Each addition rounds at the magnitude of the
+    running sum, of the order of the logits' RMS, and with terms of random
+    sign those roundings add like a random walk: about sqrt(H/2) * u * RMS
+    for one logit, about 3.5 * sqrt(H) * u * RMS for the largest of a
+    million.  The factor 8 leaves twice that.  The softmax and the
+    renormalisation move a weight or a probability by at most half the
+    largest logit error (p(1-p) <= 1/4 twice), so weights and probabilities
+    take routing_tol / 2."""
+    return 8.0 * math.sqrt(H) * ROUND32 * max(1.0, logit_rms)
+
+
+def assert_routing(got, ref, H: int, logits_ref, what: str, half: bool = True):
+    """Absolute check of a routing output (weights or probabilities when
+    `half`, logits otherwise) against the bound of routing_tol."""
+    g = got.detach().to("cpu", torch.float64).numpy() if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
+    r = np.asarray(ref, np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    lr = np.asarray(logits_ref, np.float64)
+    tol = routing_tol(H, float(np.sqrt(np.mean(lr * lr))) if lr.size else 1.0)
+    if half:
+        tol *= 0.5
+    e = float(np.max(np.abs(g - r))) if r.size else 0.0
+    assert e <= tol, f"{what}: max|err| = {e:.3e} > {tol:.3e} (H = {H})"
+    return e, tol
 
 
 def make_case(shape: MoEShape, seed: int = 0, device="cuda", with_dy=None, repair: bool = True) -> dict:

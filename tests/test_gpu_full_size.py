@@ -10,7 +10,7 @@ import torch
 import dropless_top_moe_b200 as moe
 from gen import WORKLOADS
 from oracle import moe_oracle as om
-from tests._cases import assert_scaled, make_case
+from tests._cases import assert_routing, assert_scaled, make_case
 
 pytestmark = pytest.mark.gpu
 
@@ -24,7 +24,7 @@ def _fwd_full(name, n_sample, seed=0):
     assert layer.status() == 0
     ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
     np.testing.assert_array_equal(layer.top_experts.cpu().numpy(), ref["top_experts"])
-    assert_scaled(layer.weights, ref["weights"], "f32", "routing weights")
+    assert_routing(layer.weights, ref["weights"], shape.H, ref["logits"], "routing weights")
     m = om.dispatch_meta(ref["top_experts"], shape.E)
     for k in ("indices", "bins", "padded_bins"):
         np.testing.assert_array_equal(getattr(layer, k).cpu().numpy(), m[k], err_msg=k)

@@ -7,7 +7,7 @@ import torch
 import dropless_top_moe_b200 as moe
 from gen import WORKLOADS
 from oracle import moe_oracle as om
-from tests._cases import TOL, assert_scaled, make_case, small_shape
+from tests._cases import TOL, assert_routing, assert_scaled, make_case, small_shape
 
 pytestmark = pytest.mark.gpu
 
@@ -21,7 +21,7 @@ def run_fwd(shape, c, training=False):
 
 def check_routing_and_meta(layer, shape, ref):
     np.testing.assert_array_equal(layer.top_experts.cpu().numpy(), ref["top_experts"])
-    assert_scaled(layer.weights, ref["weights"], "f32", "routing weights")
+    assert_routing(layer.weights, ref["weights"], shape.H, ref["logits"], "routing weights")
     m = om.dispatch_meta(ref["top_experts"], shape.E)
     np.testing.assert_array_equal(layer.indices.cpu().numpy(), m["indices"])
     np.testing.assert_array_equal(layer.bins.cpu().numpy(), m["bins"])

@@ -11,7 +11,7 @@ import torch
 import dropless_top_moe_b200 as moe
 from gen import WORKLOADS, random_counts, MoEShape
 from oracle import moe_oracle as om
-from tests._cases import TOL, assert_scaled, make_case, scaled_err, small_shape
+from tests._cases import TOL, assert_routing, assert_scaled, make_case, scaled_err, small_shape
 
 pytestmark = pytest.mark.gpu
 
@@ -41,10 +41,10 @@ def test_route_matches_oracle(shape):
     r = moe.moe_route(c["x"], c["W_r"], shape.K, want_logits=True, want_probs=True)
     ref = om.route(c["x_cpu"], c["W_r_cpu"], shape.K)
     np.testing.assert_array_equal(r["top_experts"].cpu().numpy(), ref["top_experts"])
-    assert_scaled(r["weights"], ref["weights"], "f32", "routing weights")
-    assert_scaled(r["probs"], ref["probs"], "f32", "probs")
+    assert_routing(r["weights"], ref["weights"], shape.H, ref["logits"], "routing weights")
+    assert_routing(r["probs"], ref["probs"], shape.H, ref["logits"], "probs")
     lg = r["logits"].cpu().double().numpy()
-    assert np.max(np.abs(lg - ref["logits"])) <= 1e-4 * max(1.0, np.max(np.abs(ref["logits"])))
+    assert_routing(lg, ref["logits"], shape.H, ref["logits"], "logits", half=False)
     # the decision margin also holds on the GPU's own logits
     assert om.topk_gaps(lg, shape.K).min() >= 0.9e-3
     assert moe.device_status(r["ws"]) == 0
