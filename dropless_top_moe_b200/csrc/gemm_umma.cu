@@ -10,15 +10,17 @@
 // static shapes without host sync).
 //
 // One CTA (or one CTA pair, cta_group::2) per SM, 10 warps:
-//   warp 0      producer: A and B tiles by TMA into a STAGES-deep smem ring
+//   warp 0      producer: A and B tiles by TMA into a STAGES-deep smem ring,
+//               one 64-deep k block per stage (two for a CTA pair)
 //               (optionally A rows gathered from x with tile::gather4)
 //   warp 1      TMEM allocator and MMA issuer (one thread): tcgen05.mma per
 //               16-deep k step, fp32 accumulators in TMEM, double-buffered
 //               where two accumulator sets fit so the epilogue of tile i
 //               overlaps the main loop of tile i+1
 //   warps 2..9  epilogue, two warps per TMEM lane quarter: tcgen05.ld rows ->
-//               registers -> fused math -> global (through a per-warp
-//               shared-memory scratch where that coalesces the accesses)
+//               registers -> fused math -> global, 32 x 32 chunks through
+//               a per-warp shared-memory scratch (TMA stores, or coalesced
+//               64-byte row segments for the weight gradients)
 // Tile shapes: BN output columns; MT 128-row tiles per CTA; CG = 2 pairs two
 // CTAs on one M = 256 MMA (each CTA holds its 128 rows and half of B's
 // columns); an expert's odd last tile runs as an M = 128 pair MMA.
@@ -60,6 +62,7 @@ enum Split { SPLIT_NONE = 0, SPLIT_K = 1, SPLIT_N = 2 };
 
 struct Params {
   CUtensorMap ta0, ta1, tb0, tb1;
+  CUtensorMap to0, to1, to2;   // outputs of the TMA-store epilogues (32 x 32 boxes)
   const int32_t* padded_bins;
   int E;
   int64_t P;          // rows of row-indexed buffers (ROWS/WGRAD) or tokens (DENSE)
@@ -102,7 +105,12 @@ template <int BN, int MT, int CG = 1>
 struct Shape {
   static constexpr int A_BYTES = MT * BM * BK * 2;
   static constexpr int B_BYTES = (CG == 2 ? BN / 2 : BN) * BK * 2;   // a pair splits B's columns
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SUB_BYTES = A_BYTES + B_BYTES;                 // one BK-deep k block
+  // k blocks per pipeline stage: a pair's four M = 256 MMAs per k block take
+  // less time than the issuing thread's per-stage work (barrier wait, commit,
+  // four issues), so a pair stage holds two k blocks
+  static constexpr int KSUB = CG == 2 ? 2 : 1;
+  static constexpr int STAGE_BYTES = KSUB * SUB_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
   static constexpr int ACC_COLS = MT * BN;                       // one accumulator set
   static constexpr int ACC_BUFS = 2 * ACC_COLS <= 512 ? 2 : 1;   // double-buffer when it fits
@@ -219,9 +227,61 @@ __device__ __forceinline__ void load_row_bf16x32(const __nv_bfloat16* src, float
   }
 }
 
-// Shared-memory scratch per epilogue warp for coalesced stores: 32 rows x 64
-// bytes (one 32-column chunk of bf16).
-constexpr int kStoreScratch = 32 * 64;
+// Shared-memory scratch per epilogue warp: 32 rows x 64 bytes (one 32-column
+// chunk of bf16) per buffer.
+constexpr int kStoreBuf = 32 * 64;
+
+// How an epilogue writes its rows.  A TMEM load gives each lane one row, so a
+// store straight from registers sends 32 rows per warp instruction.
+//   STORE_TMA        the chunk goes through one of two scratch buffers to a
+//                    TMA store (SwiGLU, SwiGLU backward, plain stores:
+//                    measured 4-9 % faster per GEMM on B200 than storing
+//                    from registers or through the warp)
+//   STORE_COALESCED  through one scratch buffer to 64-byte row segments by
+//                    the warp (the weight gradients: TMA stores measured 5 %
+//                    slower there)
+//   STORE_DIRECT     straight from registers (the dense router dx)
+enum StoreMode { STORE_DIRECT = 0, STORE_COALESCED = 1, STORE_TMA = 2 };
+template <int EPI>
+__host__ __device__ constexpr int store_mode() {
+  return (EPI == EPI_STORE || EPI == EPI_SWIGLU_BWD || EPI == EPI_SWIGLU) ? STORE_TMA
+         : (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) ? STORE_COALESCED
+                                                       : STORE_DIRECT;
+}
+template <int EPI>
+__host__ __device__ constexpr int scratch_bytes() {
+  return store_mode<EPI>() == STORE_TMA ? 2 * kStoreBuf
+         : store_mode<EPI>() == STORE_COALESCED || EPI == EPI_SWIGLU_BWD ? kStoreBuf : 0;
+}
+
+// TMA store of a warp's 32 x 32 bf16 chunk: lane i holds row i's 32 values v;
+// (x, y) = (first column, first row) of the chunk in map m.  The chunk is
+// written to one of the warp's two scratch buffers (nb alternates) in the
+// 64-byte swizzle layout the map expects -- 16-byte piece q of row r at
+// position q ^ ((r >> 1) & 3), which also keeps the writes free of bank
+// conflicts -- and one lane hands it to the TMA unit.  Before a buffer is
+// rewritten, the store that used it two chunks earlier must have read it.
+__device__ __forceinline__ void store_chunk_tma(uint32_t scratch, int& nb, int lane, const CUtensorMap* m,
+                                                int x, int y, const float* v) {
+  const uint32_t buf = scratch + (uint32_t)(nb * kStoreBuf);
+  nb ^= 1;
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t a = buf + (uint32_t)(lane * 64) + ((uint32_t)(q ^ ((lane >> 1) & 3)) << 4);
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(pack_bf16x2(v[8 * q + 0], v[8 * q + 1])),
+                 "r"(pack_bf16x2(v[8 * q + 2], v[8 * q + 3])), "r"(pack_bf16x2(v[8 * q + 4], v[8 * q + 5])),
+                 "r"(pack_bf16x2(v[8 * q + 6], v[8 * q + 7]))
+                 : "memory");
+  }
+  fence_proxy_async();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(m, buf, x, y);
+    bulk_commit();
+  }
+}
 
 // Store a warp's 32 x 32 bf16 chunk: lane i holds row i's 32 values v; base
 // points at the chunk's first element (row 0), ld is the row stride.  Storing
@@ -277,14 +337,16 @@ __device__ __forceinline__ void rows_from_coalesced(uint32_t scratch, int lane, 
 }
 
 // Epilogue of one 128-row half: TMEM columns [tacc, tacc + BN) of this
-// thread's row -> fused math -> global memory.  scratch: this warp's
-// kStoreScratch bytes of shared memory (EPI_STORE), else 0.
+// thread's row -> fused math -> global memory (store_mode<EPI>).  scratch:
+// this warp's scratch_bytes<EPI>() bytes of shared memory; nb: the warp's next
+// TMA-store buffer, carried across calls.
 template <int BN, int SCHED, int EPI>
 __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, uint32_t tacc, int row,
-                                              int part, uint32_t scratch = 0) {
+                                              int part, uint32_t scratch, int& nb) {
   const int64_t grow = tl.row0 + row;                 // ROWS/DENSE global row
   const int lane = row & 31;
   const int64_t row_base = grow - lane;               // the warp's first row (ROWS/DENSE)
+  const int yb = (int)row_base;
   // the two warps of a lane quarter split the columns: part 0 / part 1
   constexpr int NC = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
   const int c_begin = part * (NC / 2), c_end = c_begin + NC / 2;
@@ -303,10 +365,10 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
         uf[j] = __uint_as_float(u[j]);
         a[j] = silu_f(gf[j]) * uf[j];
       }
-      if (p.out0) store_row_bf16x32(p.out0 + grow * p.ldo + tl.n0 + c, a);
+      if (p.out0) store_chunk_tma(scratch, nb, lane, &p.to0, tl.n0 + c, yb, a);
       if (p.out1) {
-        store_row_bf16x32(p.out1 + grow * p.ldo + tl.n0 + c, gf);
-        store_row_bf16x32(p.out2 + grow * p.ldo + tl.n0 + c, uf);
+        store_chunk_tma(scratch, nb, lane, &p.to1, tl.n0 + c, yb, gf);
+        store_chunk_tma(scratch, nb, lane, &p.to2, tl.n0 + c, yb, uf);
       }
     }
   } else if constexpr (EPI == EPI_STORE) {
@@ -318,34 +380,30 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       float v[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-      if (scratch) store_chunk_coalesced(scratch, lane, p.out0 + row_base * p.ldo + tl.n0 + c, p.ldo, v);
-      else store_row_bf16x32(p.out0 + grow * p.ldo + tl.n0 + c, v);
+      store_chunk_tma(scratch, nb, lane, &p.to0, tl.n0 + c, yb, v);
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-    const int64_t off = grow * p.ldo + tl.n0;
 #pragma unroll 1
     for (int c = c_begin; c < c_end; c += 32) {
       uint32_t r[32];
       tmem_ld_32(tacc + c, r);
       float gf[32], uf[32], dg[32], du[32];
-      if (scratch) {
-        // G and U as 64-byte row segments, 4 lanes per row (each element is
-        // read here before this warp writes it, so dG, dU may alias G, U)
-        uint4 wg[4], wu[4];
+      // G and U as 64-byte row segments, 4 lanes per row, exchanged through
+      // the first scratch buffer once no store still reads it (each element
+      // is read here before this warp stores it, so dG, dU may alias G, U)
+      uint4 wg[4], wu[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int64_t o = (row_base + 8 * i + (lane >> 2)) * p.ldo + tl.n0 + c + 8 * (lane & 3);
-          wg[i] = *reinterpret_cast<const uint4*>(p.aux0 + o);
-          wu[i] = *reinterpret_cast<const uint4*>(p.aux1 + o);
-        }
-        tmem_ld_wait();
-        rows_from_coalesced(scratch, lane, wg, gf);
-        rows_from_coalesced(scratch, lane, wu, uf);
-      } else {
-        load_row_bf16x32(p.aux0 + off + c, gf);
-        load_row_bf16x32(p.aux1 + off + c, uf);
-        tmem_ld_wait();
+      for (int i = 0; i < 4; ++i) {
+        const int64_t o = (row_base + 8 * i + (lane >> 2)) * p.ldo + tl.n0 + c + 8 * (lane & 3);
+        wg[i] = *reinterpret_cast<const uint4*>(p.aux0 + o);
+        wu[i] = *reinterpret_cast<const uint4*>(p.aux1 + o);
       }
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      tmem_ld_wait();
+      rows_from_coalesced(scratch, lane, wg, gf);
+      rows_from_coalesced(scratch, lane, wu, uf);
+      nb = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float da = __uint_as_float(r[j]);
@@ -353,8 +411,8 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
         dg[j] = da * uf[j] * sig * (1.f + gf[j] * (1.f - sig));
         du[j] = da * gf[j] * sig;
       }
-      store_row_bf16x32(p.out0 + off + c, dg);
-      store_row_bf16x32(p.out1 + off + c, du);
+      store_chunk_tma(scratch, nb, lane, &p.to0, tl.n0 + c, yb, dg);
+      store_chunk_tma(scratch, nb, lane, &p.to1, tl.n0 + c, yb, du);
     }
   } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) {
     const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
@@ -464,6 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   using S = Shape<BN, MT, CG>;
   constexpr int STAGES = S::STAGES;
   constexpr int STAGE_BYTES = S::STAGE_BYTES;
+  constexpr int SUB_BYTES = S::SUB_BYTES;
+  constexpr int KSUB = S::KSUB;
   constexpr int A_BYTES = S::A_BYTES;
   constexpr int B_BYTES = S::B_BYTES;
   constexpr int ACC_BUFS = S::ACC_BUFS;
@@ -497,13 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * S::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int32_t* s_unit_start = reinterpret_cast<int32_t*>(tmem_holder + 4);   // [E + 1]
-  // kStoreScratch bytes per epilogue warp for coalesced stores, 128-byte
-  // aligned.  Used by the plain-store and weight-gradient epilogues (measured
-  // 2-8 % faster on B200); the SwiGLU epilogues, whose two or three outputs
-  // would make as many round trips and which CTA pairs overlap with the
-  // main loop anyway, measured up to 4 % slower with it and store directly.
-  constexpr bool kCoalesced = EPI == EPI_STORE || EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR || EPI == EPI_SWIGLU_BWD;
-  const uint32_t store_scratch = (smem_u32(s_unit_start + 260) + 127u) & ~127u;
+  // scratch_bytes<EPI>() per epilogue warp, 512-byte aligned (the 64-byte
+  // swizzle of the TMA stores repeats every 512 bytes)
+  constexpr int kScratch = scratch_bytes<EPI>();
+  const uint32_t store_scratch = (smem_u32(s_unit_start + 260) + 511u) & ~511u;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;          // 0 = leader
@@ -607,42 +664,44 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
 #pragma unroll
           for (int i = 0; i < 4; ++i) nx[i] = tl.nkb > 0 ? tok_of(tl.row0 + 4 * g + i) : p.g_N;
         }
-        for (int kb = 0; kb < tl.nkb; ++kb) {
+        for (int kb0 = 0; kb0 < tl.nkb; kb0 += KSUB) {
+          const int nsub = (tl.nkb - kb0) < KSUB ? (tl.nkb - kb0) : KSUB;
           int w_ok = 1;
           if (lane == 0)
             w_ok = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kTimeoutNs) ? 1 : 0;
           w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
           if (!w_ok) { ok = false; break; }
-          const uint32_t sa = base + stage * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
           const uint32_t fb = PAIR ? map_to_rank(full_bar(stage), 0) : full_bar(stage);
-          const int kc = SCHED == SCHED_WGRAD ? (int)(tl.row0 + (int64_t)kb * BK) : kb * BK;
-          if (lane == 0) {
-            if (!PAIR || rank == 0) mbar_expect_tx(full_bar(stage), tx);
-            load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, kc, &p.tb0, LONE && tl.halves == 1);
-          }
-          if constexpr (SCHED == SCHED_WGRAD) {
-            int cur[4];
+          if (lane == 0 && (!PAIR || rank == 0)) mbar_expect_tx(full_bar(stage), tx * (uint32_t)nsub);
+          for (int j = 0; j < nsub; ++j) {
+            const int kb = kb0 + j;
+            const uint32_t sa = base + stage * STAGE_BYTES + j * SUB_BYTES;
+            const uint32_t sb = sa + A_BYTES;
+            const int kc = SCHED == SCHED_WGRAD ? (int)(tl.row0 + (int64_t)kb * BK) : kb * BK;
+            if (lane == 0) load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, kc, &p.tb0, LONE && tl.halves == 1);
+            if constexpr (SCHED == SCHED_WGRAD) {
+              int cur[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) cur[i] = nx[i];
-            for (int h = 0; h < n_mma_h; ++h) {
-              const int hh = PAIR ? 2 * h + (int)rank : h;
-              const uint32_t dst = sa + h * (BM * BK * 2) + jb * 8192 + g * 512;
-              const int m = tl.m0 + BM * hh + 64 * jb;
-              if constexpr (PAIR) tma_gather4_pair(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
-              else tma_gather4(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
-            }
-            if (kb + 1 < tl.nkb) {
+              for (int i = 0; i < 4; ++i) cur[i] = nx[i];
+              for (int h = 0; h < n_mma_h; ++h) {
+                const int hh = PAIR ? 2 * h + (int)rank : h;
+                const uint32_t dst = sa + h * (BM * BK * 2) + jb * 8192 + g * 512;
+                const int m = tl.m0 + BM * hh + 64 * jb;
+                if constexpr (PAIR) tma_gather4_pair(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
+                else tma_gather4(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
+              }
+              if (kb + 1 < tl.nkb) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) nx[i] = tok_of((int64_t)kc + BK + 4 * g + i);
-            }
-          } else {
+                for (int i = 0; i < 4; ++i) nx[i] = tok_of((int64_t)kc + BK + 4 * g + i);
+              }
+            } else {
 #pragma unroll
-            for (int h = 0; h < MT; ++h) {
-              if (h < n_mma_h) {
-                const uint32_t dst = sa + h * (BM * BK * 2) + lane * 512;
-                if constexpr (PAIR) tma_gather4_pair(dst, &p.ta0, fb, kc, tk[h][0], tk[h][1], tk[h][2], tk[h][3]);
-                else tma_gather4(dst, &p.ta0, fb, kc, tk[h][0], tk[h][1], tk[h][2], tk[h][3]);
+              for (int h = 0; h < MT; ++h) {
+                if (h < n_mma_h) {
+                  const uint32_t dst = sa + h * (BM * BK * 2) + lane * 512;
+                  if constexpr (PAIR) tma_gather4_pair(dst, &p.ta0, fb, kc, tk[h][0], tk[h][1], tk[h][2], tk[h][3]);
+                  else tma_gather4(dst, &p.ta0, fb, kc, tk[h][0], tk[h][1], tk[h][2], tk[h][3]);
+                }
               }
             }
           }
@@ -666,49 +725,51 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
         if constexpr (PAIR) tx = 2u * (uint32_t)(n_mma_h * BM * BK * 2 + B_BYTES);   // both CTAs' loads
         else tx = (uint32_t)tl.halves * BM * BK * 2 +
                   (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)B_BYTES);
-        for (int kb = 0; kb < tl.nkb; ++kb) {
+        for (int kb0 = 0; kb0 < tl.nkb; kb0 += KSUB) {
+          const int nsub = (tl.nkb - kb0) < KSUB ? (tl.nkb - kb0) : KSUB;
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
-          const uint32_t sa = base + stage * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
-          if constexpr (PAIR) {
-            const uint32_t fb = map_to_rank(full_bar(stage), 0);      // the leader's barrier
-            if (rank == 0) mbar_expect_tx(full_bar(stage), tx);
-            if constexpr (SCHED == SCHED_WGRAD) {
-              const int krow = (int)(tl.row0 + (int64_t)kb * BK);
-              for (int h = 0; h < n_mma_h; ++h) {
-                const int m = tl.m0 + BM * (2 * h + (int)rank);
-                tma_load_2d_pair(sa + h * (BM * BK * 2), &p.ta0, fb, m, krow);
-                tma_load_2d_pair(sa + h * (BM * BK * 2) + 8192, &p.ta0, fb, m + 64, krow);
+          const uint32_t fb = PAIR ? map_to_rank(full_bar(stage), 0) : full_bar(stage);   // the leader's barrier
+          if (!PAIR || rank == 0) mbar_expect_tx(full_bar(stage), tx * (uint32_t)nsub);
+          for (int j = 0; j < nsub; ++j) {
+            const int kb = kb0 + j;
+            const uint32_t sa = base + stage * STAGE_BYTES + j * SUB_BYTES;
+            const uint32_t sb = sa + A_BYTES;
+            if constexpr (PAIR) {
+              if constexpr (SCHED == SCHED_WGRAD) {
+                const int krow = (int)(tl.row0 + (int64_t)kb * BK);
+                for (int h = 0; h < n_mma_h; ++h) {
+                  const int m = tl.m0 + BM * (2 * h + (int)rank);
+                  tma_load_2d_pair(sa + h * (BM * BK * 2), &p.ta0, fb, m, krow);
+                  tma_load_2d_pair(sa + h * (BM * BK * 2) + 8192, &p.ta0, fb, m + 64, krow);
+                }
+                load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, krow, &p.tb0);
+              } else {
+                int k = kb * BK;
+                const CUtensorMap* ta = &p.ta0;
+                const CUtensorMap* tb = &p.tb0;
+                if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
+                const bool lone = LONE && tl.halves == 1;
+                for (int h = 0; h < n_mma_h; ++h)
+                  tma_load_2d_pair(sa + h * (BM * BK * 2), ta, fb, k,
+                                   (int)tl.row0 + (lone ? 64 * (int)rank : BM * (2 * h + (int)rank)));
+                load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, k, tb, lone);
               }
-              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, krow, &p.tb0);
             } else {
-              int k = kb * BK;
-              const CUtensorMap* ta = &p.ta0;
-              const CUtensorMap* tb = &p.tb0;
-              if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
-              const bool lone = LONE && tl.halves == 1;
-              for (int h = 0; h < n_mma_h; ++h)
-                tma_load_2d_pair(sa + h * (BM * BK * 2), ta, fb, k,
-                                 (int)tl.row0 + (lone ? 64 * (int)rank : BM * (2 * h + (int)rank)));
-              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, k, tb, lone);
-            }
-          } else {
-            const uint32_t fb = full_bar(stage);
-            mbar_expect_tx(fb, tx);
-            if constexpr (SCHED == SCHED_WGRAD) {
-              const int krow = (int)(tl.row0 + (int64_t)kb * BK);
-              // A = X^T: 64-wide MN boxes of the [rows, M] matrix, 2 per half
+              if constexpr (SCHED == SCHED_WGRAD) {
+                const int krow = (int)(tl.row0 + (int64_t)kb * BK);
+                // A = X^T: 64-wide MN boxes of the [rows, M] matrix, 2 per half
 #pragma unroll
-              for (int j = 0; j < 2 * MT; ++j) tma_load_2d(sa + j * 8192, &p.ta0, fb, tl.m0 + 64 * j, krow);
-              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, 0u, krow, &p.tb0);
-            } else {
-              int k = kb * BK;
-              const CUtensorMap* ta = &p.ta0;
-              const CUtensorMap* tb = &p.tb0;
-              if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
-              tma_load_2d(sa, ta, fb, k, (int)tl.row0);
-              if (MT == 2 && tl.halves == 2) tma_load_2d(sa + BM * BK * 2, ta, fb, k, (int)tl.row0 + BM);
-              load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, 0u, k, tb);
+                for (int q = 0; q < 2 * MT; ++q) tma_load_2d(sa + q * 8192, &p.ta0, fb, tl.m0 + 64 * q, krow);
+                load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, 0u, krow, &p.tb0);
+              } else {
+                int k = kb * BK;
+                const CUtensorMap* ta = &p.ta0;
+                const CUtensorMap* tb = &p.tb0;
+                if (SPLIT == SPLIT_K && k >= p.ksplit) { k -= p.ksplit; ta = &p.ta1; tb = &p.tb1; }
+                tma_load_2d(sa, ta, fb, k, (int)tl.row0);
+                if (MT == 2 && tl.halves == 2) tma_load_2d(sa + BM * BK * 2, ta, fb, k, (int)tl.row0 + BM);
+                load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, 0u, k, tb);
+              }
             }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -738,31 +799,37 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
         const uint32_t idesc = (LONE && tl.halves == 1) ? idesc_lone : idesc_full;
-        for (int kb = 0; kb < tl.nkb; ++kb) {
+        for (int kb0 = 0; kb0 < tl.nkb; kb0 += KSUB) {
+          const int nsub = (tl.nkb - kb0) < KSUB ? (tl.nkb - kb0) : KSUB;
           if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = base + stage * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
-            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            if constexpr (PAIR) {
+          for (int j = 0; j < KSUB; ++j) {
+            if (j < nsub) {
+              const uint32_t sa = base + stage * STAGE_BYTES + j * SUB_BYTES;
+              const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-              for (int h = 0; h < MT; ++h) {
-                if (2 * h < tl.halves) {
-                  const uint32_t ah = sa + h * (BM * BK * 2);
-                  const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
-                  mma_bf16_pair(d_tmem + h * BN, ad, bd, idesc, accum);
-                }
-              }
-            } else {
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
+                const uint32_t accum = ((kb0 + j) | kk) != 0 ? 1u : 0u;
+                if constexpr (PAIR) {
 #pragma unroll
-              for (int h = 0; h < MT; ++h) {
-                if (h < tl.halves) {
-                  const uint32_t ah = sa + h * (BM * BK * 2);
-                  const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
-                  mma_bf16(d_tmem + h * BN, ad, bd, idesc, accum);
+                  for (int h = 0; h < MT; ++h) {
+                    if (2 * h < tl.halves) {
+                      const uint32_t ah = sa + h * (BM * BK * 2);
+                      const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
+                      mma_bf16_pair(d_tmem + h * BN, ad, bd, idesc, accum);
+                    }
+                  }
+                } else {
+#pragma unroll
+                  for (int h = 0; h < MT; ++h) {
+                    if (h < tl.halves) {
+                      const uint32_t ah = sa + h * (BM * BK * 2);
+                      const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
+                      mma_bf16(d_tmem + h * BN, ad, bd, idesc, accum);
+                    }
+                  }
                 }
               }
             }
@@ -788,6 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     const int part = (warp - 2) >> 2;             // which half of the columns
     const int row = q * 32 + lane;                // row inside a 128-row half
     const uint32_t tempty_leader0 = PAIR ? map_to_rank(tempty_bar(0), 0) : 0u;
+    int nb = 0;                                   // next TMA-store scratch buffer
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t t = tile0; t < ntiles; t += tstep) {
@@ -830,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           th.row0 = tl.row0 + 64 * (int)rank;
           th.n0 = tl.n0 + g * (EPI == EPI_SWIGLU ? BN / 4 : BN / 2);
           epilogue_half<BN / 2, SCHED, EPI>(p, th, tacc, (q & 1) * 32 + lane, part,
-                                            kCoalesced ? store_scratch + (warp - 2) * kStoreScratch : 0u);
+                                            kScratch ? store_scratch + (warp - 2) * kScratch : 0u, nb);
           lone_done = true;
         }
       }
@@ -845,7 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           Tile th = tl;
           if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + j * BM; else th.row0 = tl.row0 + j * BM;
           epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part,
-                                        kCoalesced ? store_scratch + (warp - 2) * kStoreScratch : 0u);
+                                        kScratch ? store_scratch + (warp - 2) * kScratch : 0u, nb);
         }
       } else {
 #pragma unroll 1
@@ -854,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           Tile th = tl;
           if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + h * BM; else th.row0 = tl.row0 + h * BM;
           epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part,
-                                        kCoalesced ? store_scratch + (warp - 2) * kStoreScratch : 0u);
+                                        kScratch ? store_scratch + (warp - 2) * kScratch : 0u, nb);
         }
       }
       tc_fence_before();
@@ -865,6 +933,9 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
       }
       if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
     }
+    // the TMA stores have read their scratch and written global memory
+    if (store_mode<EPI>() == STORE_TMA && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -911,6 +982,20 @@ static bool map2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t oute
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 map over a row-major [outer, inner] output for TMA stores of
+// 32 x 32 chunks, 64-byte swizzle (one 64-byte chunk row per swizzle row).
+static bool map_out2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_elems) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_elems * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D bf16 map over [d2, d1, d0] (d0 contiguous), 128-byte swizzle, box depth 1.
 static bool map3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
                   uint32_t box0, uint32_t box1) {
@@ -944,8 +1029,9 @@ static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upp
   Params p = p_in;
   if (p.group_m <= 0) p.group_m = S::UNIT >= 4 ? (kGroupM * 2) / S::UNIT : kGroupM;
   auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA>;
-  constexpr bool coalesced = EPI == EPI_STORE || EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR || EPI == EPI_SWIGLU_BWD;
-  const size_t smem = S::SMEM + (coalesced ? (size_t)kEpiWarps * kStoreScratch + 128 : 0);
+  constexpr size_t scratch = scratch_bytes<EPI>() ? (size_t)kEpiWarps * scratch_bytes<EPI>() + 512 : 0;
+  static_assert(S::SMEM + scratch <= 232448, "shared memory per CTA");
+  const size_t smem = S::SMEM + scratch;
   // once per device: later calls (a CUDA graph capture among them) only launch
   static bool smem_set[64] = {false};
   int dev = 0;
@@ -1044,6 +1130,9 @@ moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const 
   if (!a_ok || !map3d(&p.tb0, W1, F, H, E, 64, 64) || !map3d(&p.tb1, W3, F, H, E, 64, 64))
     return MOE_ERR_CUDA;
   if (ga) set_gather(&p, ga);
+  if ((act && !map_out2d(&p.to0, act, F, P, F)) || (G && !map_out2d(&p.to1, G, F, P, F)) ||
+      (U && !map_out2d(&p.to2, U, F, P, F)))
+    return MOE_ERR_CUDA;
   p.kdim = H;
   p.n_mma = 256;
   p.n_tiles = F / 128;
@@ -1069,7 +1158,9 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
   {
     Params p = blank_params(pb, E, P, status);
     const int bn = (H % 256 == 0) ? 256 : 128;
-    if (!map2d(&p.ta0, act, F, P, F, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, 64)) return MOE_ERR_CUDA;
+    if (!map2d(&p.ta0, act, F, P, F, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, 64) ||
+        !map_out2d(&p.to0, out, H, P, H))
+      return MOE_ERR_CUDA;
     p.kdim = F;
     p.n_mma = bn;
     p.n_tiles = H / bn;
@@ -1098,7 +1189,8 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     Params p = blank_params(pb, E, P, status);
     const int bn = (F % 256 == 0) ? 256 : 128;
     const bool pair = pref && bn == 256;
-    if (!map2d(&p.ta0, d_out, H, P, H, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, pair ? bn / 2 : bn))
+    if (!map2d(&p.ta0, d_out, H, P, H, 64, 128) || !map3d(&p.tb0, W2, H, F, E, 64, pair ? bn / 2 : bn) ||
+        !map_out2d(&p.to0, dG, F, P, F) || !map_out2d(&p.to1, dU, F, P, F))
       return MOE_ERR_CUDA;
     p.kdim = H;
     p.n_mma = bn;
@@ -1163,7 +1255,8 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     const bool pair = false;    // see the kernel choice note above
     const uint32_t box = pair ? bn / 2 : bn;
     if (!map2d(&p.ta0, dG, F, P, F, 64, 128) || !map2d(&p.ta1, dU, F, P, F, 64, 128) ||
-        !map3d(&p.tb0, W1, F, H, E, 64, box) || !map3d(&p.tb1, W3, F, H, E, 64, box))
+        !map3d(&p.tb0, W1, F, H, E, 64, box) || !map3d(&p.tb1, W3, F, H, E, 64, box) ||
+        !map_out2d(&p.to0, dx_perm, H, P, H))
       return MOE_ERR_CUDA;
     p.kdim = 2 * F;
     p.ksplit = F;
