@@ -261,6 +261,19 @@ __host__ __device__ constexpr int scratch_bytes() {
 // position q ^ ((r >> 1) & 3), which also keeps the writes free of bank
 // conflicts -- and one lane hands it to the TMA unit.  Before a buffer is
 // rewritten, the store that used it two chunks earlier must have read it.
+// Lane i's row i of a 32 x 32 bf16 chunk into scratch buffer buf, in the
+// 64-byte swizzle layout of the output maps.
+__device__ __forceinline__ void stage_chunk(uint32_t buf, int lane, const float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t a = buf + (uint32_t)(lane * 64) + ((uint32_t)(q ^ ((lane >> 1) & 3)) << 4);
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(pack_bf16x2(v[8 * q + 0], v[8 * q + 1])),
+                 "r"(pack_bf16x2(v[8 * q + 2], v[8 * q + 3])), "r"(pack_bf16x2(v[8 * q + 4], v[8 * q + 5])),
+                 "r"(pack_bf16x2(v[8 * q + 6], v[8 * q + 7]))
+                 : "memory");
+  }
+}
+
 __device__ __forceinline__ void store_chunk_tma(uint32_t scratch, int& nb, int lane, const CUtensorMap* m,
                                                 int x, int y, const float* v) {
   const uint32_t buf = scratch + (uint32_t)(nb * kStoreBuf);
@@ -372,15 +385,30 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       }
     }
   } else if constexpr (EPI == EPI_STORE) {
+    // two chunks per round: both TMEM loads under one wait, both buffers
+    // under one proxy fence
 #pragma unroll 1
-    for (int c = c_begin; c < c_end; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32(tacc + c, r);
+    for (int c = c_begin; c < c_end; c += 64) {
+      uint32_t r0[32], r1[32];
+      tmem_ld_32(tacc + c, r0);
+      tmem_ld_32(tacc + c + 32, r1);
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
       tmem_ld_wait();
       float v[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-      store_chunk_tma(scratch, nb, lane, &p.to0, tl.n0 + c, yb, v);
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
+      stage_chunk(scratch, lane, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
+      stage_chunk(scratch + kStoreBuf, lane, v);
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&p.to0, scratch, tl.n0 + c, yb);
+        tma_store_2d(&p.to0, scratch + kStoreBuf, tl.n0 + c + 32, yb);
+        bulk_commit();
+      }
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
 #pragma unroll 1
@@ -403,7 +431,6 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       tmem_ld_wait();
       rows_from_coalesced(scratch, lane, wg, gf);
       rows_from_coalesced(scratch, lane, wu, uf);
-      nb = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float da = __uint_as_float(r[j]);
@@ -411,8 +438,16 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
         dg[j] = da * uf[j] * sig * (1.f + gf[j] * (1.f - sig));
         du[j] = da * gf[j] * sig;
       }
-      store_chunk_tma(scratch, nb, lane, &p.to0, tl.n0 + c, yb, dg);
-      store_chunk_tma(scratch, nb, lane, &p.to1, tl.n0 + c, yb, du);
+      // both buffers are free: every earlier store was waited for above
+      stage_chunk(scratch, lane, dg);
+      stage_chunk(scratch + kStoreBuf, lane, du);
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&p.to0, scratch, tl.n0 + c, yb);
+        tma_store_2d(&p.to1, scratch + kStoreBuf, tl.n0 + c, yb);
+        bulk_commit();
+      }
     }
   } else if constexpr (EPI == EPI_WGRAD || EPI == EPI_WGRAD_PAIR) {
     const int64_t off = (int64_t)tl.e * p.out_estride + (int64_t)(tl.m0 + row) * p.ldo + tl.n0;
