@@ -50,10 +50,10 @@ constexpr int BK = 64;              // one 128-byte swizzle row of bf16
 constexpr int kEpiWarps = 8;              // two warps per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
-// M units per raster group (L2 reuse of the weight panels): 4 units of 256
-// rows, about one expert's rows at the training step's 1024 tokens per
-// expert; measured 1-3 % faster per GEMM than 8 units, 16 slower
-constexpr int kGroupM = 4;
+// Most M units per raster group (groups never span two experts, see
+// get_tile): 8 units of up to 256 rows, so an expert of up to 2048 rows streams
+// each weight column panel once
+constexpr int kGroupM = 8;
 
 enum Sched { SCHED_ROWS = 0, SCHED_WGRAD = 1, SCHED_DENSE = 2 };
 enum Epi { EPI_SWIGLU = 0, EPI_STORE = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3, EPI_WGRAD_PAIR = 4,
@@ -123,25 +123,16 @@ struct Shape {
   static constexpr int UNIT = MT * CG;
 };
 
-// Rows of the grouped buffers actually used, clamped to the buffers' rows.
-__device__ __forceinline__ int64_t used_rows(const Params& p) {
-  int64_t rows = p.padded_bins[p.E - 1];
-  return rows > p.P ? p.P : rows;
-}
 
-// Number of M units for the ROWS schedule: 128-row tiles (UNIT = 1) or
-// groups of UNIT consecutive 128-row tiles of the same expert (the last unit
-// of an expert may hold fewer).  s_unit_start[e] = first unit of expert e.
-template <int UNIT>
-__device__ __forceinline__ int64_t rows_units(const Params& p, const int32_t* s_unit_start) {
-  if constexpr (UNIT == 1) return used_rows(p) / BM;
-  return s_unit_start[p.E];
-}
+// Number of M units for the ROWS schedule: groups of UNIT consecutive 128-row
+// tiles of the same expert (the last unit of an expert may hold fewer).
+// s_unit_start[e] = first unit of expert e; s_unit_start[E] = all units.
+__device__ __forceinline__ int64_t rows_units(const int32_t* s_unit_start, int E) { return s_unit_start[E]; }
 
 template <int SCHED, int BN, int UNIT, int EPI>
 __device__ __forceinline__ int64_t total_tiles(const Params& p, const int32_t* s_unit_start) {
   if constexpr (SCHED == SCHED_ROWS) {
-    return rows_units<UNIT>(p, s_unit_start) * p.n_tiles;
+    return rows_units(s_unit_start, p.E) * p.n_tiles;
   } else if constexpr (SCHED == SCHED_WGRAD) {
     return (int64_t)p.E * p.m_tiles_w * p.n_tiles;
   } else {
@@ -154,32 +145,34 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int64_t t, const int32
   constexpr int NOUT = (EPI == EPI_SWIGLU || EPI == EPI_WGRAD_PAIR) ? BN / 2 : BN;
   Tile tl;
   if constexpr (SCHED == SCHED_ROWS) {
-    const int64_t num_m = rows_units<UNIT>(p, s_unit_start);
-    const int64_t per_group = (int64_t)p.group_m * p.n_tiles;
-    const int64_t g = t / per_group;
-    const int64_t first_m = g * p.group_m;
-    const int64_t gm = (num_m - first_m) < p.group_m ? (num_m - first_m) : p.group_m;
-    const int64_t local = t - g * per_group;
-    const int64_t mu = first_m + local % gm;          // M unit
-    const int64_t nt = local / gm;
-    if constexpr (UNIT == 1) {
-      tl.row0 = mu * BM;
-      tl.e = expert_of_row(p.padded_bins, p.E, tl.row0);
-      tl.halves = 1;
-    } else {
-      // expert = last e with s_unit_start[e] <= mu
-      int lo = 0, hi = p.E - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if ((int64_t)s_unit_start[mid] <= mu) lo = mid; else hi = mid - 1;
-      }
-      tl.e = lo;
-      const int64_t pstart = tl.e ? p.padded_bins[tl.e - 1] : 0;
-      const int64_t ntile_e = (p.padded_bins[tl.e] - pstart) / BM;
-      const int64_t k = mu - s_unit_start[tl.e];
-      tl.row0 = pstart + k * UNIT * BM;
-      tl.halves = (int)((ntile_e - UNIT * k) >= UNIT ? UNIT : (ntile_e - UNIT * k));
+    // Raster aligned to experts: expert e owns tiles [s_unit_start[e] * n,
+    // s_unit_start[e + 1] * n) of the n column tiles; its units are cut into
+    // nearly equal groups of at most group_m, and a group's tiles run
+    // unit-fastest, so each weight column panel serves all the group's units
+    // back to back and no group mixes two experts' weights (on B200 this
+    // takes GEMM1's DRAM traffic from 1.52x to 1.06x its algorithmic bytes).
+    const int64_t n = p.n_tiles;
+    int lo = 0, hi = p.E - 1;
+    while (lo < hi) {                                  // last e owning tiles <= t
+      const int mid = (lo + hi + 1) >> 1;
+      if ((int64_t)s_unit_start[mid] * n <= t) lo = mid; else hi = mid - 1;
     }
+    tl.e = lo;
+    const int64_t units_e = s_unit_start[lo + 1] - s_unit_start[lo];
+    const int64_t local = t - (int64_t)s_unit_start[lo] * n;
+    const int64_t nch = (units_e + p.group_m - 1) / p.group_m;   // groups of the expert
+    const int64_t cs = (units_e + nch - 1) / nch;                // units per group (last: fewer)
+    const int64_t c = local / (cs * n);
+    const int64_t gm = (c == nch - 1) ? units_e - cs * (nch - 1) : cs;
+    const int64_t lg = local - c * cs * n;
+    const int64_t k = c * cs + lg % gm;                          // unit within the expert
+    const int64_t nt = lg / gm;
+    const int64_t pstart = tl.e ? p.padded_bins[tl.e - 1] : 0;
+    int64_t pend = p.padded_bins[tl.e];
+    if (pend > p.P) pend = p.P;
+    const int64_t ntile_e = pend > pstart ? (pend - pstart) / BM : 0;
+    tl.row0 = pstart + k * UNIT * BM;
+    tl.halves = (int)((ntile_e - UNIT * k) >= UNIT ? UNIT : (ntile_e - UNIT * k));
     tl.m0 = 0;
     tl.n0 = (int)(nt * NOUT);
     tl.nkb = p.kdim / BK;
@@ -615,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     fence_barrier_init();
     fence_proxy_async();
   }
-  if (SCHED == SCHED_ROWS && UNIT > 1 && warp == 2) {
+  if (SCHED == SCHED_ROWS && warp == 2) {
     // units per expert = ceil(tiles_e / UNIT); exclusive scan over experts
     int carry = 0;
     for (int e0 = 0; e0 < p.E; e0 += 32) {
@@ -1062,7 +1055,7 @@ template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int 
 static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upper, cudaStream_t s) {
   using S = Shape<BN, MT, CG>;
   Params p = p_in;
-  if (p.group_m <= 0) p.group_m = S::UNIT >= 4 ? (kGroupM * 2) / S::UNIT : kGroupM;
+  if (p.group_m <= 0) p.group_m = kGroupM;
   auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA>;
   constexpr size_t scratch = scratch_bytes<EPI>() ? (size_t)kEpiWarps * scratch_bytes<EPI>() + 512 : 0;
   static_assert(S::SMEM + scratch <= 232448, "shared memory per CTA");
