@@ -102,6 +102,11 @@ BWD_SMALL = [
     small_shape("bf16_bwd", N=640, H=256, E=8, K=2, F=256, training=True),
     small_shape("bf16_bwd_e64", N=900, H=256, E=64, K=4, F=384, training=True),
     small_shape("bf16_bwd_h128", N=400, H=128, E=16, K=4, F=128, training=True),
+    # every token to both experts, so each expert holds N rows: more than 8
+    # row units, and the grouped GEMMs' raster cuts an expert into several
+    # groups (H=384: 128-row units in GEMM2 and the dgrad to x)
+    small_shape("bf16_bwd_big_experts", N=2500, H=256, E=2, K=2, F=256, training=True),
+    small_shape("bf16_bwd_big_h384", N=1500, H=384, E=2, K=2, F=256, training=True),
 ]
 
 

@@ -147,7 +147,10 @@ GROUPED = [("f32", 128, 256, 4, [200, 0, 37, 300]),
            ("bf16", 128, 256, 4, [130, 0, 1, 400]),
            ("bf16", 256, 384, 8, [0, 0, 129, 255, 256, 1, 0, 700]),
            ("bf16", 384, 1408, 3, [257, 64, 640]),
-           ("bf16", 512, 512, 2, [0, 1000])]
+           ("bf16", 512, 512, 2, [0, 1000]),
+           # experts of more than 8 row units: several raster groups per expert
+           ("bf16", 256, 256, 3, [2700, 0, 4500]),
+           ("bf16", 384, 256, 2, [1300, 2100])]
 
 
 @pytest.mark.parametrize("dtype,H,F,E,counts", GROUPED)
