@@ -42,7 +42,8 @@ using namespace umma;
 
 constexpr int kRows = 128;                 // tokens per row tile
 constexpr int kRBK = 64;                   // k block (one 128-byte swizzle row of bf16)
-constexpr int kRouteThreads = 192;
+constexpr int kRouteThreads = 192;       // router weight gradient
+constexpr int kRouteRowThreads = 256;    // router: 2 (S = 1) to 16 (S = 8) threads per routed row
 constexpr int kA = kRows * kRBK * 2;       // A bytes per stage
 constexpr uint64_t kRouteTimeoutNs = 2000000000ull;
 constexpr int kRouteSlots = 148;           // SMs the split aims to fill (fixed: results must not depend on the GPU)
@@ -88,11 +89,11 @@ __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
 // Insert (v, id) into a descending list of the K largest; a strict '>' keeps
 // an earlier, lower id above an equal value, so ties go to the lower id when
 // ids arrive in increasing order.
-template <int KMAX>
+template <int KMAX, bool EXACT = false>
 __device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals)[KMAX], int (&ids)[KMAX]) {
 #pragma unroll
   for (int j = KMAX - 1; j >= 0; --j) {
-    if (j < K && v > vals[j]) {
+    if ((EXACT || j < K) && v > vals[j]) {
       if (j > 0 && v > vals[j - 1]) {
         vals[j] = vals[j - 1];
         ids[j] = ids[j - 1];
@@ -104,8 +105,40 @@ __device__ __forceinline__ void topk_insert(float v, int id, int K, float (&vals
   }
 }
 
+// Top-K of one routed row over experts [e0, e1) of its logits in shared
+// memory (`mine`), merged across the TPR threads of the row (consecutive
+// lanes): each thread keeps the sorted list of its own expert range, then
+// the lists fold pairwise towards the row's first thread, the higher-id
+// partner's list inserted into the lower one's in its sorted order.  With
+// strict '>' insertion an equal value stays behind every element already in
+// the list, and the lower thread holds the lower ids, so the result equals
+// one pass over all experts in increasing id order (ties to the lower id).
+template <int KMAX, bool EXACT>
+__device__ __forceinline__ void row_topk(const float* mine, int e0, int e1, int K, int TPR, int lane,
+                                         float (&vals)[KMAX], int (&ids)[KMAX]) {
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
+#pragma unroll 4
+  for (int e = e0; e < e1; ++e) topk_insert<KMAX, EXACT>(mine[e], e, K, vals, ids);
+  const int sub = lane % TPR;
+  for (int d = 1; d < TPR; d <<= 1) {
+    float ov[KMAX];
+    int oi[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      ov[j] = __shfl_down_sync(0xffffffffu, vals[j], d);
+      oi[j] = __shfl_down_sync(0xffffffffu, ids[j], d);
+    }
+    if (sub % (2 * d) == 0) {
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (EXACT || j < K) topk_insert<KMAX, EXACT>(ov[j], oi[j], K, vals, ids);
+    }
+  }
+}
+
 template <int EPT, bool B_MN, int KMAX>
-__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_constant__ RouteParams p) {
+__global__ void __launch_bounds__(kRouteRowThreads, 1) route_kernel(const __grid_constant__ RouteParams p) {
   using S_ = RouteShape<EPT>;
   constexpr int STAGES = S_::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -119,7 +152,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * S_::STAGE + 8 * (2 * STAGES + 1));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* s_hist = reinterpret_cast<int*>(tmem_holder + 4);    // [256] expert counts of this CTA's rows
-  const uint32_t part = base;                                 // S = 1: partial logits, after the main loop
+  const uint32_t part = base;                                 // the (partial) logits, after the main loop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t S = cluster_nctarank();
@@ -205,15 +238,14 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
       if (ok) mma_commit(tfull);
       else *abort_flag = 1;
     }
-  } else {
-    // --------------------------------- TMEM -> partial logits (smem or global)
+  } else if (warp < 6) {
+    // --------------------------------- TMEM -> (partial) logits in shared memory
     int ok = 0;
     if (lane == 0) ok = mbar_wait_bounded(tfull, 0, abort_flag, p.status, kRouteTimeoutNs) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     tc_fence_after();
     const int qd = warp & 3;                       // TMEM lane quarter of this warp
     const int row = qd * 32 + lane;
-    const int64_t t = (int64_t)row0 + row;
     const uint32_t dst = part + (uint32_t)(row * S_::STRIDE) * 4u;
 #pragma unroll
     for (int c = 0; c < EPT; ++c) {
@@ -226,68 +258,95 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const __grid_co
 #pragma unroll
         for (int j = 0; j < 32; ++j) r[j] = 0u;
       }
-      if (S == 1) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) st_shared_f32(dst + (uint32_t)(c * 32 + j) * 4u, __uint_as_float(r[j]));
-      } else if (t < p.N) {
-        // n_mma is a multiple of 16: whole 16-column halves of the chunk
-        float4* g = reinterpret_cast<float4*>(p.part + ((size_t)rank * p.N + t) * p.n_mma + c * 32);
-        const int nv = (p.n_mma - c * 32) >= 32 ? 8 : 4;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < nv)
-            g[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                               __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-      }
+      for (int j = 0; j < 32; ++j) st_shared_f32(dst + (uint32_t)(c * 32 + j) * 4u, __uint_as_float(r[j]));
     }
   }
   tc_fence_before();
-  if (S > 1) cluster_sync();     // every CTA's partial logits published (release / acquire, cluster scope)
-  else __syncthreads();
+  __syncthreads();               // this CTA's (partial) logits of its 128 rows are in shared memory
+  if (S > 1) {
+    // publish the rows other CTAs of the cluster finish: this CTA's partial
+    // [rank][N][n_mma] block, coalesced 16-byte stores; its own rows stay here
+    const int vpr = p.n_mma / 4;
+    const float* rb = reinterpret_cast<const float*>(gbase);
+    for (int v = (int)threadIdx.x; v < kRows * vpr; v += (int)blockDim.x) {
+      const int row = v / vpr, c = (v % vpr) * 4;
+      const int64_t t = (int64_t)row0 + row;
+      if (row / (kRows / (int)S) != (int)rank && t < p.N) {
+        const float* src = rb + row * S_::STRIDE + c;
+        *reinterpret_cast<float4*>(p.part + ((size_t)rank * p.N + t) * p.n_mma + c) =
+            make_float4(src[0], src[1], src[2], src[3]);
+      }
+    }
+    cluster_sync();              // every CTA's partials published (release / acquire, cluster scope)
+  }
   tc_fence_after();
 
   // ------------------------------------------------ rows: partials -> routing
-  // One thread per row: CTA r finishes rows [r*R, (r+1)*R), R = 128 / S.
-  // Pass 1 sums the row's partial logits (over s = 0..S-1 in order), keeps the
-  // running max and the sorted top-K list; the probabilities, when wanted,
-  // take two more passes over the summed row, kept in this CTA's own shared
-  // memory row (S = 1: in place; S > 1 the pipeline buffers are free).
+  // CTA r finishes rows [r*R, (r+1)*R), R = 128 / S.  With S > 1 all threads
+  // first sum the rows' partial logits (over s = 0..S-1 in order, coalesced)
+  // into this CTA's shared-memory rows (the pipeline buffers are free); with
+  // S = 1 the logits are there already.  Then TPR = blockDim / R threads per
+  // row select its top K (row_topk) and the row's first thread finishes it.
   const int rows_per = kRows / (int)S;
-  if ((int)threadIdx.x < rows_per) {
-    const int row = (int)rank * rows_per + (int)threadIdx.x;
-    const int64_t t = (int64_t)row0 + row;
-    if (t < p.N) {
-      float* mine = reinterpret_cast<float*>(gbase) + row * S_::STRIDE;
-      float vals[KMAX];
-      int ids[KMAX];
+  float* const rowbuf = reinterpret_cast<float*>(gbase);
+  if (S > 1) {
+    // this CTA's rows of partial s are one contiguous [rows][n_mma] block;
+    // 16-byte loads, four per thread in flight per partial; its own partial
+    // (s = rank) is read from shared memory, the sum kept in the order s = 0..S-1
+    const int cols = p.n_mma;                              // a multiple of 16
+    const int64_t first = (int64_t)row0 + (int64_t)rank * rows_per;
+    const int64_t left = p.N - first;
+    const int nrows = left < rows_per ? (left > 0 ? (int)left : 0) : rows_per;
+    const int vpr = cols / 4, nvec = nrows * vpr;
+    for (int v0 = (int)threadIdx.x; v0 < nvec; v0 += 4 * (int)blockDim.x) {
+      float4 acc[4];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) { vals[j] = -INFINITY; ids[j] = 0; }
-
-#pragma unroll 1
-      for (int c = 0; c < p.E; c += 32) {
-        float v[32];
-        if (S == 1) {
+      for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (uint32_t s = 0; s < S; ++s) {
+        const float4* src = reinterpret_cast<const float4*>(p.part + ((size_t)s * p.N + first) * cols);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = mine[c + j];
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.f;
-          for (uint32_t s = 0; s < S; ++s) {
-            const float* src = p.part + ((size_t)s * p.N + t) * p.n_mma + c;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c + j < p.n_mma) v[j] += src[j];
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (c + j < p.E) {
-            if (S > 1 && p.probs) mine[c + j] = v[j];
-            topk_insert<KMAX>(v[j], c + j, p.K, vals, ids);
-            if (p.logits) p.logits[t * p.E + c + j] = v[j];
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * (int)blockDim.x;
+          if (v < nvec) {
+            float4 x;
+            if (s == rank) {
+              const float* o = rowbuf + ((int)rank * rows_per + v / vpr) * S_::STRIDE + (v % vpr) * 4;
+              x = make_float4(o[0], o[1], o[2], o[3]);
+            } else {
+              x = src[v];
+            }
+            acc[u].x += x.x; acc[u].y += x.y; acc[u].z += x.z; acc[u].w += x.w;
           }
         }
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * (int)blockDim.x;
+        if (v < nvec) {
+          float* dst = rowbuf + ((int)rank * rows_per + v / vpr) * S_::STRIDE + (v % vpr) * 4;
+          dst[0] = acc[u].x; dst[1] = acc[u].y; dst[2] = acc[u].z; dst[3] = acc[u].w;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  {
+    const int TPR = (int)blockDim.x / rows_per;            // 2, 4, 8 or 16: divides 32
+    const int row = (int)rank * rows_per + (int)threadIdx.x / TPR;
+    const int sub = (int)threadIdx.x % TPR;
+    const int64_t t = (int64_t)row0 + row;
+    const float* mine = rowbuf + row * S_::STRIDE;
+    const int span = (p.E + TPR - 1) / TPR;
+    const int e0 = t < p.N ? (sub * span < p.E ? sub * span : p.E) : 0;
+    const int e1 = t < p.N ? ((sub + 1) * span < p.E ? (sub + 1) * span : p.E) : 0;
+    float vals[KMAX];
+    int ids[KMAX];
+    if (p.K == KMAX) row_topk<KMAX, true>(mine, e0, e1, p.K, TPR, lane, vals, ids);
+    else row_topk<KMAX, false>(mine, e0, e1, p.K, TPR, lane, vals, ids);
+    if (p.logits)
+      for (int e = e0; e < e1; ++e) p.logits[t * p.E + e] = mine[e];
+    if (t < p.N && sub == 0) {
       const float m = vals[0];   // the row's largest logit
       if (p.probs) {
         float Z = 0.f;
@@ -379,7 +438,7 @@ moe_status launch_route(const RouteParams& p, int S, int tiles, cudaStream_t s) 
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(tiles * S), 1, 1);
-  cfg.blockDim = dim3(kRouteThreads, 1, 1);
+  cfg.blockDim = dim3(kRouteRowThreads, 1, 1);
   cfg.dynamicSmemBytes = S_::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -462,10 +521,12 @@ moe_status route_umma(const void* x, const void* W_r, int N, int H, int E, int K
   p.status = status;
   const int tiles = (int)cdiv(N, kRows);
   const int S = route_split(N, H, E, K);
-#define MOE_ROUTE_K(EPT_, MN_)                                                 \
-  return K <= 8 ? launch_route<EPT_, MN_, 8>(p, S, tiles, s)                  \
-                : (K <= 16 ? launch_route<EPT_, MN_, 16>(p, S, tiles, s)      \
-                           : launch_route<EPT_, MN_, 32>(p, S, tiles, s))
+#define MOE_ROUTE_K(EPT_, MN_)                                                               \
+  return K <= 2 ? launch_route<EPT_, MN_, 2>(p, S, tiles, s)                                 \
+                : K <= 4 ? launch_route<EPT_, MN_, 4>(p, S, tiles, s)                        \
+                         : K <= 8 ? launch_route<EPT_, MN_, 8>(p, S, tiles, s)               \
+                                  : (K <= 16 ? launch_route<EPT_, MN_, 16>(p, S, tiles, s)   \
+                                             : launch_route<EPT_, MN_, 32>(p, S, tiles, s))
   switch (ept * 2 + (mn ? 1 : 0)) {
     case 3: MOE_ROUTE_K(1, true);
     case 2: MOE_ROUTE_K(1, false);
