@@ -488,14 +488,17 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
 // lone unit (an M = 128 pair MMA, see the kernel) CTA r's half feeds the TMEM
 // lanes 64r.. of both CTAs, so with SPLIT_N each CTA takes 64 columns of W1
 // and the same 64 of W3, keeping a gate and its up projection in one lane.
+// slab: bytes between the 64-wide MN slabs of an MN-major B in shared memory
+// (8 KB: one 64-deep k block per box; 16 KB: 128-deep boxes, see the kernel).
 template <int BN, int CG, int SCHED, bool B_MN, int SPLIT>
 __device__ __forceinline__ void load_b(const Params& p, const Tile& tl, uint32_t sb, uint32_t fb,
-                                       uint32_t rank, int k, const CUtensorMap* tb, bool lone = false) {
+                                       uint32_t rank, int k, const CUtensorMap* tb, bool lone = false,
+                                       uint32_t slab = 8192) {
   if constexpr (CG == 2) {
     if constexpr (SCHED == SCHED_ROWS && B_MN && SPLIT == SPLIT_N && BN == 256) {
       if (lone) {   // one 64-column box of W1 and the same of W3 per CTA
         tma_load_3d_pair(sb, &p.tb0, fb, tl.n0 + 64 * (int)rank, k, tl.e);
-        tma_load_3d_pair(sb + 8192, &p.tb1, fb, tl.n0 + 64 * (int)rank, k, tl.e);
+        tma_load_3d_pair(sb + slab, &p.tb1, fb, tl.n0 + 64 * (int)rank, k, tl.e);
         return;
       }
     }
@@ -503,17 +506,17 @@ __device__ __forceinline__ void load_b(const Params& p, const Tile& tl, uint32_t
 #pragma unroll
       for (int j = 0; j < BN / 128; ++j) {
         if (SPLIT == SPLIT_N)
-          tma_load_2d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k);
+          tma_load_2d_pair(sb + j * slab, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k);
         else
-          tma_load_2d_pair(sb + j * 8192, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k);
+          tma_load_2d_pair(sb + j * slab, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k);
       }
     } else if constexpr (B_MN) {
 #pragma unroll
       for (int j = 0; j < BN / 128; ++j) {
         if (SPLIT == SPLIT_N)
-          tma_load_3d_pair(sb + j * 8192, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k, tl.e);
+          tma_load_3d_pair(sb + j * slab, rank ? &p.tb1 : &p.tb0, fb, tl.n0 + 64 * j, k, tl.e);
         else
-          tma_load_3d_pair(sb + j * 8192, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k, tl.e);
+          tma_load_3d_pair(sb + j * slab, tb, fb, tl.n0 + (BN / 2) * (int)rank + 64 * j, k, tl.e);
       }
     } else {
       tma_load_3d_pair(sb, tb, fb, k, tl.n0 + (BN / 2) * (int)rank, tl.e);
@@ -550,10 +553,22 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   using S = Shape<BN, MT, CG>;
   constexpr int STAGES = S::STAGES;
   constexpr int STAGE_BYTES = S::STAGE_BYTES;
-  constexpr int SUB_BYTES = S::SUB_BYTES;
   constexpr int KSUB = S::KSUB;
+  // Stage layout: the A tiles of the stage's KSUB k blocks, then their B
+  // tiles.  A K-major operand is one box per k block.  An MN-major operand of
+  // a two-k-block stage (CTA pairs) comes as one 128-deep box per 64-wide MN
+  // slab, the slab's two k blocks back to back (16 KB slabs, WSLAB apart):
+  // half the TMA operations of 64-deep boxes, which the single producer
+  // thread issues one by one.
+  constexpr bool WIDE = KSUB == 2 && MT == 1;
+  constexpr bool A_WIDE = WIDE && A_MN;
+  constexpr bool B_WIDE = WIDE && B_MN;
+  constexpr uint32_t WSLAB = 2 * 8192;
   constexpr int A_BYTES = S::A_BYTES;
   constexpr int B_BYTES = S::B_BYTES;
+  constexpr int A_REG = KSUB * A_BYTES;                 // bytes of a stage's A tiles
+  static_assert(!WIDE || (!A_MN && !B_MN) || (A_BYTES == 2 * 8192 && B_BYTES == 2 * 8192),
+                "wide boxes: two 64-wide MN slabs per operand");
   constexpr int ACC_BUFS = S::ACC_BUFS;
   constexpr int ACC_COLS = S::ACC_COLS;
   constexpr int UNIT = S::UNIT;
@@ -673,9 +688,10 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           return j < cnt ? p.g_indices[bstart + j] / p.g_K : p.g_N;
         };
         const int n_mma_h = PAIR ? (tl.halves + 1) / 2 : tl.halves;
-        uint32_t tx;
-        if constexpr (PAIR) tx = 2u * (uint32_t)(n_mma_h * BM * BK * 2 + B_BYTES);
-        else tx = (uint32_t)tl.halves * BM * BK * 2 + (uint32_t)B_BYTES;
+        // bytes landing per k block (A, B) and per stage (wide boxes bring
+        // both k blocks of a stage whatever nsub is)
+        const uint32_t txa = (PAIR ? 2u : 1u) * (uint32_t)((PAIR ? n_mma_h : tl.halves) * BM * BK * 2);
+        const uint32_t txb = (PAIR ? 2u : 1u) * (uint32_t)B_BYTES;
         int tk[MT][4];      // ROWS: this lane's four tokens of each half
         int nx[4];          // WGRAD: this lane's four tokens of the next k block
         if constexpr (SCHED == SCHED_ROWS) {
@@ -700,20 +716,31 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
           if (!w_ok) { ok = false; break; }
           const uint32_t fb = PAIR ? map_to_rank(full_bar(stage), 0) : full_bar(stage);
-          if (lane == 0 && (!PAIR || rank == 0)) mbar_expect_tx(full_bar(stage), tx * (uint32_t)nsub);
+          if (lane == 0 && (!PAIR || rank == 0))
+            mbar_expect_tx(full_bar(stage), txa * (uint32_t)(A_WIDE ? KSUB : nsub) + txb * (uint32_t)(B_WIDE ? KSUB : nsub));
+          const uint32_t st0 = base + stage * STAGE_BYTES;
           for (int j = 0; j < nsub; ++j) {
             const int kb = kb0 + j;
-            const uint32_t sa = base + stage * STAGE_BYTES + j * SUB_BYTES;
-            const uint32_t sb = sa + A_BYTES;
+            const uint32_t sa = st0 + j * A_BYTES;               // K-major A of k block j
+            const uint32_t sb = st0 + A_REG + j * B_BYTES;       // K-major B of k block j
             const int kc = SCHED == SCHED_WGRAD ? (int)(tl.row0 + (int64_t)kb * BK) : kb * BK;
-            if (lane == 0) load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, kc, &p.tb0, LONE && tl.halves == 1);
+            if (lane == 0) {
+              if constexpr (B_WIDE) {
+                if (j == 0) load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, st0 + A_REG, fb, rank, kc, &p.tb0,
+                                                               LONE && tl.halves == 1, WSLAB);
+              } else {
+                load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, kc, &p.tb0, LONE && tl.halves == 1);
+              }
+            }
             if constexpr (SCHED == SCHED_WGRAD) {
               int cur[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) cur[i] = nx[i];
               for (int h = 0; h < n_mma_h; ++h) {
                 const int hh = PAIR ? 2 * h + (int)rank : h;
-                const uint32_t dst = sa + h * (BM * BK * 2) + jb * 8192 + g * 512;
+                // MN-major A gathered k row by k row: slab jb, rows 4g.. of k block j
+                const uint32_t dst = A_WIDE ? st0 + jb * WSLAB + j * 8192 + g * 512
+                                            : sa + h * (BM * BK * 2) + jb * 8192 + g * 512;
                 const int m = tl.m0 + BM * hh + 64 * jb;
                 if constexpr (PAIR) tma_gather4_pair(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
                 else tma_gather4(dst, &p.ta0, fb, m, cur[0], cur[1], cur[2], cur[3]);
@@ -749,28 +776,42 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
         // MMAs of this tile: with a pair, MMA h covers tiles 2h and 2h+1 of the
         // unit (one per CTA) and runs when tile 2h exists
         const int n_mma_h = PAIR ? (tl.halves + 1) / 2 : tl.halves;
-        uint32_t tx;
-        if constexpr (PAIR) tx = 2u * (uint32_t)(n_mma_h * BM * BK * 2 + B_BYTES);   // both CTAs' loads
-        else tx = (uint32_t)tl.halves * BM * BK * 2 +
-                  (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)B_BYTES);
+        // bytes landing per k block (A, B; a pair counts both CTAs' loads)
+        const uint32_t txa = PAIR ? 2u * (uint32_t)(n_mma_h * BM * BK * 2) : (uint32_t)tl.halves * BM * BK * 2;
+        const uint32_t txb = PAIR ? 2u * (uint32_t)B_BYTES
+                                  : (SCHED == SCHED_DENSE ? (uint32_t)p.n_mma * BK * 2 : (uint32_t)B_BYTES);
         for (int kb0 = 0; kb0 < tl.nkb; kb0 += KSUB) {
           const int nsub = (tl.nkb - kb0) < KSUB ? (tl.nkb - kb0) : KSUB;
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status, kTimeoutNs)) { ok = false; break; }
           const uint32_t fb = PAIR ? map_to_rank(full_bar(stage), 0) : full_bar(stage);   // the leader's barrier
-          if (!PAIR || rank == 0) mbar_expect_tx(full_bar(stage), tx * (uint32_t)nsub);
+          if (!PAIR || rank == 0)
+            mbar_expect_tx(full_bar(stage), txa * (uint32_t)(A_WIDE ? KSUB : nsub) + txb * (uint32_t)(B_WIDE ? KSUB : nsub));
+          const uint32_t st0 = base + stage * STAGE_BYTES;
           for (int j = 0; j < nsub; ++j) {
             const int kb = kb0 + j;
-            const uint32_t sa = base + stage * STAGE_BYTES + j * SUB_BYTES;
-            const uint32_t sb = sa + A_BYTES;
+            const uint32_t sa = st0 + j * A_BYTES;               // K-major A of k block j
+            const uint32_t sb = st0 + A_REG + j * B_BYTES;       // K-major B of k block j
             if constexpr (PAIR) {
               if constexpr (SCHED == SCHED_WGRAD) {
                 const int krow = (int)(tl.row0 + (int64_t)kb * BK);
-                for (int h = 0; h < n_mma_h; ++h) {
-                  const int m = tl.m0 + BM * (2 * h + (int)rank);
-                  tma_load_2d_pair(sa + h * (BM * BK * 2), &p.ta0, fb, m, krow);
-                  tma_load_2d_pair(sa + h * (BM * BK * 2) + 8192, &p.ta0, fb, m + 64, krow);
+                if constexpr (A_WIDE) {
+                  if (j == 0) {          // both k blocks of the stage, one 128-deep box per slab
+                    const int m = tl.m0 + BM * (int)rank;
+                    tma_load_2d_pair(st0, &p.ta0, fb, m, krow);
+                    tma_load_2d_pair(st0 + WSLAB, &p.ta0, fb, m + 64, krow);
+                  }
+                } else {
+                  for (int h = 0; h < n_mma_h; ++h) {
+                    const int m = tl.m0 + BM * (2 * h + (int)rank);
+                    tma_load_2d_pair(sa + h * (BM * BK * 2), &p.ta0, fb, m, krow);
+                    tma_load_2d_pair(sa + h * (BM * BK * 2) + 8192, &p.ta0, fb, m + 64, krow);
+                  }
                 }
-                load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, krow, &p.tb0);
+                if constexpr (B_WIDE) {
+                  if (j == 0) load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, st0 + A_REG, fb, rank, krow, &p.tb0, false, WSLAB);
+                } else {
+                  load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, krow, &p.tb0);
+                }
               } else {
                 int k = kb * BK;
                 const CUtensorMap* ta = &p.ta0;
@@ -780,7 +821,11 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
                 for (int h = 0; h < n_mma_h; ++h)
                   tma_load_2d_pair(sa + h * (BM * BK * 2), ta, fb, k,
                                    (int)tl.row0 + (lone ? 64 * (int)rank : BM * (2 * h + (int)rank)));
-                load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, k, tb, lone);
+                if constexpr (B_WIDE) {
+                  if (j == 0) load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, st0 + A_REG, fb, rank, k, tb, lone, WSLAB);
+                } else {
+                  load_b<BN, CG, SCHED, B_MN, SPLIT>(p, tl, sb, fb, rank, k, tb, lone);
+                }
               }
             } else {
               if constexpr (SCHED == SCHED_WGRAD) {
@@ -834,18 +879,21 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
 #pragma unroll
           for (int j = 0; j < KSUB; ++j) {
             if (j < nsub) {
-              const uint32_t sa = base + stage * STAGE_BYTES + j * SUB_BYTES;
-              const uint32_t sb = sa + A_BYTES;
+              const uint32_t st0 = base + stage * STAGE_BYTES;
+              const uint32_t sa = st0 + j * A_BYTES;
+              const uint32_t sb = st0 + A_REG + j * B_BYTES;
 #pragma unroll
               for (int kk = 0; kk < BK / 16; ++kk) {
-                const uint64_t bd = B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32);
+                const uint64_t bd = B_WIDE ? desc_mn_sw128(st0 + A_REG + j * 8192 + kk * 2048, WSLAB)
+                                           : (B_MN ? desc_mn_sw128(sb + kk * 2048, 8192) : desc_k_sw128(sb + kk * 32));
                 const uint32_t accum = ((kb0 + j) | kk) != 0 ? 1u : 0u;
                 if constexpr (PAIR) {
 #pragma unroll
                   for (int h = 0; h < MT; ++h) {
                     if (2 * h < tl.halves) {
                       const uint32_t ah = sa + h * (BM * BK * 2);
-                      const uint64_t ad = A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32);
+                      const uint64_t ad = A_WIDE ? desc_mn_sw128(st0 + j * 8192 + kk * 2048, WSLAB)
+                                                 : (A_MN ? desc_mn_sw128(ah + kk * 2048, 8192) : desc_k_sw128(ah + kk * 32));
                       mma_bf16_pair(d_tmem + h * BN, ad, bd, idesc, accum);
                     }
                   }
@@ -1155,7 +1203,8 @@ moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const 
   typedef __nv_bfloat16 bf;
   Params p = blank_params(pb, E, P, status);
   const bool a_ok = ga ? map2d(&p.ta0, ga->x, H, ga->N, H, 64, 1) : map2d(&p.ta0, x_perm, H, P, H, 64, 128);
-  if (!a_ok || !map3d(&p.tb0, W1, F, H, E, 64, 64) || !map3d(&p.tb1, W3, F, H, E, 64, 64))
+  // CTA pairs read MN-major operands in 128-deep boxes (two k blocks, see the kernel)
+  if (!a_ok || !map3d(&p.tb0, W1, F, H, E, 64, 128) || !map3d(&p.tb1, W3, F, H, E, 64, 128))
     return MOE_ERR_CUDA;
   if (ga) set_gather(&p, ga);
   if ((act && !map_out2d(&p.to0, act, F, P, F)) || (G && !map_out2d(&p.to1, G, F, P, F)) ||
@@ -1239,7 +1288,8 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     Params p = blank_params(pb, E, P, status);
     const int bn = (H % 256 == 0) ? 256 : 128;
     const int unit = (bn == 256 && F % 256 == 0) ? 2 : 1;
-    if (!map2d(&p.ta0, act, F, P, F, 64, 64) || !map2d(&p.tb0, d_out, H, P, H, 64, 64)) return MOE_ERR_CUDA;
+    const uint32_t kbox = unit == 2 && pref ? 128 : 64;   // CTA pairs: 128-deep MN-major boxes
+    if (!map2d(&p.ta0, act, F, P, F, 64, kbox) || !map2d(&p.tb0, d_out, H, P, H, 64, kbox)) return MOE_ERR_CUDA;
     p.n_mma = bn;
     p.m_tiles_w = F / (BM * unit);
     p.n_tiles = H / bn;
@@ -1257,8 +1307,9 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
   {
     Params p = blank_params(pb, E, P, status);
     const int unit = (H % 256 == 0) ? 2 : 1;
-    const bool a_ok = ga ? map2d(&p.ta0, ga->x, H, ga->N, H, 64, 1) : map2d(&p.ta0, x_perm, H, P, H, 64, 64);
-    if (!a_ok || !map2d(&p.tb0, dG, F, P, F, 64, 64) || !map2d(&p.tb1, dU, F, P, F, 64, 64))
+    const uint32_t kbox = unit == 2 && (pref || ga) ? 128 : 64;   // CTA pairs: 128-deep MN-major boxes
+    const bool a_ok = ga ? map2d(&p.ta0, ga->x, H, ga->N, H, 64, 1) : map2d(&p.ta0, x_perm, H, P, H, 64, kbox);
+    if (!a_ok || !map2d(&p.tb0, dG, F, P, F, 64, kbox) || !map2d(&p.tb1, dU, F, P, F, 64, kbox))
       return MOE_ERR_CUDA;
     if (ga) set_gather(&p, ga);
     p.n_mma = 256;
