@@ -47,8 +47,11 @@ namespace umma {
 
 constexpr int BM = 128;
 constexpr int BK = 64;              // one 128-byte swizzle row of bf16
-constexpr int kEpiWarps = 8;              // two warps per TMEM lane quarter
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+// Epilogue warps per CTA: 8 (two per TMEM lane quarter, splitting the
+// columns), or 16 for the single-CTA 256-row plain-store GEMMs, whose one
+// accumulator set keeps the epilogue off the main loop's critical path only
+// if it drains fast (four warps per lane quarter, one scratch buffer each)
+constexpr int kEpiWarps = 8;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 // Most M units per raster group (groups never span two experts, see
 // get_tile): 8 units of up to 256 rows, so an expert of up to 2048 rows streams
@@ -344,18 +347,19 @@ __device__ __forceinline__ void rows_from_coalesced(uint32_t scratch, int lane, 
 
 // Epilogue of one 128-row half: TMEM columns [tacc, tacc + BN) of this
 // thread's row -> fused math -> global memory (store_mode<EPI>).  scratch:
-// this warp's scratch_bytes<EPI>() bytes of shared memory; nb: the warp's next
-// TMA-store buffer, carried across calls.
-template <int BN, int SCHED, int EPI>
+// this warp's shared memory (scratch_bytes<EPI>(), or one buffer when NPART
+// is 4); nb: the warp's next TMA-store buffer, carried across calls.
+template <int BN, int SCHED, int EPI, int NPART = 2>
 __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, uint32_t tacc, int row,
                                               int part, uint32_t scratch, int& nb) {
   const int64_t grow = tl.row0 + row;                 // ROWS/DENSE global row
   const int lane = row & 31;
   const int64_t row_base = grow - lane;               // the warp's first row (ROWS/DENSE)
   const int yb = (int)row_base;
-  // the two warps of a lane quarter split the columns: part 0 / part 1
+  // the NPART warps of a lane quarter split the columns
   constexpr int NC = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
-  const int c_begin = part * (NC / 2), c_end = c_begin + NC / 2;
+  static_assert((NC / NPART) % 32 == 0, "whole 32-column chunks per warp");
+  const int c_begin = part * (NC / NPART), c_end = c_begin + NC / NPART;
   if constexpr (EPI == EPI_SWIGLU) {
     // out0 = act (NULL when only G and U are wanted: backward recompute)
 #pragma unroll 1
@@ -375,6 +379,26 @@ __device__ __forceinline__ void epilogue_half(const Params& p, const Tile& tl, u
       if (p.out1) {
         store_chunk_tma(scratch, nb, lane, &p.to1, tl.n0 + c, yb, gf);
         store_chunk_tma(scratch, nb, lane, &p.to2, tl.n0 + c, yb, uf);
+      }
+    }
+  } else if constexpr (EPI == EPI_STORE && NPART == 4) {
+    // one scratch buffer: a chunk per round, the previous store read first
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32(tacc + c, r);
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      tmem_ld_wait();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      stage_chunk(scratch, lane, v);
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&p.to0, scratch, tl.n0 + c, yb);
+        bulk_commit();
       }
     }
   } else if constexpr (EPI == EPI_STORE) {
@@ -548,8 +572,8 @@ __device__ __forceinline__ void load_b(const Params& p, const Tile& tl, uint32_t
   }
 }
 
-template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT, bool GA>
-__global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
+template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT, bool GA, int EW>
+__global__ void __launch_bounds__(64 + 32 * EW, 1) umma_gemm_kernel(const __grid_constant__ Params p) {
   using S = Shape<BN, MT, CG>;
   constexpr int STAGES = S::STAGES;
   constexpr int STAGE_BYTES = S::STAGE_BYTES;
@@ -602,7 +626,9 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
   int32_t* s_unit_start = reinterpret_cast<int32_t*>(tmem_holder + 4);   // [E + 1]
   // scratch_bytes<EPI>() per epilogue warp, 512-byte aligned (the 64-byte
   // swizzle of the TMA stores repeats every 512 bytes)
-  constexpr int kScratch = scratch_bytes<EPI>();
+  static_assert(EW == kEpiWarps || (EW == 16 && CG == 1 && MT == 2 && EPI == EPI_STORE),
+                "16 epilogue warps: single-CTA 256-row plain stores");
+  constexpr int kScratch = EW == 16 ? kStoreBuf : scratch_bytes<EPI>();
   const uint32_t store_scratch = (smem_u32(s_unit_start + 260) + 511u) & ~511u;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -613,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int a = 0; a < ACC_BUFS; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), PAIR ? 2 * kEpiWarps : kEpiWarps);
+      mbar_init(tempty_bar(a), PAIR ? 2 * EW : EW);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -997,7 +1023,7 @@ __global__ void __launch_bounds__(kThreads, 1) umma_gemm_kernel(const __grid_con
           const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS + h * BN);
           Tile th = tl;
           if (SCHED == SCHED_WGRAD) th.m0 = tl.m0 + h * BM; else th.row0 = tl.row0 + h * BM;
-          epilogue_half<BN, SCHED, EPI>(p, th, tacc, row, part,
+          epilogue_half<BN, SCHED, EPI, EW / 4>(p, th, tacc, row, part,
                                         kScratch ? store_scratch + (warp - 2) * kScratch : 0u, nb);
         }
       }
@@ -1099,13 +1125,15 @@ static int sm_count() {
   return cache[dev];
 }
 
-template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT, bool GA = false>
+template <int BN, int MT, int CG, int SCHED, int EPI, bool A_MN, bool B_MN, int SPLIT, bool GA = false,
+          int EW = kEpiWarps>
 static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upper, cudaStream_t s) {
   using S = Shape<BN, MT, CG>;
   Params p = p_in;
   if (p.group_m <= 0) p.group_m = kGroupM;
-  auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA>;
-  constexpr size_t scratch = scratch_bytes<EPI>() ? (size_t)kEpiWarps * scratch_bytes<EPI>() + 512 : 0;
+  auto kern = umma_gemm_kernel<BN, MT, CG, SCHED, EPI, A_MN, B_MN, SPLIT, GA, EW>;
+  constexpr size_t per_warp = EW == 16 ? kStoreBuf : scratch_bytes<EPI>();
+  constexpr size_t scratch = per_warp ? (size_t)EW * per_warp + 512 : 0;
   static_assert(S::SMEM + scratch <= 232448, "shared memory per CTA");
   const size_t smem = S::SMEM + scratch;
   // once per device: later calls (a CUDA graph capture among them) only launch
@@ -1122,7 +1150,7 @@ static moe_status launch(const char* name, const Params& p_in, int64_t tiles_upp
   }
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(64 + 32 * EW, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1244,7 +1272,7 @@ moe_status grouped_swiglu_umma(const void* x_perm, const void* W1, const void* W
     p.out0 = (bf*)out;
     p.ldo = H;
     const int64_t up = (P / BM) * p.n_tiles;
-    if (bn == 256) return launch<256, 2, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
+    if (bn == 256) return launch<256, 2, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE, false, 16>("gemm2", p, up, s);
     return launch<128, 1, 1, SCHED_ROWS, EPI_STORE, false, true, SPLIT_NONE>("gemm2", p, up, s);
   }
 }
@@ -1345,7 +1373,7 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.ldo = H;
     const int64_t up = (P / BM) * p.n_tiles;
     st = pair ? launch<256, 1, 2, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s)
-         : bn == 256 ? launch<256, 2, 1, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s)
+         : bn == 256 ? launch<256, 2, 1, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K, false, 16>("dgrad_x", p, up, s)
                      : launch<128, 1, 1, SCHED_ROWS, EPI_STORE, false, false, SPLIT_K>("dgrad_x", p, up, s);
     if (st != MOE_OK) return st;
   }
