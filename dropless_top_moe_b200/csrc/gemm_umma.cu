@@ -984,7 +984,10 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1) umma_gemm_kernel(const __grid
         }
       }
       int ok = 0;
-      if (lane == 0) ok = mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag, p.status, kTimeoutNs) ? 1 : 0;
+      // a wait that spans the tile's main loop: sleep between polls (measured
+      // 1-2.5 % faster per GEMM in the power-capped step: the clock gains
+      // more than the up to 256 ns a late wake-up costs)
+      if (lane == 0) ok = mbar_wait_bounded_sleep(tfull_bar(acc), acc_phase, abort_flag, p.status, kTimeoutNs) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();

@@ -59,6 +59,25 @@ __device__ __forceinline__ void fence_proxy_async() {
 // Wait until phase `parity` of the barrier completes, or give up after
 // `timeout_ns` (then set *abort_flag and the status bit) or when another role
 // has already given up.  A correct pipeline never comes near the limit.
+// The same, sleeping 256 ns between polls: for waits that usually last a whole
+// main loop (fewer issue slots and less power spent polling).
+__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                        int* status, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(256);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > timeout_ns) {
+        *abort_flag = 1;
+        if (status) atomicOr(status, MOE_DEVERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort_flag, int* status,
                                                   uint64_t timeout_ns) {
