@@ -32,6 +32,11 @@ ROUTE_SHAPES = [
     small_shape("r_split8_e64", N=1000, H=4096, E=64, K=6),
     small_shape("r_split4_e256", N=700, H=1024, E=256, K=8, skew="normal", skew_param=1.0),
     small_shape("r_split2_e40_k12", N=6000, H=1024, E=40, K=12),
+    # the largest top-K lists (K up to 32), merged over 2 (S = 1), 8 (S = 4)
+    # and 16 (S = 8) threads per row
+    small_shape("r_bf16_e64_k32", N=500, H=256, E=64, K=32),
+    small_shape("r_split4_e256_k20", N=600, H=1024, E=256, K=20, skew="normal", skew_param=1.0),
+    small_shape("r_split8_e64_k32", N=300, H=4096, E=64, K=32),
 ]
 
 
