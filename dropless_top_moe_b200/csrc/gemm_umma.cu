@@ -9,15 +9,17 @@
 // MegaBlocks grouped path copies them to the host; MoonEP sec. 02 argues for
 // static shapes without host sync).
 //
-// One CTA (or one CTA pair, cta_group::2) per SM, 10 warps:
+// One CTA (or one CTA pair, cta_group::2) per SM, 10 warps (18 in the
+// single-CTA 256-row plain-store GEMMs, whose epilogue has 16 warps):
 //   warp 0      producer: A and B tiles by TMA into a STAGES-deep smem ring,
-//               one 64-deep k block per stage (two for a CTA pair)
+//               one 64-deep k block per stage (two for a CTA pair, whose
+//               MN-major operands come in 128-deep boxes)
 //               (optionally A rows gathered from x with tile::gather4)
 //   warp 1      TMEM allocator and MMA issuer (one thread): tcgen05.mma per
 //               16-deep k step, fp32 accumulators in TMEM, double-buffered
 //               where two accumulator sets fit so the epilogue of tile i
 //               overlaps the main loop of tile i+1
-//   warps 2..9  epilogue, two warps per TMEM lane quarter: tcgen05.ld rows ->
+//   warps 2..   epilogue, two (four) warps per TMEM lane quarter: tcgen05.ld rows ->
 //               registers -> fused math -> global, 32 x 32 chunks through
 //               a per-warp shared-memory scratch (TMA stores, or coalesced
 //               64-byte row segments for the weight gradients)
