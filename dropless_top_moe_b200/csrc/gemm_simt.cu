@@ -9,14 +9,17 @@
 //             reachable by strides; epilogues: plain store, SwiGLU forward,
 //             SwiGLU backward.
 // wgrad mode  C_e[m, n] = sum over the group's rows r of A[r, m] * B[r, n]
-// Accumulation is fp32 in increasing k: deterministic.
+// Accumulation is fp32 in increasing k: deterministic.  The next k slice is
+// loaded into registers while the current one is multiplied from shared
+// memory (small layers are latency-bound: one global round trip per slice).
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace moe {
 
 constexpr int kSB = 64;   // block tile (rows and columns)
-constexpr int kSK = 16;   // k slice
+constexpr int kSK = 32;   // k slice
+constexpr int kSL = kSB * kSK / 256;   // elements of a slice each thread loads, per operand
 
 enum SimtEpi { SIMT_STORE = 0, SIMT_SWIGLU = 1, SIMT_SWIGLU_BWD = 2, SIMT_DUAL = 3 };
 
@@ -42,42 +45,55 @@ gemm_rows_simt_kernel(const T* __restrict__ A0, const T* __restrict__ A1, int64_
     for (int j = 0; j < 4; ++j) { acc[i][j] = 0.f; acc2[i][j] = 0.f; }
 
   const int passes = (EPI == SIMT_DUAL) ? 2 : 1;
-  for (int pass = 0; pass < passes; ++pass) {
+  const int nsl = (Kd + kSK - 1) / kSK, total = passes * nsl;
+  float ra[kSL], rb[kSL], rb2[(EPI == SIMT_SWIGLU) ? kSL : 1];
+  // slice sl: pass sl / nsl (SIMT_DUAL's second A, B pair), k from (sl % nsl) * kSK
+  auto fetch = [&](int sl) {
+    const int pass = sl / nsl, k0 = (sl % nsl) * kSK;
     const T* A = pass ? A1 : A0;
     const T* B = pass ? B1 : B0;
-    for (int k0 = 0; k0 < Kd; k0 += kSK) {
-      for (int q = threadIdx.x; q < kSB * kSK; q += 256) {
-        const int r = q / kSK, kk = q % kSK;
-        const int k = k0 + kk;
-        As[kk][r] = (k < Kd) ? to_f<T>(A[(row0 + r) * lda + k]) : 0.f;
-        const int c = q % kSB, kb = q / kSB;
-        const int kb_k = k0 + kb;
-        const int64_t boff = (int64_t)e * sBe + (int64_t)kb_k * sBk + (int64_t)(n0 + c) * sBn;
-        const bool ok = kb_k < Kd && n0 + c < Nd;
-        Bs[kb][c] = ok ? to_f<T>(B[boff]) : 0.f;
-        if (EPI == SIMT_SWIGLU) Bs2[kb][c] = ok ? to_f<T>(B1[boff]) : 0.f;
+#pragma unroll
+    for (int l = 0; l < kSL; ++l) {
+      const int q = (int)threadIdx.x + l * 256;
+      const int r = q / kSK, k = k0 + q % kSK;
+      ra[l] = (k < Kd) ? to_f<T>(A[(row0 + r) * lda + k]) : 0.f;
+      const int c = q % kSB, kb_k = k0 + q / kSB;
+      const int64_t boff = (int64_t)e * sBe + (int64_t)kb_k * sBk + (int64_t)(n0 + c) * sBn;
+      const bool ok = kb_k < Kd && n0 + c < Nd;
+      rb[l] = ok ? to_f<T>(B[boff]) : 0.f;
+      if (EPI == SIMT_SWIGLU) rb2[l] = ok ? to_f<T>(B1[boff]) : 0.f;
+    }
+  };
+  fetch(0);
+  for (int sl = 0; sl < total; ++sl) {
+#pragma unroll
+    for (int l = 0; l < kSL; ++l) {
+      const int q = (int)threadIdx.x + l * 256;
+      As[q % kSK][q / kSK] = ra[l];
+      Bs[q / kSB][q % kSB] = rb[l];
+      if (EPI == SIMT_SWIGLU) Bs2[q / kSB][q % kSB] = rb2[l];
+    }
+    __syncthreads();
+    if (sl + 1 < total) fetch(sl + 1);
+#pragma unroll
+    for (int kk = 0; kk < kSK; ++kk) {
+      float a[4], b[4], b2[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        b[j] = Bs[kk][tx * 4 + j];
+        if (EPI == SIMT_SWIGLU) b2[j] = Bs2[kk][tx * 4 + j];
       }
-      __syncthreads();
 #pragma unroll
-      for (int kk = 0; kk < kSK; ++kk) {
-        float a[4], b[4], b2[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          b[j] = Bs[kk][tx * 4 + j];
-          if (EPI == SIMT_SWIGLU) b2[j] = Bs2[kk][tx * 4 + j];
+          acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+          if (EPI == SIMT_SWIGLU) acc2[i][j] = fmaf(a[i], b2[j], acc2[i][j]);
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-            if (EPI == SIMT_SWIGLU) acc2[i][j] = fmaf(a[i], b2[j], acc2[i][j]);
-          }
-      }
-      __syncthreads();
     }
+    __syncthreads();
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -121,14 +137,27 @@ gemm_wgrad_simt_kernel(const T* __restrict__ A, int64_t lda, const T* __restrict
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  float ra[kSL], rb[kSL];
+  auto fetch = [&](int64_t r0) {
+#pragma unroll
+    for (int l = 0; l < kSL; ++l) {
+      const int q = (int)threadIdx.x + l * 256;
+      const int c = q % kSB;
+      const int64_t r = r0 + q / kSB;
+      ra[l] = (r < r_end && m0 + c < Md) ? to_f<T>(A[r * lda + m0 + c]) : 0.f;
+      rb[l] = (r < r_end && n0 + c < Nd) ? to_f<T>(B[r * ldb + n0 + c]) : 0.f;
+    }
+  };
+  if (r_begin < r_end) fetch(r_begin);
   for (int64_t r0 = r_begin; r0 < r_end; r0 += kSK) {
-    for (int q = threadIdx.x; q < kSB * kSK; q += 256) {
-      const int c = q % kSB, kk = q / kSB;
-      const int64_t r = r0 + kk;
-      As[kk][c] = (r < r_end && m0 + c < Md) ? to_f<T>(A[r * lda + m0 + c]) : 0.f;
-      Bs[kk][c] = (r < r_end && n0 + c < Nd) ? to_f<T>(B[r * ldb + n0 + c]) : 0.f;
+#pragma unroll
+    for (int l = 0; l < kSL; ++l) {
+      const int q = (int)threadIdx.x + l * 256;
+      As[q / kSB][q % kSB] = ra[l];
+      Bs[q / kSB][q % kSB] = rb[l];
     }
     __syncthreads();
+    if (r0 + kSK < r_end) fetch(r0 + kSK);
 #pragma unroll
     for (int kk = 0; kk < kSK; ++kk) {
       float a[4], b[4];
