@@ -744,8 +744,10 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1) umma_gemm_kernel(const __grid
           w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
           if (!w_ok) { ok = false; break; }
           const uint32_t fb = PAIR ? map_to_rank(full_bar(stage), 0) : full_bar(stage);
+          // A arrives gathered, k block by k block (nsub of them); a wide B box
+          // brings both k blocks of the stage
           if (lane == 0 && (!PAIR || rank == 0))
-            mbar_expect_tx(full_bar(stage), txa * (uint32_t)(A_WIDE ? KSUB : nsub) + txb * (uint32_t)(B_WIDE ? KSUB : nsub));
+            mbar_expect_tx(full_bar(stage), txa * (uint32_t)nsub + txb * (uint32_t)(B_WIDE ? KSUB : nsub));
           const uint32_t st0 = base + stage * STAGE_BYTES;
           for (int j = 0; j < nsub; ++j) {
             const int kb = kb0 + j;
