@@ -422,8 +422,18 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
   const int64_t P = p_max(N, E, K);
   const RowGather ga = {x, indices, bins, N, K};
   const uint32_t stamp = (uint32_t)layer_stamp_byte(training, aux_alpha, capacity) * 0x01010101u;
-  MOE_TRACED("layer_flags_check", s, (layer_stamp_check_kernel<<<1, 32, 0, s>>>(w.status, (int)stamp)));
-  MOE_LAUNCH_CHECK();
+  // the sparse router backward walks the kept assignments only; the aux loss
+  // and dropped assignments need every (token, expert) logit: dense path
+  const bool dense_router = (aux_alpha != 0.0f || capacity > 0) && N > 0;
+  // First launch: the check of the forward's recorded flags; on the sparse
+  // router path it is fused into the W_r^T transpose that path needs.
+  const bool wrt_first = !dense_router && N > 0;
+  if (wrt_first) {
+    MOE_TRY(transpose_matrix(W_r, H, E, dt, w.ur_scratch, s, 0, w.status, (int)stamp));
+  } else {
+    MOE_TRACED("layer_flags_check", s, (layer_stamp_check_kernel<<<1, 32, 0, s>>>(w.status, (int)stamp)));
+    MOE_LAUNCH_CHECK();
+  }
   const bool gather = (training & MOE_LAYER_GATHER_ROWS) != 0;
   training &= 3;
   void* gate_up = w.gate_up;
@@ -442,7 +452,6 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
   }
   // the sparse router backward of a bf16 layer takes x^T D on the tensor
   // cores; the combine backward writes D (bf16) beside the dlogits
-  const bool dense_router = (aux_alpha != 0.0f || capacity > 0) && N > 0;
   void* Dh = (!dense_router && dt == MOE_BF16 && router_wgrad_tc_supported(H, E))
                  ? unpermute_router_bwd_dh(w.ur_scratch, N, H, E, P)
                  : nullptr;
@@ -450,9 +459,8 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
                            w.dlogit, w.d_out, s, top_experts, Dh));
   MOE_TRY(swiglu_bwd_any(w.d_out, w.x_perm, w.act, gate_up, W1, W3, W2, padded_bins, E, H, F, P, dt,
                          w.d_gate_up, dW1, dW3, dW2, w.dx_perm, w.status, s, gather ? &ga : nullptr));
-  // the sparse router backward walks the kept assignments only; the aux loss
-  // and dropped assignments need every (token, expert) logit: dense path
-  // (the router probabilities exist only when the forward computed the loss)
+  // dense path: the router probabilities exist only when the forward
+  // computed the loss
   if (dense_router)
     MOE_TRY(dense_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, w.routed_bins,
                              aux_alpha != 0.0f ? w.probs : nullptr, N, H, E, K, dt, aux_alpha, aux_grad, dx,
@@ -460,7 +468,7 @@ moe_status moe_layer_bwd(const void* dy, const void* x, const void* W_r, const v
   else
     MOE_TRY(unpermute_router_bwd(w.dx_perm, w.dlogit, x, W_r, top_experts, w.pos, indices, bins,
                                  padded_bins, N, H, E, K, P, dt, dx, dW_r, w.ur_scratch, w.status, s,
-                                 Dh != nullptr));
+                                 Dh != nullptr, wrt_first));
   return MOE_OK;
 }
 

@@ -53,17 +53,22 @@ moe_status combine_bwd_rows(const void* dy, const void* out, const float* w, con
                             const int32_t* bins, const int32_t* pb, int N, int K, int H, int E,
                             moe_dtype dt, float* dw, float* dlogit, void* d_out, cudaStream_t s,
                             const int32_t* top = nullptr, void* Dh = nullptr);
+// status != NULL: the same launch checks the layer forward's recorded flags
+// (status[1]) against `expect` and sets MOE_DEVERR_MODE on a mismatch.
 moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s,
-                            int C_pad = 0);
+                            int C_pad = 0, int* status = nullptr, int expect = 0);
 size_t unpermute_router_bwd_scratch(int N, int H, int E, int64_t P);
-// Where, inside that scratch, the bf16 D [N, E] of the tensor-core router
-// weight gradient lives (combine_bwd_rows can write it there: dh_ready).
+// W_r^T sits at its start (the layer backward makes it in its first launch:
+// wrt_ready); where, inside that scratch, the bf16 D [N, E] of the
+// tensor-core router weight gradient lives (combine_bwd_rows can write it
+// there: dh_ready).
 void* unpermute_router_bwd_dh(void* scratch, int N, int H, int E, int64_t P);
 moe_status unpermute_router_bwd(const void* dx_perm, const float* dlogit, const void* x,
                                 const void* W_r, const int32_t* top, const int32_t* pos,
                                 const int32_t* indices, const int32_t* bins, const int32_t* padded_bins,
                                 int N, int H, int E, int K, int64_t P, moe_dtype dt, void* dx,
-                                void* dWr, void* scratch, int* status, cudaStream_t s, bool dh_ready = false);
+                                void* dWr, void* scratch, int* status, cudaStream_t s, bool dh_ready = false,
+                                bool wrt_ready = false);
 
 // aux.cu - load-balancing loss and the dense router backward it needs
 size_t aux_loss_scratch(int N, int E);

@@ -226,8 +226,13 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ out, const fl
 
 // outT[c][r] = in[r][c] for c < C, and 0 for C <= c < C_pad (zero rows that
 // pad a transposed operand to an MMA width), through a shared-memory tile.
+// status != NULL: the layer backward's first launch also checks the flags the
+// forward recorded (status[1]) against `expect`, setting MOE_DEVERR_MODE.
 template <typename T>
-__global__ void transpose_kernel(const T* __restrict__ in, int R, int C, int C_pad, T* __restrict__ outT) {
+__global__ void transpose_kernel(const T* __restrict__ in, int R, int C, int C_pad, T* __restrict__ outT,
+                                 int* status, int expect) {
+  if (status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0 && status[1] != expect)
+    atomicOr(status, MOE_DEVERR_MODE);
   __shared__ T tile[32][33];
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
@@ -454,15 +459,15 @@ moe_status combine_bwd_rows(const void* dy, const void* out, const float* w, con
 }
 
 moe_status transpose_matrix(const void* in, int R, int C, moe_dtype dt, void* outT, cudaStream_t s,
-                            int C_pad) {
+                            int C_pad, int* status, int expect) {
   if (C_pad < C) C_pad = C;
   dim3 grid((unsigned)cdiv(C_pad, 32), (unsigned)cdiv(R, 32)), block(32, 8);
   if (dt == MOE_F32)
     MOE_TRACED("transpose", s, (transpose_kernel<float><<<grid, block, 0, s>>>((const float*)in, R, C, C_pad,
-                                                                                (float*)outT)));
+                                                                                (float*)outT, status, expect)));
   else
     MOE_TRACED("transpose", s, (transpose_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-                                   (const __nv_bfloat16*)in, R, C, C_pad, (__nv_bfloat16*)outT)));
+                                   (const __nv_bfloat16*)in, R, C, C_pad, (__nv_bfloat16*)outT, status, expect)));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -490,11 +495,14 @@ static moe_status unpermute_router_bwd_t(const void* dx_perm, const float* dlogi
                                          const int32_t* indices, const int32_t* bins,
                                          const int32_t* padded_bins, int N, int H, int E, int K,
                                          int64_t P, void* dx, void* dWr, void* scratch, int* status,
-                                         cudaStream_t s, bool dh_ready) {
+                                         cudaStream_t s, bool dh_ready, bool wrt_ready) {
   T* WrT = (T*)scratch;
   float* part = (float*)((char*)scratch + al256b((size_t)E * H * 4));
-  moe_status st = transpose_matrix(W_r, H, E, sizeof(T) == 4 ? MOE_F32 : MOE_BF16, WrT, s);
-  if (st != MOE_OK) return st;
+  moe_status st = MOE_OK;
+  if (!wrt_ready) {
+    st = transpose_matrix(W_r, H, E, sizeof(T) == 4 ? MOE_F32 : MOE_BF16, WrT, s);
+    if (st != MOE_OK) return st;
+  }
   MOE_TRACED("unpermute_dx", s, (unpermute_dx_kernel<T><<<row_grid(N), kRowThreads, 0, s>>>((const T*)dx_perm, dlogit, WrT, top, pos,
                                                              N, H, K, (T*)dx)));
   MOE_LAUNCH_CHECK();
@@ -539,13 +547,13 @@ moe_status unpermute_router_bwd(const void* dx_perm, const float* dlogit, const 
                                 const void* W_r, const int32_t* top, const int32_t* pos,
                                 const int32_t* indices, const int32_t* bins, const int32_t* padded_bins,
                                 int N, int H, int E, int K, int64_t P, moe_dtype dt, void* dx, void* dWr,
-                                void* scratch, int* status, cudaStream_t s, bool dh_ready) {
+                                void* scratch, int* status, cudaStream_t s, bool dh_ready, bool wrt_ready) {
   return dt == MOE_F32
              ? unpermute_router_bwd_t<float>(dx_perm, dlogit, x, W_r, top, pos, indices, bins, padded_bins, N, H,
-                                             E, K, P, dx, dWr, scratch, status, s, dh_ready)
+                                             E, K, P, dx, dWr, scratch, status, s, dh_ready, wrt_ready)
              : unpermute_router_bwd_t<__nv_bfloat16>(dx_perm, dlogit, x, W_r, top, pos, indices, bins,
                                                      padded_bins, N, H, E, K, P, dx, dWr, scratch, status, s,
-                                                     dh_ready);
+                                                     dh_ready, wrt_ready);
 }
 
 }  // namespace moe
