@@ -77,6 +77,9 @@ struct Params {
   int n_tiles;        // tiles along N
   int m_tiles_w;      // WGRAD: tiles along M
   int group_m;        // ROWS: M units per raster group
+  // ROWS: which experts the launch covers: 0 all, 1 those of two or more
+  // 128-row tiles, 2 those of exactly one (each then one unit; UNIT = 1)
+  int single_mode;
   // Gathered A (GA kernels): ta0 maps the token matrix [g_N, kdim or M] with
   // one-row boxes; padded row r of expert e holds token
   // g_indices[g_bins[e-1] + r - padded_bins[e-1]] / g_K, pad rows read zeros
@@ -663,6 +666,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1) umma_gemm_kernel(const __grid
         if (hi > p.P) hi = p.P;
         const int64_t tiles = hi > lo ? (hi - lo) / BM : 0;
         u = (int)((tiles + UNIT - 1) / UNIT);
+        if (p.single_mode == 1 && tiles == 1) u = 0;
+        else if (p.single_mode == 2) u = tiles == 1 ? 1 : 0;
       }
       int incl = u;
 #pragma unroll
@@ -1254,6 +1259,22 @@ moe_status gemm1_umma(const void* x_perm, const void* W1, const void* W3, const 
   p.ldo = F;
   const int64_t up = (P / BM) * p.n_tiles;
   if (ga) return launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N, true>(name, p, up, s);
+  // Many experts of a single 128-row tile (row buffer of at most 4 tiles per
+  // expert on average: fine-grained layers): a pair would run each of them as
+  // a lone unit, which costs about as much as a full one, so they go to a
+  // second, single-CTA launch (M = 128 per SM, no rows idle) and the pairs
+  // take the experts of two or more tiles.
+  if (P <= (int64_t)E * 4 * BM) {
+    p.single_mode = 1;
+    moe_status st = launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>(name, p, up, s);
+    if (st != MOE_OK) return st;
+    Params q = p;
+    q.single_mode = 2;
+    // single-CTA stages hold one k block: 64-deep weight boxes
+    if (!map3d(&q.tb0, W1, F, H, E, 64, 64) || !map3d(&q.tb1, W3, F, H, E, 64, 64)) return MOE_ERR_CUDA;
+    const int64_t uq = (int64_t)E * q.n_tiles;
+    return launch<256, 1, 1, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>("gemm1_swiglu_single", q, uq, s);
+  }
   return launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU, false, true, SPLIT_N>(name, p, up, s);
 }
 
@@ -1313,10 +1334,21 @@ moe_status grouped_swiglu_bwd_umma(const void* d_out, const void* x_perm, const 
     p.out1 = dU;
     p.ldo = F;
     const int64_t up = (P / BM) * p.n_tiles;
+    // as in GEMM1: with many one-tile experts those run on single CTAs
+    const bool split = pair && P <= (int64_t)E * 4 * BM;
+    if (split) p.single_mode = 1;
     st = pair ? launch<256, 1, 2, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s)
          : bn == 256 ? launch<256, 1, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s)
                      : launch<128, 1, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd", p, up, s);
     if (st != MOE_OK) return st;
+    if (split) {
+      Params q = p;
+      q.single_mode = 2;
+      if (!map3d(&q.tb0, W2, H, F, E, 64, bn)) return MOE_ERR_CUDA;   // a single CTA reads all BN rows
+      st = launch<256, 1, 1, SCHED_ROWS, EPI_SWIGLU_BWD, false, false, SPLIT_NONE>("dgrad_w2_swiglu_bwd_single", q,
+                                                                                 (int64_t)E * q.n_tiles, s);
+      if (st != MOE_OK) return st;
+    }
   }
   // dW2_e = act_e^T * d_out_e   [F, H]
   {

@@ -155,7 +155,10 @@ GROUPED = [("f32", 128, 256, 4, [200, 0, 37, 300]),
            ("bf16", 512, 512, 2, [0, 1000]),
            # experts of more than 8 row units: several raster groups per expert
            ("bf16", 256, 256, 3, [2700, 0, 4500]),
-           ("bf16", 384, 256, 2, [1300, 2100])]
+           ("bf16", 384, 256, 2, [1300, 2100]),
+           # mostly one-tile experts: GEMM1 splits into a pair launch and a
+           # single-CTA launch for the one-tile experts
+           ("bf16", 256, 256, 16, [100, 300, 5, 128, 129, 0, 60, 700, 1, 90, 256, 257, 40, 128, 77, 500])]
 
 
 @pytest.mark.parametrize("dtype,H,F,E,counts", GROUPED)
