@@ -25,7 +25,9 @@
 //               64-byte row segments for the weight gradients)
 // Tile shapes: BN output columns; MT 128-row tiles per CTA; CG = 2 pairs two
 // CTAs on one M = 256 MMA (each CTA holds its 128 rows and half of B's
-// columns); an expert's odd last tile runs as an M = 128 pair MMA.
+// columns); an expert's odd last tile runs as an M = 128 pair MMA, except
+// that experts of a single tile can be left to a second, single-CTA launch
+// (Params::single_mode) where many of them would each cost a pair unit.
 // Schedules
 //   ROWS   C[rows of group e, :] = A[rows, :] * B_e   (forward, dgrad)
 //   WGRAD  C_e = A[group e rows, :]^T * B[group e rows, :]   (weight grads;
