@@ -296,22 +296,30 @@ class Tracer:
         call("moe_trace_detach")
 
     def per_kernel(self):
-        """kernel name -> (total ms, launches) over the launches recorded.
-        GEMM1 and the SwiGLU-backward dgrad of a layer with many one-tile
-        experts run as two launches each (CTA pairs, then the one-tile experts
-        on single CTAs); their times are summed under the one kernel name
-        whose work model covers both."""
+        """kernel name -> (total ms, launches) over the launches recorded."""
         per = {}
         for i in range(min(self.count.value, self.cap)):
             name = self.labels[i].decode()
             d = self.evs[2 * i].elapsed_time(self.evs[2 * i + 1])
             tot, n = per.get(name, (0.0, 0))
             per[name] = (tot + d, n + 1)
-        for part, whole in (("gemm1_swiglu_single", "gemm1_swiglu"),
-                            ("dgrad_w2_swiglu_bwd_single", "dgrad_w2_swiglu_bwd")):
-            if part in per and whole in per:
-                per[whole] = (per[whole][0] + per.pop(part)[0], per[whole][1])
-        return per
+        return fold_split_launches(per)
+
+
+# GEMM1 and the SwiGLU-backward dgrad of a layer with many one-tile experts
+# run as two launches each (CTA pairs, then the one-tile experts on single
+# CTAs): second launch -> the kernel whose work model covers both.
+SPLIT_LAUNCHES = (("gemm1_swiglu_single", "gemm1_swiglu"),
+                  ("dgrad_w2_swiglu_bwd_single", "dgrad_w2_swiglu_bwd"))
+
+
+def fold_split_launches(per):
+    """Sum each second launch's time into its kernel, whose launch count
+    (one per step) the work model divides by."""
+    for part, whole in SPLIT_LAUNCHES:
+        if part in per and whole in per:
+            per[whole] = (per[whole][0] + per.pop(part)[0], per[whole][1])
+    return per
 
 
 def launches_per_step(step, tracer):

@@ -88,3 +88,17 @@ def test_recorded_traffic_only_for_the_captured_source_and_workload(tmp_path, mo
     assert bench.recorded_traffic("k_new", "train_step") == 1e9
     assert bench.recorded_traffic("k_old", "train_step") is None
     assert bench.recorded_traffic("k_list", "train_step") == 3e9
+
+
+def test_split_gemm_launches_fold_into_their_kernel():
+    sys.path.insert(0, ROOT)
+    import bench
+    per = {"gemm1_swiglu": (10.0, 5), "gemm1_swiglu_single": (2.5, 5), "gemm2": (4.0, 5),
+           "dgrad_w2_swiglu_bwd_single": (1.0, 5)}
+    out = bench.fold_split_launches(dict(per))
+    # time summed, launches of the main kernel kept (its work model is per step)
+    assert out["gemm1_swiglu"] == (12.5, 5)
+    assert "gemm1_swiglu_single" not in out
+    assert out["gemm2"] == (4.0, 5)
+    # a second launch without its main kernel is left alone
+    assert out["dgrad_w2_swiglu_bwd_single"] == (1.0, 5)
