@@ -113,7 +113,7 @@ def kernel_rooflines(per, steps, timed_ms, fl, by, peaks):
     algorithmic FLOPs / HBM bytes per launch.  Each kernel with a work model
     gets its achieved rate and the fraction of the roof it meets first: the
     sustained bf16 tensor peak or the HBM copy bandwidth (both measured; a
-    kernel with both models, the router, is judged by its arithmetic
+    kernel with both models, the router, is rated by its arithmetic
     intensity against the ridge; the dispatch metadata, a few hundred KB,
     is latency-bound and gets no fraction).  Stage totals: the grouped GEMMs against
     the tensor peak, the bandwidth-bound row kernels against HBM, and the

@@ -47,7 +47,7 @@ def test_kernel_rooflines_fractions_and_stage_totals():
     k, st = bench.kernel_rooflines(per, 2, 20.0, fl, by, peaks)
     assert k["gemm_a"]["tflops"] == 500.0 and k["gemm_a"]["bound"] == "tensor" and k["gemm_a"]["frac"] == 0.5
     assert k["gemm_b"]["frac"] == 1.0
-    # router: 10 FLOP per byte, below the ridge, so judged against HBM: 1e8 B in 50 us = 2000 GB/s
+    # router: 10 FLOP per byte, below the ridge, so rated against HBM: 1e8 B in 50 us = 2000 GB/s
     assert k["router"]["bound"] == "hbm" and k["router"]["gbs"] == 2000.0 and k["router"]["frac"] == 0.4
     assert k["rows"]["gbs"] == 5000.0 and k["rows"]["frac"] == 1.0
     assert "frac" not in k["other"] and k["other"]["share"] == 0.025
