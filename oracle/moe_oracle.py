@@ -214,11 +214,13 @@ def maxvio(hist, N: int, K: int, E: int) -> float:
 
 
 def permute(x, pos, K: int, P: int) -> np.ndarray:
-    """Padded gather: row pos[t*K+k] of the result is token t; pads stay 0."""
+    """Padded gather: row pos[t*K+k] of the result is token t; pads stay 0.
+    A dropped assignment (pos -1, token dropping) is not gathered."""
     xv = f64(x)
     out = np.zeros((P, xv.shape[1]), dtype=np.float64)
     for i, p in enumerate(np.asarray(pos).reshape(-1)):
-        out[p] = xv[i // K]
+        if p >= 0:
+            out[p] = xv[i // K]
     return out
 
 
@@ -259,14 +261,16 @@ def grouped_swiglu(x_perm, W1, W3, W2, padded_bins):
 
 
 def combine(O, weights, pos, N: int, K: int):
-    """y[t] = sum over k of weights[t,k] * O[pos[t*K+k]] (MegaBlocks sec. 2.1)."""
+    """y[t] = sum over k of weights[t,k] * O[pos[t*K+k]] (MegaBlocks sec. 2.1);
+    a dropped assignment (pos -1) adds nothing (icman sec. 3.4)."""
     Ov = np.asarray(O, np.float64)
     w = np.asarray(weights, np.float64)
     p = np.asarray(pos).reshape(N, K)
     y = np.zeros((N, Ov.shape[1]))
     for t in range(N):
         for k in range(K):
-            y[t] += w[t, k] * Ov[p[t, k]]
+            if p[t, k] >= 0:
+                y[t] += w[t, k] * Ov[p[t, k]]
     return y
 
 

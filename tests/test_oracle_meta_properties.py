@@ -56,3 +56,28 @@ def test_dispatch_meta_matches_sort_primitives(case):
     assert int(m["padded_bins"][-1]) <= om.padded_rows_max(N, E, K)
     # the kept mask is the same selection
     np.testing.assert_array_equal(om.kept_mask(te, E, capacity).reshape(-1), kept)
+
+
+@settings(max_examples=60, deadline=None)
+@given(routing(), st.integers(1, 5))
+def test_permute_then_combine_with_identity_experts(case, H):
+    """With every expert the identity, combine(permute(x)) gives each token
+    x_t times the sum of its kept routing weights: the whole of x_t when
+    nothing is dropped (the weights sum to 1), less when assignments are
+    dropped; pad rows and dropped assignments carry nothing."""
+    te, E, K, N, capacity = case
+    rng = np.random.default_rng(N * 31 + E)
+    x = rng.standard_normal((N, H))
+    w = rng.random((N, K)) + 0.1
+    w = w / w.sum(axis=1, keepdims=True)
+    m = om.dispatch_meta(te, E, capacity=capacity)
+    P = om.padded_rows_max(N, E, K)
+    xp = om.permute(x, m["pos"], K, P)
+    kept = om.kept_mask(te, E, capacity)
+    # every gathered row is its token's row; pad rows are zero
+    used = np.zeros(P, dtype=bool)
+    pos = m["pos"].reshape(N, K)
+    used[pos[kept]] = True
+    assert not np.any(xp[~used])
+    y = om.combine(xp, w, m["pos"], N, K)
+    np.testing.assert_allclose(y, x * (w * kept).sum(axis=1, keepdims=True), rtol=1e-12, atol=1e-12)
